@@ -1,0 +1,33 @@
+"""Plain float64 CPU oracle for the butterfly transform + low-bit quantization path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or link
+this package: only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` use it.  It shares
+no code with the CUDA library (no kernels, headers, tables or helpers); the only
+thing both sides consume is the seeded input generator module, which holds none
+of the method's arithmetic.
+
+What it computes, and where the method is stated:
+
+* ``butterfly``  - the orthogonal butterfly transform Q built from Givens
+  rotations with continuous angles (ButterflyQuant abstract, arXiv 2509.09679;
+  explainer article, section "butterfly"), its inverse Q^T, the Kronecker
+  composite B_m (x) O_r for widths that are not a power of two (explainer
+  article, section "butterfly", last paragraph), and the backward pass
+  (dX, dtheta) that gradient-based calibration needs (abstract: "enables smooth
+  optimization").
+* ``quant``      - per-group asymmetric round-to-nearest quantization with fp16
+  scale and zero point and little-endian INT2/INT4 packing (2-bit weights:
+  explainer article, section "training & results"; RTN block quantizer: WUSH
+  technical summary, section 2 "method").  The pages give no formula; the
+  readings taken are listed in the module docstring and in the design notes.
+
+Parity status: every function here is pinned by an independent check in
+``tests/test_oracle_pins.py`` (closed forms, the Hadamard special case against
+``scipy.linalg.hadamard``, explicit dense stage matrices, ``numpy.kron``, finite
+differences, brute-force quantizer search).  The stage order, Kronecker order,
+quantizer details and packing layout are conventions the pages leave open;
+those are pinned by convention plus self-consistency only.
+"""
+
+from . import butterfly, quant  # noqa: F401

@@ -1,0 +1,443 @@
+"""Pins of the float64 oracle against facts the pages and the mathematics fix.
+
+None of these checks re-types the oracle's own formulas: each compares it with
+an independent construction (explicit dense stage matrices, scipy's Sylvester
+Hadamard matrix, numpy.kron, central finite differences, exact rational
+arithmetic, hand-worked fixtures under tests/golden/).
+"""
+
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+from oracle import butterfly as bf
+from oracle import quant as oq
+from rotation_bit_quantization_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def rand_theta(m, seed):
+    return wl.uniform_angles(np.random.default_rng(seed), m)
+
+
+# ---------------------------------------------------------------- transform
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16, 64, 256])
+def test_orthogonal_by_construction(m):
+    # abstract: "guaranteeing orthogonality by construction"
+    Q = bf.dense_q(rand_theta(m, m), m)
+    assert np.abs(Q @ Q.T - np.eye(m)).max() < 1e-12
+    assert np.abs(Q.T @ Q - np.eye(m)).max() < 1e-12
+
+
+@pytest.mark.parametrize("m", [2, 8, 32, 128, 512])
+def test_stagewise_matches_dense_stage_product(m):
+    # two independent constructions of Q x: index-pair updates vs explicit matrices
+    th = rand_theta(m, 100 + m)
+    x = np.random.default_rng(m).standard_normal((5, m))
+    ref = x @ bf.dense_q(th, m).T
+    assert np.abs(bf.forward(th, x) - ref).max() < 1e-12 * np.abs(x).max() * m
+
+
+@pytest.mark.parametrize("m", [16, 1024])
+def test_norm_preservation_and_invariance(m):
+    # computational invariance y = Wx = (W Q^T)(Q x) (abstract)
+    th = rand_theta(m, 7)
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((4, m))
+    W = rng.standard_normal((6, m))
+    qx = bf.forward(th, x)
+    wq = bf.forward(th, W)             # rows of W Q^T are Q w_r
+    assert np.allclose(np.linalg.norm(qx, axis=1), np.linalg.norm(x, axis=1), rtol=1e-12, atol=0)
+    lhs = wq @ qx.T
+    rhs = W @ x.T
+    assert np.abs(lhs - rhs).max() <= 1e-12 * np.abs(W).sum(1).max() * np.abs(x).max()
+
+
+@pytest.mark.parametrize("m", [4, 64, 4096])
+def test_inverse_is_transpose(m):
+    th = rand_theta(m, 11)
+    x = np.random.default_rng(5).standard_normal((3, m))
+    back = bf.inverse(th, bf.forward(th, x))
+    assert np.linalg.norm(back - x) <= 1e-13 * np.linalg.norm(x)
+    if m <= 64:
+        Q = bf.dense_q(th, m)
+        inv_cols = bf.inverse(th, np.eye(m)).T      # column k = Q^T e_k
+        assert np.abs(inv_cols - Q.T).max() < 1e-13
+
+
+def test_parameter_count():
+    # abstract: n log n / 2 learnable parameters
+    assert bf.num_angles(256) == 1024
+    assert bf.num_angles(4096) == 24576
+    assert bf.num_angles(1024) == 5120
+    with pytest.raises(ValueError):
+        bf.num_stages(5120)
+
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16, 32, 64])
+def test_hadamard_special_case(m):
+    # explainer, section "butterfly": H_n is a butterfly with particular angles;
+    # abstract: Hadamard coherence mu = 1/sqrt(n).
+    th = np.full((bf.num_stages(m), m // 2), np.pi / 4, dtype=np.float32)
+    Q = bf.dense_q(th, m)
+    H = scipy.linalg.hadamard(m).astype(np.float64)
+    P = np.sqrt(m) * Q * H                      # must be the outer product 1 d^T, d in {+-1}
+    d = P[0]
+    assert np.allclose(np.abs(d), 1.0, atol=2e-7)
+    assert np.allclose(P, np.ones((m, 1)) * d[None, :], atol=2e-7)
+    assert np.allclose(np.abs(Q), 1 / np.sqrt(m), atol=2e-7)
+    # signs: the Kronecker power of (1, -1)
+    dk = np.array([1.0])
+    for _ in range(bf.num_stages(m)):
+        dk = np.kron(dk, np.array([1.0, -1.0]))
+    assert np.array_equal(np.sign(d), dk)
+
+
+def test_hadamard_golden_n4():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "hadamard_n4.txt")) if l.strip() and not l.startswith("#")]
+    G = np.array(rows, dtype=np.float64) / 2.0
+    th = np.full((2, 2), np.pi / 4, dtype=np.float32)
+    assert np.abs(bf.dense_q(th, 4) - G).max() < 1e-7
+
+
+@pytest.mark.parametrize("m", [8, 64, 256])
+def test_coherence_lower_bound(m):
+    # rows of an orthogonal matrix have unit norm, so max |Q_ij| >= 1/sqrt(n)
+    for seed in range(3):
+        Q = bf.dense_q(rand_theta(m, 1000 + seed), m)
+        assert np.abs(Q).max() >= 1 / np.sqrt(m) - 1e-15
+
+
+def test_zero_angles_identity():
+    m = 32
+    th = np.zeros((5, 16), dtype=np.float32)
+    x = np.random.default_rng(0).standard_normal((3, m))
+    assert np.array_equal(bf.forward(th, x), x)
+    assert np.array_equal(bf.dense_q(th, m), np.eye(m))
+
+
+def test_single_stage_rotation_matches_textbook_2x2():
+    # m = 2: Q is the plain Givens rotation [[c, -s], [s, c]]
+    t = np.float32(0.3)
+    th = np.array([[t]], dtype=np.float32)
+    c, s = np.cos(np.float64(t)), np.sin(np.float64(t))
+    assert np.allclose(bf.dense_q(th, 2), [[c, -s], [s, c]], atol=0, rtol=0)
+    y = bf.forward(th, np.array([[1.0, 0.0], [0.0, 1.0]]))
+    assert np.allclose(y, [[c, s], [-s, c]])
+
+
+@pytest.mark.parametrize("m,r", [(4, 3), (8, 5), (16, 2)])
+def test_kronecker_composite(m, r):
+    # explainer, section "butterfly": Kronecker-product composite for non-power-of-2 widths
+    th = rand_theta(m, 20 + r)
+    O = wl.random_orthogonal(np.random.default_rng(r), r).astype(np.float64)
+    x = np.random.default_rng(9).standard_normal((4, m * r))
+    K = np.kron(bf.dense_q(th, m), O)
+    assert np.abs(bf.kron_forward(th, O, x, m) - x @ K.T).max() < 1e-12
+    assert np.abs(bf.kron_inverse(th, O, x, m) - x @ K).max() < 1e-12
+    Of = O.astype(np.float32).astype(np.float64)
+    Kf = np.kron(bf.dense_q(th, m), Of)
+    assert np.abs(Kf @ Kf.T - np.eye(m * r)).max() < 1e-6     # O stored in float32
+
+
+# ---------------------------------------------------------------- backward
+
+def _loss(th, x, dy):
+    return float((bf.forward(th, x) * dy).sum())
+
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16])
+def test_backward_finite_differences(m):
+    L = bf.num_stages(m)
+    rng = np.random.default_rng(40 + m)
+    th = rng.uniform(-np.pi, np.pi, (L, m // 2))      # float64 angles for the FD check
+    x = rng.standard_normal((3, m))
+    dy = rng.standard_normal((3, m))
+    # the oracle casts angles to float32 first; use float32-representable angles
+    th = th.astype(np.float32)
+    _, dx, dth = bf.backward(th, x, dy)
+    h = 1e-6
+    fd = np.zeros_like(dth)
+    thd = th.astype(np.float64)
+    for s in range(L):
+        for p in range(m // 2):
+            tp = thd.copy(); tp[s, p] += h
+            tm = thd.copy(); tm[s, p] -= h
+            fd[s, p] = (_loss_f64(tp, x, dy) - _loss_f64(tm, x, dy)) / (2 * h)
+    assert np.abs(fd - dth).max() <= 1e-7 * max(1.0, np.abs(dth).max())
+    Q = bf.dense_q(th, m)
+    assert np.abs(dx - dy @ Q).max() < 1e-12
+
+
+def _loss_f64(th64, x, dy):
+    """Loss with float64 angles (stage matrices built from float64 cos/sin), for finite differences."""
+    m = x.shape[1]
+    v = x.copy()
+    for s in range(bf.num_stages(m)):
+        B = np.zeros((m, m))
+        half = 1 << s
+        for i in range(m):
+            if (i >> s) & 1:
+                continue
+            j = i + half
+            p = ((i >> (s + 1)) << s) | (i & (half - 1))
+            c, sn = np.cos(th64[s, p]), np.sin(th64[s, p])
+            B[i, i], B[i, j], B[j, i], B[j, j] = c, -sn, sn, c
+        v = v @ B.T
+    return float((v * dy).sum())
+
+
+def test_backward_zero_angles_closed_form():
+    # theta = 0: every stage is the identity, v = x, g = dy, so
+    # dtheta[s, p] = dy_j x_i - dy_i x_j for the pair (i, j) of stage s
+    m = 8
+    th = np.zeros((3, 4), dtype=np.float32)
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((1, m))
+    dy = np.zeros((1, m)); dy[0, 2] = 1.5; dy[0, 3] = -0.5
+    _, dx, dth = bf.backward(th, x, dy)
+    assert np.array_equal(dx, dy)
+    # stage 0 pair p=1 is (2, 3)
+    assert np.isclose(dth[0, 1], dy[0, 3] * x[0, 2] - dy[0, 2] * x[0, 3])
+    # stage 1: pairs (0,2),(1,3),(4,6),(5,7) -> p=0 is (0,2), p=1 is (1,3)
+    assert np.isclose(dth[1, 0], dy[0, 2] * x[0, 0] - dy[0, 0] * x[0, 2])
+    assert np.isclose(dth[1, 1], dy[0, 3] * x[0, 1] - dy[0, 1] * x[0, 3])
+    # stage 2: pairs (i, i+4): (2,6) is p=2 and (3,7) is p=3
+    assert np.isclose(dth[2, 2], dy[0, 6] * x[0, 2] - dy[0, 2] * x[0, 6])
+    assert np.isclose(dth[2, 3], dy[0, 7] * x[0, 3] - dy[0, 3] * x[0, 7])
+    assert dth[2, 0] == 0.0 and dth[0, 0] == 0.0
+
+
+def test_kron_backward_finite_differences():
+    m, r = 4, 3
+    L = 2
+    rng = np.random.default_rng(77)
+    th = rng.uniform(-np.pi, np.pi, (L, m // 2)).astype(np.float32)
+    O = wl.random_orthogonal(rng, r).astype(np.float64)
+    x = rng.standard_normal((2, m * r))
+    dy = rng.standard_normal((2, m * r))
+    y, dx, dth = bf.kron_backward(th, O, x, dy, m)
+    K = np.kron(bf.dense_q(th, m), O)
+    assert np.abs(y - x @ K.T).max() < 1e-12
+    assert np.abs(dx - dy @ K).max() < 1e-12
+    h = 1e-6
+    for s in range(L):
+        for p in range(m // 2):
+            tp = th.astype(np.float64); tp[s, p] += h
+            tm = th.astype(np.float64); tm[s, p] -= h
+            Kp = np.kron(_dense_f64(tp, m), O)
+            Km = np.kron(_dense_f64(tm, m), O)
+            fd = ((x @ Kp.T * dy).sum() - (x @ Km.T * dy).sum()) / (2 * h)
+            assert abs(fd - dth[s, p]) <= 1e-7 * max(1.0, abs(dth[s, p]))
+
+
+def _dense_f64(th64, m):
+    Q = np.eye(m)
+    for s in range(bf.num_stages(m)):
+        B = np.zeros((m, m))
+        half = 1 << s
+        for i in range(m):
+            if (i >> s) & 1:
+                continue
+            j = i + half
+            p = ((i >> (s + 1)) << s) | (i & (half - 1))
+            c, sn = np.cos(th64[s, p]), np.sin(th64[s, p])
+            B[i, i], B[i, j], B[j, i], B[j, j] = c, -sn, sn, c
+        Q = B @ Q
+    return Q
+
+
+def test_backward_abs_scale_bounds_dtheta():
+    m = 16
+    th = rand_theta(m, 3)
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((10, m)); dy = rng.standard_normal((10, m))
+    _, _, dth = bf.backward(th, x, dy)
+    A = bf.backward_abs_scale(th, x, dy)
+    assert np.all(np.abs(dth) <= A * (1 + 1e-12))
+
+
+# ---------------------------------------------------------------- quantizer
+
+def _golden_quant():
+    out = []
+    for line in open(os.path.join(GOLDEN, "quant_handcases.txt")):
+        if not line.strip() or line.startswith("#"):
+            continue
+        head, vals, codes, scale, zero = [p.strip() for p in line.split("|")]
+        bits, group = map(int, head.split())
+        out.append((bits, group, np.array(vals.split(), dtype=np.float32),
+                    np.array(codes.split(), dtype=np.uint8), float(scale), float(zero)))
+    return out
+
+
+@pytest.mark.parametrize("case", range(5))
+def test_quant_golden_handcases(case):
+    bits, group, vals, codes, scale, zero = _golden_quant()[case]
+    q, s16, z16 = oq.quantize_codes(vals[None, :], bits, group)
+    assert np.array_equal(q[0], codes)
+    assert s16.view(np.float16)[0, 0] == np.float16(scale)
+    assert z16.view(np.float16)[0, 0] == np.float16(zero)
+
+
+def _round_half_even(fr: Fraction) -> int:
+    fl = fr.numerator // fr.denominator
+    rem = fr - fl
+    if rem > Fraction(1, 2):
+        return fl + 1
+    if rem < Fraction(1, 2):
+        return fl
+    return fl if fl % 2 == 0 else fl + 1
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quant_matches_exact_rational_rounding(bits):
+    # exact rational x/s, rounded half to even, equals the float32-step code unless
+    # float32 x/s lies within an ulp of a tie (then either side is a valid reading)
+    rng = np.random.default_rng(bits)
+    qmax = 2 ** bits - 1
+    y = (rng.standard_normal((64, 32)) * rng.uniform(0.01, 10, (64, 1))).astype(np.float32)
+    q, s16, z16 = oq.quantize_codes(y, bits, 32)
+    s = s16.view(np.float16).astype(np.float32)
+    z = z16.view(np.float16).astype(np.float32)
+    checked = 0
+    for r in range(64):
+        sf = Fraction(float(s[r, 0]))
+        zf = int(z[r, 0])
+        for k in range(32):
+            t = Fraction(float(y[r, k])) / sf
+            ratio32 = np.float32(y[r, k]) / np.float32(s[r, 0])
+            frac = abs(float(t) - np.floor(float(t)) - 0.5)
+            if frac < 4 * np.spacing(np.float32(abs(ratio32)) + np.float32(1)):
+                continue
+            want = min(max(_round_half_even(t) + zf, 0), qmax)
+            assert q[r, k] == want
+            checked += 1
+    assert checked > 64 * 32 * 0.99
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_quant_error_bound_and_bruteforce(bits):
+    rng = np.random.default_rng(10 + bits)
+    qmax = 2 ** bits - 1
+    y = rng.standard_normal((50, 16)).astype(np.float32)
+    q, s16, z16 = oq.quantize_codes(y, bits, 16)
+    xh = oq.dequantize(q, s16, z16, 16)
+    s = s16.view(np.float16).astype(np.float32)
+    z = z16.view(np.float16).astype(np.float32)
+    for r in range(50):
+        for k in range(16):
+            # brute force: the code minimises |(q - z) s - x| over [0, qmax]
+            errs = [abs((c - float(z[r, 0])) * float(s[r, 0]) - float(y[r, k])) for c in range(qmax + 1)]
+            best = min(errs)
+            assert errs[q[r, k]] <= best + 1e-6 * float(s[r, 0])
+            if 0 < q[r, k] < qmax:
+                assert abs(xh[r, k] - y[r, k]) <= float(s[r, 0]) / 2 * (1 + 1e-6)
+    # scale is the fp16 rounding of (hi - lo) / qmax
+    lo = y.min(1); hi = y.max(1)
+    assert np.array_equal(s16[:, 0], (((hi - lo) / np.float32(qmax)).astype(np.float16)).view(np.uint16))
+
+
+def test_quant_degenerate_and_underflow():
+    y = np.full((1, 8), 2.5, dtype=np.float32)
+    q, s16, z16 = oq.quantize_codes(y, 4, 8)
+    assert s16.view(np.float16)[0, 0] == 1.0 and z16.view(np.float16)[0, 0] == 0.0
+    assert np.all(q == 2)          # z = clamp(rint(-2.5)) = 0; rint(2.5) = 2 (half to even)
+    # fp16 underflow of the scale: range 1e-9 -> scale32 ~ 7e-11 -> fp16 0 -> s = 1
+    y2 = np.array([[0.0, 1e-9, 0.0, 0.0]], dtype=np.float32)
+    q2, s2, z2 = oq.quantize_codes(y2, 2, 4)
+    assert s2.view(np.float16)[0, 0] == 1.0
+
+
+def test_pack_layout():
+    c4 = np.array([[1, 2, 15, 0]], dtype=np.uint8)
+    assert oq.pack(c4, 4).tolist() == [[0x21, 0x0F]]
+    c2 = np.array([[1, 2, 3, 0, 3, 3, 3, 3]], dtype=np.uint8)
+    assert oq.pack(c2, 2).tolist() == [[0x39, 0xFF]]
+    rng = np.random.default_rng(0)
+    for bits in (2, 4):
+        c = rng.integers(0, 2 ** bits, (3, 64)).astype(np.uint8)
+        assert np.array_equal(oq.unpack(oq.pack(c, bits), bits, 64), c)
+
+
+def test_bf16_rounding_matches_torch():
+    torch = pytest.importorskip("torch")
+    a = np.random.default_rng(0).standard_normal(100000).astype(np.float32) * 100
+    a[:4] = [1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -0.0, 65504.0]
+    ours = wl.bf16_bits_from_f32(a)
+    ref = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    assert np.array_equal(wl.f32_from_bf16_bits(ours), torch.from_numpy(a).to(torch.bfloat16).float().numpy())
+
+
+# ---------------------------------------------------------------- planted mistakes
+# Each case plants a plausible bug in a copy of an oracle step and checks that
+# the independent pins above would reject it.
+
+def _fwd_with(stage_fn, th, x, order=None):
+    m = x.shape[-1]
+    L = bf.num_stages(m)
+    for s in (order if order is not None else range(L)):
+        x = stage_fn(th, x, s)
+    return x
+
+
+def test_planted_sign_flip_is_caught():
+    m = 16
+    th = rand_theta(m, 5)
+    x = np.random.default_rng(1).standard_normal((2, m))
+    wrong = _fwd_with(lambda t, v, s: bf.apply_stage(t, v, s, transpose=True), th, x)
+    assert np.abs(wrong - x @ bf.dense_q(th, m).T).max() > 1e-3
+
+
+def test_planted_stage_order_is_caught():
+    m = 16
+    th = rand_theta(m, 6)
+    x = np.random.default_rng(2).standard_normal((2, m))
+    wrong = _fwd_with(bf.apply_stage, th, x, order=reversed(range(4)))
+    assert np.abs(wrong - x @ bf.dense_q(th, m).T).max() > 1e-3
+
+
+def test_planted_pair_index_is_caught():
+    m = 16
+    th = rand_theta(m, 7)
+    x = np.random.default_rng(3).standard_normal((2, m))
+
+    def bad_stage(t, v, s):
+        i, j, p = bf.pair_indices(m, s)
+        p = p[::-1]                      # angle looked up for the wrong pair
+        c, sn = np.cos(t[s][p].astype(np.float64)), np.sin(t[s][p].astype(np.float64))
+        y = v.copy()
+        y[..., i] = c * v[..., i] - sn * v[..., j]
+        y[..., j] = sn * v[..., i] + c * v[..., j]
+        return y
+
+    wrong = _fwd_with(bad_stage, th, x)
+    assert np.abs(wrong - x @ bf.dense_q(th, m).T).max() > 1e-3
+
+
+def test_planted_dropped_gradient_term_is_caught():
+    m = 4
+    rng = np.random.default_rng(9)
+    th = rng.uniform(-np.pi, np.pi, (2, 2)).astype(np.float32)
+    x = rng.standard_normal((3, m)); dy = rng.standard_normal((3, m))
+    y = bf.forward(th, x)
+    v, g = y.copy(), dy.copy()
+    dth_wrong = np.zeros((2, 2))
+    for s in (1, 0):
+        i, j, p = bf.pair_indices(m, s)
+        dth_wrong[s, p] += (g[:, j] * v[:, i]).sum(0)          # the - g_i v_j term dropped
+        g = bf.apply_stage(th, g, s, transpose=True)
+        v = bf.apply_stage(th, v, s, transpose=True)
+    h = 1e-6
+    thd = th.astype(np.float64)
+    tp = thd.copy(); tp[0, 0] += h
+    tm = thd.copy(); tm[0, 0] -= h
+    fd = (_loss_f64(tp, x, dy) - _loss_f64(tm, x, dy)) / (2 * h)
+    assert abs(fd - dth_wrong[0, 0]) > 1e-3
+
