@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Throughput of the butterfly transform + quantize path on B200.
+
+Default workload (N=1 line): the LLaMA-2-7B activation shape, n = 4096,
+2048 rows of bf16 input, fused Q x + INT4 asymmetric RTN in groups of 128
+(packed 2 codes/byte, fp16 scale/zero).  One step = one bq_transform_quantize
+call over the batch, inputs resident in HBM; the per-layer angle table is
+prepared once before timing (the angles are fixed at inference).  The input
+(16.8 MB) is smaller than L2, so L2 is flushed (256 MB write) before every
+timed step, outside the CUDA-event pair that times the step.
+
+Multi-GPU (torchrun, one process per GPU): rows are independent, so every
+rank processes its own batch of the same shape (weak scaling, no collective
+on the data path); the step time is the max over ranks.
+
+--impl reference times the float64 CPU oracle (tests' ground truth) on a
+bounded sample of the same workload on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+FP32_PEAK_DERIVED = 148 * 128 * 2 * 1.965e9   # SMs x FP32 lanes x 2 flop x max SM clock
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- workloads
+
+def workload_spec(name: str):
+    from rotation_bit_quantization_b200 import workloads as wl
+    if name == "act4096":
+        return dict(make=lambda rank: wl.act_4096(2048, seed_offset=rank), kind="quant", rows=2048, n=4096,
+                    bits=4, group=128, label="act n=4096 rows=2048 bf16 -> Qx + INT4 RTN g128 (LLaMA-2-7B activation shape)")
+    if name == "weight4096":
+        return dict(make=lambda rank: wl.weight_4096(11008), kind="quant", rows=11008, n=4096, bits=2, group=128,
+                    label="weight n=4096 rows=11008 bf16 -> W Q^T + INT2 RTN g128 (W2A16)")
+    if name == "act5120":
+        return dict(make=lambda rank: wl.act_5120(8192), kind="quant", rows=8192, n=5120, bits=4, group=128,
+                    label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> INT4 RTN g128 (LLaMA-2-13B shape)")
+    raise SystemExit(f"unknown workload {name}")
+
+
+def flops_per_row(m: int, r: int) -> float:
+    """Algorithmic flops of one row: 6 per rotation (4 mul + 2 add), (m/2) log2 m rotations per sub-row,
+    plus 2 r^2 per contiguous group for a dense Kronecker factor."""
+    L = m.bit_length() - 1
+    f = 6.0 * (m // 2) * L * r
+    if r > 1:
+        f += 2.0 * r * r * m
+    return f
+
+
+def bytes_per_row(n: int, in_bytes: int, bits: int, group: int) -> float:
+    """Algorithmic HBM bytes of one row: input + packed codes + fp16 scale and zero per group."""
+    return n * in_bytes + n * bits / 8 + 4 * (n // group)
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "rotation_bit_quantization_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode()); h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary, if it was
+    captured on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None, None
+    with open(p) as f:
+        rec = json.load(f).get(workload)
+    if not rec or rec.get("source_hash") != kernel_source_hash():
+        return None, None
+    return rec.get("dram_bytes_per_launch"), rec.get("kernel")
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", str(gpu_index),
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1])); mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_rate(w, rows_target_s: float, max_rows: int):
+    """Rows/s of the float64 oracle (transform + float32-step quantizer) on the host cores."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from oracle import butterfly as ob
+    from oracle import quant as oq
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    cores = len(os.sched_getaffinity(0))
+    src = w.x if w.x is not None else w.w
+    dt = w.x_dtype if w.x is not None else w.w_dtype
+    chunk = 32
+
+    def one(lo):
+        xs = src[lo:lo + chunk]
+        xf = (wl.f32_from_bf16_bits(xs) if dt == "bf16" else xs).astype(np.float64)
+        y = ob.forward(w.theta, xf) if w.r == 1 else ob.kron_forward(w.theta, w.O, xf, w.m)
+        oq.quantize_pack(y.astype(np.float32), w.bits, w.group)
+        return xs.shape[0]
+
+    # calibrate on one chunk, then run a bounded sample on all cores
+    t0 = time.perf_counter(); one(0); t1 = time.perf_counter()
+    per_chunk = t1 - t0
+    nchunks = max(cores, int(rows_target_s * cores / max(per_chunk, 1e-6)))
+    nchunks = min(nchunks, max_rows // chunk)
+    starts = [(k * chunk) % (src.shape[0] - chunk + 1) for k in range(nchunks)]
+    t0 = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        done = sum(ex.map(one, starts))
+    el = time.perf_counter() - t0
+    return done / el, cores, f"{done} rows of the workload ({nchunks} chunks of {chunk}), {el:.1f} s on {cores} threads"
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args, spec, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import rotation_bit_quantization_b200 as bq
+    from rotation_bit_quantization_b200 import build as bq_build
+
+    bq_build.build()
+    bq.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = spec["make"](rank)
+    rows, n, bits, group = spec["rows"], spec["n"], spec["bits"], spec["group"]
+    src = w.x if w.x is not None else w.w
+    src_dtype = w.x_dtype if w.x is not None else w.w_dtype
+    assert src_dtype == "bf16"
+    x_host = torch.from_numpy(src.view(np.int16)).view(torch.bfloat16)
+    x = x_host.to(dev)
+    theta = torch.from_numpy(w.theta).to(dev)
+    O = None if w.O is None else torch.from_numpy(w.O).to(dev)
+    layer = bq.Layer(theta, O)
+    codes, scale, zero = bq.quant_outputs(rows, n, bits, group, dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bq.bq_transform_quantize(layer, x, bits, group, codes, scale, zero)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    wall0 = time.perf_counter()
+    for s, e in evs:
+        flush.zero_()
+        s.record(stream)
+        step()
+        e.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    step_ms = [s.elapsed_time(e) for s, e in evs]
+    total_ms = float(sum(step_ms))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_total_ms = float(t.item())
+    ms_per_step = max_total_ms / args.steps
+    value = rows * world / (ms_per_step * 1e-3)
+
+    # end to end through the public API with host buffers: H2D input, kernel, D2H codes/scale/zero
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_host.pin_memory()
+        c_pin = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+        s_pin = torch.empty(scale.shape, dtype=scale.dtype).pin_memory()
+        z_pin = torch.empty(zero.shape, dtype=zero.dtype).pin_memory()
+        x_e2e = torch.empty_like(x)
+
+        def e2e_step():
+            x_e2e.copy_(x_pin, non_blocking=True)
+            bq.bq_transform_quantize(layer, x_e2e, bits, group, codes, scale, zero)
+            c_pin.copy_(codes, non_blocking=True)
+            s_pin.copy_(scale, non_blocking=True)
+            z_pin.copy_(zero, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e_ms = float(te.item()) / args.steps
+        e2e = {"value": rows * world / (e2e_ms * 1e-3), "unit": "rows/s",
+               "h2d_bytes_per_step": int(x_pin.numel() * x_pin.element_size()),
+               "d2h_bytes_per_step": int(c_pin.numel() * c_pin.element_size() + s_pin.numel() * 2 + z_pin.numel() * 2),
+               "ms_per_step": e2e_ms}
+
+    peaks, peak_src = load_peaks()
+    fl_launch = flops_per_row(w.m, w.r) * rows
+    by_launch = bytes_per_row(n, 2, bits, group) * rows
+    avg_launch_s = (total_ms / args.steps) * 1e-3
+    achieved_tf = fl_launch / avg_launch_s / 1e12
+    traffic, traffic_kernel = recorded_traffic(args.workload)
+    result = {
+        "metric": "butterfly fwd+quant rows/s and GB/s at n=4096 on 1 B200; % of FP32/HBM roofline",
+        "value": value,
+        "unit": "rows/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded; bf16 input, Student-t nu=3 with outlier channels)",
+        "config": {"workload": spec["label"], "rows_per_gpu": rows, "n": n, "bits": bits, "group": group,
+                   "global_batch": rows * world, "parallelism": f"rows sharded, dp{world}",
+                   "l2": "flushed before every timed step (256 MB write outside the timed events)",
+                   "angle_table": "prepared once per layer before timing"},
+        "gbs": by_launch * world / (ms_per_step * 1e-3) / 1e9,
+        "roofline": {
+            "bound": "alu",
+            "achieved": achieved_tf,
+            "peak": FP32_PEAK_DERIVED / 1e12,
+            "unit": "TFLOP/s",
+            "frac": achieved_tf / (FP32_PEAK_DERIVED / 1e12),
+            "traffic": traffic,
+            "peak_note": "FP32 FMA peak derived: 148 SMs x 128 lanes x 2 flop x 1.965 GHz",
+            "algorithmic_flops_per_launch": fl_launch,
+            "algorithmic_bytes_per_launch": by_launch,
+            "hbm_frac": (by_launch / avg_launch_s / 1e9) / peaks["hbm_gbs"],
+            "hbm_peak_gbs": peaks["hbm_gbs"],
+            "hbm_peak_source": peak_src,
+            "kernel": traffic_kernel,
+        },
+        "e2e": e2e,
+        "gpu_launches": args.steps,
+        "clocks": clocks,
+        "wall_s_timed_region": wall,
+        "step_ms_min": min(step_ms),
+        "step_ms_median": statistics.median(step_ms),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = cpu_oracle_rate(w, rows_target_s=10.0, max_rows=rows * 8)
+        result["cpu_baseline"] = {"value": rate, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample}
+    return result
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, spec):
+    w = spec["make"](0)
+    for _ in range(args.warmup):
+        cpu_oracle_rate(w, rows_target_s=1.0, max_rows=256)
+    rates = []
+    sample = cores = None
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        rate, cores, sample = cpu_oracle_rate(w, rows_target_s=3.0, max_rows=spec["rows"])
+        rates.append(rate)
+    el = time.perf_counter() - t0
+    value = statistics.median(rates)
+    return {
+        "impl": "reference",
+        "metric": "butterfly fwd+quant rows/s and GB/s at n=4096 on 1 B200; % of FP32/HBM roofline",
+        "value": value,
+        "unit": "rows/s",
+        "n_gpus": 1,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded)",
+        "config": {"workload": spec["label"], "rows_per_gpu": spec["rows"], "n": spec["n"], "bits": spec["bits"],
+                   "group": spec["group"]},
+        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- main
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="act4096", choices=["act4096", "weight4096", "act5120"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    spec = workload_spec(args.workload)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, spec)))
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, spec, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,150 @@
+/*
+ * bq.h - C ABI of libbq.so: the learnable orthogonal butterfly transform and
+ * its fused low-bit quantization, hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The method: ButterflyQuant (abstract, arXiv 2509.09679) rotates activations
+ * and weights with the same orthogonal Q so that a linear layer is unchanged,
+ * y = W x = (W Q^T)(Q x).  Q is a butterfly of Givens rotations with
+ * continuous angles: log2(m) stages, stage s rotating the index pairs
+ * (i, i + 2^s) with [[cos t, -sin t], [sin t, cos t]], m*log2(m)/2 angles in
+ * total (abstract; explainer article, section "butterfly").  Widths that are
+ * not a power of two use a Kronecker composite Q = B_m (x) O_r (explainer
+ * article, section "butterfly").  The angles are learned by gradient descent
+ * (abstract), which needs the backward pass exported here.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All data pointers are DEVICE pointers unless stated; the caller owns
+ *    every buffer.  The library never allocates device memory and keeps no
+ *    global state; calls on different streams are independent.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call is asynchronous on that stream; an error status is
+ *    returned before anything is launched when host-side validation fails.
+ *  - Rows are contiguous and row-major: element (row, i) is at row*n + i.
+ *  - Element index i = i1*r + i2 with i1 < m, i2 < r; B_m acts on i1, O_r on i2.
+ *  - Angle layout: theta[s*(m/2) + p] for stage s < log2(m) and pair number
+ *    p = ((i >> (s+1)) << s) | (i & (2^s - 1)) of the pair (i, i + 2^s).
+ *  - Stage order: Q = B_{L-1} ... B_1 B_0 (stage 0, stride 1, acts first).
+ *  - Data pointers must be 16-byte aligned; m must be a power of two in
+ *    [2, 4096]; r in [1, 8]; n = m*r <= 16384.
+ *  - Arithmetic is float32 (bf16 inputs are widened exactly; bf16 outputs are
+ *    rounded to nearest even).
+ *  - Errors: BQ_ERR_INVALID_ARG (bad sizes, null or misaligned pointers),
+ *    BQ_ERR_UNSUPPORTED (valid request outside what this build implements),
+ *    BQ_ERR_WORKSPACE (workspace too small), BQ_ERR_CUDA (a launch failed;
+ *    the CUDA error is left for cudaGetLastError to report).  No entry point
+ *    aborts, traps or asserts on the device.
+ */
+#ifndef BQ_H_
+#define BQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  BQ_OK = 0,
+  BQ_ERR_INVALID_ARG = 1,
+  BQ_ERR_UNSUPPORTED = 2,
+  BQ_ERR_WORKSPACE = 3,
+  BQ_ERR_CUDA = 4
+} bq_status;
+
+typedef enum { BQ_F32 = 0, BQ_BF16 = 1 } bq_dtype;
+
+/* One layer's transform.  The struct itself lives in host memory; its
+ * pointers are device pointers.
+ *   n = m*r;  table: bq_table_floats(m) floats written by bq_precompute_cs for
+ *   this layer's angles;  O: r*r float32 row-major orthogonal matrix, NULL
+ *   iff r == 1 (O is an input of the composite, not a learned parameter). */
+typedef struct {
+  int32_t n, m, r;
+  const float* table;
+  const float* O;
+} bq_layer;
+
+/* Number of floats of the per-layer prepared table for width m (0 if m is
+ * not a supported power of two). */
+size_t bq_table_floats(int32_t m);
+
+/* Angle preparation, once per layer (explainer article, section "butterfly":
+ * the angles parameterise the Givens rotations).  Reads theta[log2(m)*(m/2)]
+ * (device, float32) and writes `table` (device, bq_table_floats(m) floats):
+ * cos/sin of every angle (float64 sincos rounded to float32) plus the derived
+ * per-position coefficients and scales that the scaled-rotation kernels use.
+ * The table must be rebuilt whenever theta changes. */
+bq_status bq_precompute_cs(const float* theta, int32_t m, float* table, void* stream);
+
+/* y = Q x for every row (abstract: the activation side Q x).
+ * x: rows*n elements of type xt; y: rows*n elements of type yt.  x == y is
+ * allowed when xt == yt (each row is read completely before it is written). */
+bq_status bq_butterfly_fwd(const bq_layer* layer, const void* x, bq_dtype xt,
+                           void* y, bq_dtype yt, int64_t rows, void* stream);
+
+/* x = Q^T y for every row: stages L-1 .. 0 with every angle negated, and O_r^T
+ * for the composite (Q is orthogonal by construction, abstract).  Same layout
+ * and aliasing rule as bq_butterfly_fwd. */
+bq_status bq_butterfly_inv(const bq_layer* layer, const void* y, bq_dtype yt,
+                           void* x, bq_dtype xt, int64_t rows, void* stream);
+
+/* Bytes of workspace bq_butterfly_bwd needs for num_layers layers of width m
+ * with rows_per_layer tokens each. */
+size_t bq_butterfly_bwd_workspace_size(int32_t m, int32_t num_layers, int64_t rows_per_layer);
+
+/* Backward for calibration (abstract: angles learned by gradient-based
+ * optimisation), all layers in ONE launch.  For layer l with loss linear in
+ * Y_l and upstream gradient dY_l:
+ *   Y_l = Q_l X_l;  dX_l = Q_l^T dY_l;
+ *   dtheta_l[s*(m/2)+p] = sum over tokens of (g_j v_i - g_i v_j), where v and g
+ *   are the output and output-gradient of stage s at its pair (i, j).
+ * layers: HOST array of num_layers (<= 128) descriptors, all with the same m
+ *   and r == 1.
+ * x: [num_layers][rows_per_layer][m] of type xt; y: same shape of type yt;
+ * dy, dx: float32, same shape; dtheta: float32 [num_layers][log2(m)*(m/2)].
+ * The token reduction is deterministic (fixed-order partial sums in
+ * `workspace`, reduced by the last block of each layer); repeated calls give
+ * bitwise identical dtheta.  workspace: device, >= the size queried above,
+ * 16-byte aligned; its contents on entry are irrelevant. */
+bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers,
+                           const void* x, bq_dtype xt, void* y, bq_dtype yt,
+                           const float* dy, float* dx, float* dtheta,
+                           int64_t rows_per_layer, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Fused Q x followed by per-group asymmetric round-to-nearest quantization and
+ * packing (2-bit weights: explainer article, section "training & results";
+ * RTN block quantizer: WUSH technical summary, section 2).  Per group of
+ * `group` contiguous outputs of a row (group divides n, group % 32 == 0):
+ *   lo, hi = min, max;  scale16 = fp16_rn((hi - lo) / qmax);  s = scale16
+ *   (s = 1 when hi == lo or scale16 == 0);  z = clamp(rint(-lo / s), 0, qmax);
+ *   q = clamp(rint(y / s) + z, 0, qmax), rint half-to-even, IEEE float32
+ *   division; qmax = 2^bits - 1.
+ * The y quantized is bitwise the float32 output bq_butterfly_fwd produces.
+ * codes: [rows][n*bits/8] bytes, lowest element in the lowest bits
+ *   (INT4: q[2k] | q[2k+1] << 4; INT2: q[4k] | q[4k+1] << 2 | ...);
+ * scale_f16, zero_f16: [rows][n/group] fp16 bit patterns.  bits: 2 or 4. */
+bq_status bq_transform_quantize(const bq_layer* layer, const void* x, bq_dtype xt,
+                                int64_t rows, int32_t bits, int32_t group,
+                                uint8_t* codes, uint16_t* scale_f16,
+                                uint16_t* zero_f16, void* stream);
+
+/* Weight side of the invariance y = (W Q^T)(Q x) (abstract): row r of W Q^T
+ * is Q w_r, so this rotates every row of W [out_features][n] and quantizes and
+ * packs it exactly as bq_transform_quantize does (identical bits for identical
+ * input); the W2A16 setting uses bits = 2. */
+bq_status bq_weight_rotate_pack(const bq_layer* layer, const void* w, bq_dtype wt,
+                                int64_t out_features, int32_t bits, int32_t group,
+                                uint8_t* codes, uint16_t* scale_f16,
+                                uint16_t* zero_f16, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* bq_status_string(bq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BQ_H_ */

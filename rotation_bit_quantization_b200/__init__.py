@@ -1,0 +1,21 @@
+"""B200-native learnable butterfly transform + low-bit quantization (ButterflyQuant hot path).
+
+The compute path is libbq.so (hand-written CUDA for sm_100a, C ABI in
+include/bq.h); this package only marshals arguments to it (``_lib``), builds it
+(``build``) and draws seeded synthetic inputs (``workloads``).
+"""
+
+from ._lib import (  # noqa: F401
+    BQError,
+    Layer,
+    bq_butterfly_bwd,
+    bq_butterfly_bwd_workspace_size,
+    bq_butterfly_fwd,
+    bq_butterfly_inv,
+    bq_precompute_cs,
+    bq_transform_quantize,
+    bq_weight_rotate_pack,
+    load,
+    quant_outputs,
+    status_string,
+)

@@ -1,0 +1,215 @@
+"""ctypes binding of libbq.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls (see
+include/bq.h).  Tensors are torch CUDA tensors; their device pointers and the
+current CUDA stream are passed through unchanged.  Nothing is computed on the
+host: if libbq.so is missing or a call fails, an exception is raised (there is
+no fallback path).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libbq.so")
+
+BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_WORKSPACE, BQ_ERR_CUDA = range(5)
+BQ_F32, BQ_BF16 = 0, 1
+
+EXPORTED = (
+    "bq_table_floats",
+    "bq_precompute_cs",
+    "bq_butterfly_fwd",
+    "bq_butterfly_inv",
+    "bq_butterfly_bwd_workspace_size",
+    "bq_butterfly_bwd",
+    "bq_transform_quantize",
+    "bq_weight_rotate_pack",
+    "bq_status_string",
+)
+
+
+class BQLayer(ctypes.Structure):
+    _fields_ = [("n", ctypes.c_int32), ("m", ctypes.c_int32), ("r", ctypes.c_int32),
+                ("table", ctypes.c_void_p), ("O", ctypes.c_void_p)]
+
+
+class BQError(RuntimeError):
+    def __init__(self, name: str, status: int, text: str):
+        super().__init__(f"{name} failed: status {status} ({text})")
+        self.status = status
+
+
+_lib = None
+
+
+def load(path: str | None = None):
+    """Load libbq.so (once).  Raises if the library has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = path or LIB_PATH
+    if not os.path.exists(path):
+        raise ImportError(f"libbq.so not found at {path}; build it with "
+                          "`python -m rotation_bit_quantization_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    lp = ctypes.POINTER(BQLayer)
+    sig = {
+        "bq_table_floats": (sz, [i32]),
+        "bq_precompute_cs": (i32, [vp, i32, vp, vp]),
+        "bq_butterfly_fwd": (i32, [lp, vp, i32, vp, i32, i64, vp]),
+        "bq_butterfly_inv": (i32, [lp, vp, i32, vp, i32, i64, vp]),
+        "bq_butterfly_bwd_workspace_size": (sz, [i32, i32, i64]),
+        "bq_butterfly_bwd": (i32, [lp, i32, vp, i32, vp, i32, vp, vp, vp, i64, vp, sz, vp]),
+        "bq_transform_quantize": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+        "bq_weight_rotate_pack": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+        "bq_status_string": (ctypes.c_char_p, [i32]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().bq_status_string(status).decode()
+
+
+def _check(name: str, status: int):
+    if status != BQ_OK:
+        raise BQError(name, status, status_string(status))
+
+
+# ----------------------------------------------------------------------------- marshalling helpers
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return BQ_F32
+    if t.dtype == torch.bfloat16:
+        return BQ_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: use float32 or bfloat16")
+
+
+def _stream(stream=None):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dev(t, name):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+class Layer:
+    """One layer's prepared transform: holds the device table (and O_r) alive.
+
+    theta: float32 CUDA tensor of shape (log2 m, m/2); O: None or float32 CUDA
+    tensor (r, r).  The table is filled by bq_precompute_cs on the current stream.
+    """
+
+    def __init__(self, theta, O=None, stream=None):
+        torch = _torch()
+        lib = load()
+        _dev(theta, "theta")
+        if theta.dtype != torch.float32 or theta.dim() != 2:
+            raise ValueError("theta must be float32 of shape (log2 m, m/2)")
+        self.m = int(theta.shape[1]) * 2
+        self.r = 1 if O is None else int(O.shape[0])
+        self.n = self.m * self.r
+        floats = lib.bq_table_floats(self.m)
+        if floats == 0:
+            raise ValueError(f"unsupported butterfly width m={self.m}")
+        self.theta = theta
+        self.table = torch.empty(floats, dtype=torch.float32, device=theta.device)
+        self.O = None if O is None else _dev(O, "O")
+        bq_precompute_cs(theta, self.m, self.table, stream)
+        self.c = BQLayer(self.n, self.m, self.r, self.table.data_ptr(),
+                         None if self.O is None else self.O.data_ptr())
+
+    @property
+    def fast_form(self) -> bool:
+        """Whether the scaled two-FMA rotation form is in range for these angles (header flag)."""
+        return bool(self.table[0].item() == 1.0)
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def bq_precompute_cs(theta, m: int, table, stream=None):
+    _check("bq_precompute_cs", load().bq_precompute_cs(_ptr(theta), m, _ptr(table), _stream(stream)))
+
+
+def bq_butterfly_fwd(layer: Layer, x, y, stream=None):
+    _dev(x, "x"); _dev(y, "y")
+    rows = x.numel() // layer.n
+    _check("bq_butterfly_fwd", load().bq_butterfly_fwd(ctypes.byref(layer.c), _ptr(x), _dtype_code(x), _ptr(y),
+                                                        _dtype_code(y), rows, _stream(stream)))
+    return y
+
+
+def bq_butterfly_inv(layer: Layer, y, x, stream=None):
+    _dev(x, "x"); _dev(y, "y")
+    rows = y.numel() // layer.n
+    _check("bq_butterfly_inv", load().bq_butterfly_inv(ctypes.byref(layer.c), _ptr(y), _dtype_code(y), _ptr(x),
+                                                        _dtype_code(x), rows, _stream(stream)))
+    return x
+
+
+def bq_butterfly_bwd_workspace_size(m: int, num_layers: int, rows_per_layer: int) -> int:
+    return int(load().bq_butterfly_bwd_workspace_size(m, num_layers, rows_per_layer))
+
+
+def bq_butterfly_bwd(layers, x, y, dy, dx, dtheta, workspace, stream=None):
+    """x, y, dy, dx: (layers, rows, m); dtheta: (layers, log2 m * m/2) float32."""
+    arr = (BQLayer * len(layers))(*[l.c for l in layers])
+    for t, nm in ((x, "x"), (y, "y"), (dy, "dy"), (dx, "dx"), (dtheta, "dtheta"), (workspace, "workspace")):
+        _dev(t, nm)
+    rows = x.numel() // (len(layers) * layers[0].n)
+    _check("bq_butterfly_bwd", load().bq_butterfly_bwd(arr, len(layers), _ptr(x), _dtype_code(x), _ptr(y),
+                                                        _dtype_code(y), _ptr(dy), _ptr(dx), _ptr(dtheta), rows,
+                                                        _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                                        _stream(stream)))
+
+
+def _quant(name, layer, x, bits, group, codes, scale, zero, stream):
+    _dev(x, "x"); _dev(codes, "codes"); _dev(scale, "scale"); _dev(zero, "zero")
+    rows = x.numel() // layer.n
+    fn = getattr(load(), name)
+    _check(name, fn(ctypes.byref(layer.c), _ptr(x), _dtype_code(x), rows, bits, group, _ptr(codes), _ptr(scale),
+                    _ptr(zero), _stream(stream)))
+    return codes, scale, zero
+
+
+def quant_outputs(rows: int, n: int, bits: int, group: int, device):
+    """Allocate (codes uint8 [rows][n*bits/8], scale int16 [rows][n/group], zero int16 [rows][n/group])."""
+    torch = _torch()
+    codes = torch.empty((rows, n * bits // 8), dtype=torch.uint8, device=device)
+    scale = torch.empty((rows, n // group), dtype=torch.int16, device=device)
+    zero = torch.empty((rows, n // group), dtype=torch.int16, device=device)
+    return codes, scale, zero
+
+
+def bq_transform_quantize(layer: Layer, x, bits: int, group: int, codes, scale, zero, stream=None):
+    return _quant("bq_transform_quantize", layer, x, bits, group, codes, scale, zero, stream)
+
+
+def bq_weight_rotate_pack(layer: Layer, w, bits: int, group: int, codes, scale, zero, stream=None):
+    return _quant("bq_weight_rotate_pack", layer, w, bits, group, codes, scale, zero, stream)

@@ -1,0 +1,138 @@
+// C ABI entry points of libbq.so: host-side validation and dispatch.  Every
+// check runs before anything is launched; a failed check returns a status and
+// launches nothing.  See include/bq.h for the contract of each call.
+#include "bq_internal.cuh"
+
+namespace bq {
+namespace {
+
+bool valid_m(int m) { return m >= 2 && m <= kMaxM && (m & (m - 1)) == 0; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool valid_dtype(bq_dtype t) { return t == BQ_F32 || t == BQ_BF16; }
+
+bq_status check_layer(const bq_layer* l) {
+  if (!l) return BQ_ERR_INVALID_ARG;
+  if (!valid_m(l->m) || l->r < 1 || l->r > kMaxR) return BQ_ERR_INVALID_ARG;
+  if (static_cast<long long>(l->m) * l->r != l->n || l->n > kMaxN) return BQ_ERR_INVALID_ARG;
+  if (!l->table || !aligned16(l->table)) return BQ_ERR_INVALID_ARG;
+  if ((l->r > 1) != (l->O != nullptr)) return BQ_ERR_INVALID_ARG;
+  if (l->O && (reinterpret_cast<uintptr_t>(l->O) & 3u)) return BQ_ERR_INVALID_ARG;
+  return BQ_OK;
+}
+
+bq_status check_rows(const void* a, const void* b, int64_t rows) {
+  if (rows < 0) return BQ_ERR_INVALID_ARG;
+  if (rows == 0) return BQ_OK;
+  if (!a || !b || !aligned16(a) || !aligned16(b)) return BQ_ERR_INVALID_ARG;
+  return BQ_OK;
+}
+
+bq_status transform(const bq_layer* layer, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
+                    void* stream, bool inverse) {
+  bq_status s = check_layer(layer);
+  if (s != BQ_OK) return s;
+  if (!valid_dtype(xt) || !valid_dtype(yt)) return BQ_ERR_INVALID_ARG;
+  if ((s = check_rows(x, y, rows)) != BQ_OK) return s;
+  if (rows == 0) return BQ_OK;
+  if (x == y && xt != yt) return BQ_ERR_INVALID_ARG;
+  const KLayer L = make_klayer(*layer);
+  return launch_generic(L, x, xt, y, yt, rows, inverse, nullptr, static_cast<cudaStream_t>(stream));
+}
+
+bq_status quantize(const bq_layer* layer, const void* x, bq_dtype xt, int64_t rows, int32_t bits, int32_t group,
+                   uint8_t* codes, uint16_t* scale, uint16_t* zero, void* stream) {
+  bq_status s = check_layer(layer);
+  if (s != BQ_OK) return s;
+  if (!valid_dtype(xt)) return BQ_ERR_INVALID_ARG;
+  if (bits != 2 && bits != 4) return BQ_ERR_INVALID_ARG;
+  if (group < 32 || group > kMaxGroup || (group & 31) || layer->n % group) return BQ_ERR_INVALID_ARG;
+  if (rows < 0) return BQ_ERR_INVALID_ARG;
+  if (rows == 0) return BQ_OK;
+  if (!x || !codes || !scale || !zero) return BQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes) || !aligned16(scale) || !aligned16(zero)) return BQ_ERR_INVALID_ARG;
+  const KLayer L = make_klayer(*layer);
+  QuantArgs q{bits, group, codes, scale, zero};
+  return launch_generic(L, x, xt, nullptr, BQ_F32, rows, false, &q, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" {
+
+size_t bq_table_floats(int32_t m) {
+  if (!valid_m(m)) return 0;
+  return table_layout(m).total;
+}
+
+bq_status bq_precompute_cs(const float* theta, int32_t m, float* table, void* stream) {
+  if (!valid_m(m) || !theta || !table || !aligned16(table) || (reinterpret_cast<uintptr_t>(theta) & 3u))
+    return BQ_ERR_INVALID_ARG;
+  return launch_prepare(theta, m, table, static_cast<cudaStream_t>(stream));
+}
+
+bq_status bq_butterfly_fwd(const bq_layer* layer, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
+                           void* stream) {
+  return transform(layer, x, xt, y, yt, rows, stream, false);
+}
+
+bq_status bq_butterfly_inv(const bq_layer* layer, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
+                           void* stream) {
+  return transform(layer, y, yt, x, xt, rows, stream, true);
+}
+
+size_t bq_butterfly_bwd_workspace_size(int32_t m, int32_t num_layers, int64_t rows_per_layer) {
+  if (!valid_m(m) || num_layers < 1 || num_layers > kMaxBwdLayers || rows_per_layer < 1) return 0;
+  return bwd_workspace_bytes(m, num_layers, bwd_chunks(m, num_layers, rows_per_layer));
+}
+
+bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers, const void* x, bq_dtype xt, void* y,
+                           bq_dtype yt, const float* dy, float* dx, float* dtheta, int64_t rows_per_layer,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (!layers || num_layers < 1 || num_layers > kMaxBwdLayers) return BQ_ERR_INVALID_ARG;
+  if (!valid_dtype(xt) || !valid_dtype(yt)) return BQ_ERR_INVALID_ARG;
+  const int m = layers[0].m;
+  KLayer kl[kMaxBwdLayers];
+  for (int l = 0; l < num_layers; ++l) {
+    bq_status s = check_layer(&layers[l]);
+    if (s != BQ_OK) return s;
+    if (layers[l].m != m) return BQ_ERR_INVALID_ARG;
+    if (layers[l].r != 1) return BQ_ERR_UNSUPPORTED;
+    kl[l] = make_klayer(layers[l]);
+  }
+  if (rows_per_layer < 1) return BQ_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, y, dy, dx, dtheta, workspace};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return BQ_ERR_INVALID_ARG;
+  const int chunks = bwd_chunks(m, num_layers, rows_per_layer);
+  if (workspace_bytes < bwd_workspace_bytes(m, num_layers, chunks)) return BQ_ERR_WORKSPACE;
+  return launch_bwd(kl, num_layers, x, xt, y, yt, dy, dx, dtheta, rows_per_layer, workspace, chunks,
+                    static_cast<cudaStream_t>(stream));
+}
+
+bq_status bq_transform_quantize(const bq_layer* layer, const void* x, bq_dtype xt, int64_t rows, int32_t bits,
+                                int32_t group, uint8_t* codes, uint16_t* scale_f16, uint16_t* zero_f16,
+                                void* stream) {
+  return quantize(layer, x, xt, rows, bits, group, codes, scale_f16, zero_f16, stream);
+}
+
+bq_status bq_weight_rotate_pack(const bq_layer* layer, const void* w, bq_dtype wt, int64_t out_features,
+                                int32_t bits, int32_t group, uint8_t* codes, uint16_t* scale_f16,
+                                uint16_t* zero_f16, void* stream) {
+  return quantize(layer, w, wt, out_features, bits, group, codes, scale_f16, zero_f16, stream);
+}
+
+const char* bq_status_string(bq_status status) {
+  switch (status) {
+    case BQ_OK: return "ok";
+    case BQ_ERR_INVALID_ARG: return "invalid argument";
+    case BQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case BQ_ERR_WORKSPACE: return "workspace too small";
+    case BQ_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

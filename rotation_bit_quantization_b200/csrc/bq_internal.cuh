@@ -1,0 +1,96 @@
+// Internal declarations shared by the libbq CUDA sources (not part of the C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "bq.h"
+
+namespace bq {
+
+constexpr int kMaxM = 4096;        // largest butterfly width (power of two)
+constexpr int kMaxR = 8;           // largest dense Kronecker factor
+constexpr int kMaxN = 16384;       // largest row width m*r
+constexpr int kMaxBwdLayers = 128; // layers per backward launch (kernel-parameter array)
+constexpr int kMaxGroup = 256;     // largest quantization group
+
+// Prepared-table layout (floats), per layer of width m with L = log2(m) stages:
+//   [0, 16)            header: [0] = 1.0 when the scaled (fast) rotation form is
+//                      usable for this layer, else 0.0; [1] = m; [2] = L
+//   cs     [L][m/2]    float2 (cos, sin) of every angle
+//   fast   [L][m]      per-position coefficient of the scaled form: at stage s
+//                      position i is updated as a_i += fast[s][i] * a_{i ^ 2^s}
+//   sigma  [m]         per-position output scale of the scaled form
+struct TableLayout {
+  int m, L;
+  size_t off_cs, off_fast, off_sigma, total;
+};
+
+__host__ __device__ inline int ilog2(int v) {
+  int l = 0;
+  while ((1 << l) < v) ++l;
+  return l;
+}
+
+__host__ __device__ inline size_t round4(size_t v) { return (v + 3) & ~size_t(3); }
+
+__host__ __device__ inline TableLayout table_layout(int m) {
+  TableLayout t;
+  t.m = m;
+  t.L = ilog2(m);
+  t.off_cs = 16;
+  t.off_fast = t.off_cs + round4(size_t(t.L) * m);
+  t.off_sigma = t.off_fast + round4(size_t(t.L) * m);
+  t.total = t.off_sigma + round4(size_t(m));
+  return t;
+}
+
+// Everything a kernel needs about one layer, passed by value.
+struct KLayer {
+  int n, m, r, L;
+  const float2* cs;     // [L][m/2]
+  const float* fast;    // [L][m]
+  const float* sigma;   // [m]
+  const float* hdr;     // header (flag at hdr[0])
+  const float* O;       // [r][r] or nullptr
+};
+
+inline KLayer make_klayer(const bq_layer& l) {
+  TableLayout t = table_layout(l.m);
+  KLayer k;
+  k.n = l.n; k.m = l.m; k.r = l.r; k.L = t.L;
+  k.cs = reinterpret_cast<const float2*>(l.table + t.off_cs);
+  k.fast = l.table + t.off_fast;
+  k.sigma = l.table + t.off_sigma;
+  k.hdr = l.table;
+  k.O = l.O;
+  return k;
+}
+
+struct QuantArgs {
+  int bits, group;
+  uint8_t* codes;
+  uint16_t* scale;
+  uint16_t* zero;
+};
+
+// Launchers (defined in the .cu files).  Each returns BQ_OK or BQ_ERR_CUDA.
+bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t st);
+bq_status launch_generic(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt,
+                         int64_t rows, bool inverse, const QuantArgs* q, cudaStream_t st);
+bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt,
+                     void* y, bq_dtype yt, const float* dy, float* dx, float* dtheta,
+                     int64_t rows, void* ws, int chunks, cudaStream_t st);
+int bwd_chunks(int m, int num_layers, int64_t rows);
+size_t bwd_workspace_bytes(int m, int num_layers, int chunks);
+
+// ---------------------------------------------------------------- device helpers
+
+__device__ __forceinline__ float load_elem(const float* p) { return *p; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+__device__ __forceinline__ void store_elem(float* p, float v) { *p = v; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+}  // namespace bq

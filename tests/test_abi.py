@@ -1,0 +1,142 @@
+"""The C ABI library loads, exports every symbol include/bq.h declares, and
+rejects bad arguments on the host before touching the GPU (no compute here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from rotation_bit_quantization_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "bq.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    syms = declared_symbols()
+    for name in ("bq_butterfly_fwd", "bq_butterfly_inv", "bq_butterfly_bwd", "bq_transform_quantize",
+                 "bq_weight_rotate_pack"):
+        assert name in syms
+    assert set(syms) == set(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    for name in declared_symbols():
+        assert re.search(rf"\bT {name}\b", out), name
+
+
+def test_status_strings(lib):
+    assert _lib.status_string(0) == "ok"
+    assert "invalid" in _lib.status_string(1)
+    assert _lib.status_string(99) == "unknown status"
+
+
+def test_table_sizes(lib):
+    assert lib.bq_table_floats(4096) > 2 * 12 * 4096
+    assert lib.bq_table_floats(3) == 0
+    assert lib.bq_table_floats(8192) == 0          # above the supported width
+    assert lib.bq_table_floats(1) == 0
+
+
+def test_workspace_size(lib):
+    ws = lib.bq_butterfly_bwd_workspace_size(4096, 32, 65536)
+    assert ws >= 32 * 24576 * 4
+    assert lib.bq_butterfly_bwd_workspace_size(4096, 0, 10) == 0
+    assert lib.bq_butterfly_bwd_workspace_size(4096, 129, 10) == 0
+    assert lib.bq_butterfly_bwd_workspace_size(5000, 2, 10) == 0
+
+
+def _layer(n, m, r, table=16, O=None):
+    return _lib.BQLayer(n, m, r, table, O)
+
+
+FAKE = 0x10000  # 16-byte aligned, never dereferenced: validation fails first or nothing is launched
+
+
+@pytest.mark.parametrize("layer,why", [
+    (_layer(4096, 4096, 1, table=None), "null table"),
+    (_layer(4096, 4096, 1, table=FAKE + 4), "misaligned table"),
+    (_layer(4095, 4095, 1, table=FAKE), "m not a power of two"),
+    (_layer(8192, 8192, 1, table=FAKE), "m too large"),
+    (_layer(4096, 1024, 5, table=FAKE), "n != m*r"),
+    (_layer(5120, 1024, 5, table=FAKE), "r > 1 without O"),
+    (_layer(1024, 1024, 1, table=FAKE, O=FAKE), "O given with r == 1"),
+    (_layer(9 * 1024, 1024, 9, table=FAKE, O=FAKE), "r too large"),
+])
+def test_fwd_rejects_bad_layers(lib, layer, why):
+    st = lib.bq_butterfly_fwd(ctypes.byref(layer), FAKE, 0, FAKE, 0, 4, None)
+    assert st == _lib.BQ_ERR_INVALID_ARG, why
+
+
+def test_fwd_rejects_bad_buffers(lib):
+    good = _layer(256, 256, 1, table=FAKE)
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), None, 0, FAKE, 0, 4, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), FAKE + 8, 0, FAKE, 0, 4, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), FAKE, 7, FAKE, 0, 4, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), FAKE, 0, FAKE, 1, 4, None) == _lib.BQ_ERR_INVALID_ARG  # alias, dtypes differ
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), FAKE, 0, FAKE, 0, -1, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_fwd(ctypes.byref(good), None, 0, None, 0, 0, None) == _lib.BQ_OK   # empty: no launch
+    assert lib.bq_butterfly_inv(None, FAKE, 0, FAKE, 0, 4, None) == _lib.BQ_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("bits,group,ok", [(3, 128, False), (4, 48, False), (4, 100, False), (2, 512, False),
+                                           (4, 96, False), (4, 0, False)])
+def test_quantize_rejects_bad_settings(lib, bits, group, ok):
+    good = _layer(4096, 4096, 1, table=FAKE)
+    st = lib.bq_transform_quantize(ctypes.byref(good), FAKE, 0, 8, bits, group, FAKE, FAKE, FAKE, None)
+    assert st == _lib.BQ_ERR_INVALID_ARG
+    st = lib.bq_weight_rotate_pack(ctypes.byref(good), FAKE, 0, 8, bits, group, FAKE, FAKE, FAKE, None)
+    assert st == _lib.BQ_ERR_INVALID_ARG
+
+
+def test_quantize_rejects_null_outputs(lib):
+    good = _layer(4096, 4096, 1, table=FAKE)
+    assert lib.bq_transform_quantize(ctypes.byref(good), FAKE, 0, 8, 4, 128, None, FAKE, FAKE, None) == 1
+    assert lib.bq_transform_quantize(ctypes.byref(good), FAKE, 0, 8, 4, 128, FAKE, FAKE + 2, FAKE, None) == 1
+    assert lib.bq_transform_quantize(ctypes.byref(good), FAKE, 0, 0, 4, 128, None, None, None, None) == 0
+
+
+def test_bwd_rejects_bad_arguments(lib):
+    L = (_lib.BQLayer * 2)(_layer(64, 64, 1, table=FAKE), _layer(64, 64, 1, table=FAKE))
+    ws = lib.bq_butterfly_bwd_workspace_size(64, 2, 10)
+    args = [FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, 10, FAKE]
+    assert lib.bq_butterfly_bwd(L, 2, *args, ws - 1, None) == _lib.BQ_ERR_WORKSPACE
+    assert lib.bq_butterfly_bwd(L, 0, *args, ws, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_bwd(None, 2, *args, ws, None) == _lib.BQ_ERR_INVALID_ARG
+    bad = list(args); bad[4] = None
+    assert lib.bq_butterfly_bwd(L, 2, *bad, ws, None) == _lib.BQ_ERR_INVALID_ARG
+    mixed = (_lib.BQLayer * 2)(_layer(64, 64, 1, table=FAKE), _layer(32, 32, 1, table=FAKE))
+    assert lib.bq_butterfly_bwd(mixed, 2, *args, ws, None) == _lib.BQ_ERR_INVALID_ARG
+    kron = (_lib.BQLayer * 1)(_layer(320, 64, 5, table=FAKE, O=FAKE))
+    assert lib.bq_butterfly_bwd(kron, 1, *args, ws, None) == _lib.BQ_ERR_UNSUPPORTED
+
+
+def test_precompute_rejects_bad_width(lib):
+    assert lib.bq_precompute_cs(FAKE, 12, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_cs(None, 16, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_cs(FAKE, 16, FAKE + 4, None) == _lib.BQ_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    saved = _lib._lib
+    try:
+        _lib._lib = None
+        with pytest.raises(ImportError):
+            _lib.load(str(tmp_path / "missing.so"))
+    finally:
+        _lib._lib = saved

@@ -1,0 +1,294 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Small shapes span several work tiles and ragged tails; the full workload sizes
+are checked on sampled rows the oracle computes one by one.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import butterfly as ob
+from oracle import quant as oq
+from rotation_bit_quantization_b200 import workloads as wl
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bq():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import rotation_bit_quantization_b200 as bq_mod
+    from rotation_bit_quantization_b200 import build
+    build.build()
+    bq_mod.load()
+    return bq_mod
+
+
+def make_layer(bq, theta, O=None):
+    return bq.Layer(H.dev_f32(theta), None if O is None else H.dev_f32(O))
+
+
+def run_fwd(bq, layer, x_dev, out_dtype):
+    torch = H.torch()
+    y = torch.empty(x_dev.shape, dtype=out_dtype, device="cuda")
+    bq.bq_butterfly_fwd(layer, x_dev, y)
+    torch.cuda.synchronize()
+    return y
+
+
+# --------------------------------------------------------------------------- transform
+
+@pytest.mark.parametrize("m", [2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096])
+@pytest.mark.parametrize("rows", [1, 3, 37])
+def test_fwd_inv_f32_small(bq, m, rows):
+    torch = H.torch()
+    rng = np.random.default_rng(m * 100 + rows)
+    theta = wl.uniform_angles(rng, m)
+    x = rng.standard_normal((rows, m)).astype(np.float32) * rng.uniform(0.1, 10, (rows, 1)).astype(np.float32)
+    layer = make_layer(bq, theta)
+    y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+    ref = ob.forward(theta, x.astype(np.float64))
+    H.assert_f32_close(H.host(y), ref, x.astype(np.float64))
+    xb = torch.empty_like(y)
+    bq.bq_butterfly_inv(layer, y, xb)
+    torch.cuda.synchronize()
+    H.assert_f32_close(H.host(xb), ob.inverse(theta, H.host(y).astype(np.float64)), x.astype(np.float64))
+    H.assert_f32_close(H.host(xb), x.astype(np.float64), x.astype(np.float64))
+
+
+@pytest.mark.parametrize("m,r", [(4, 3), (16, 5), (64, 2), (256, 7), (1024, 5), (512, 8)])
+def test_kronecker_fwd_inv(bq, m, r):
+    torch = H.torch()
+    rng = np.random.default_rng(m + r)
+    theta = wl.uniform_angles(rng, m)
+    O = wl.random_orthogonal(rng, r)
+    x = rng.standard_normal((13, m * r)).astype(np.float32)
+    layer = make_layer(bq, theta, O)
+    y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+    ref = ob.kron_forward(theta, O.astype(np.float64), x.astype(np.float64), m)
+    H.assert_f32_close(H.host(y), ref, x.astype(np.float64))
+    xb = torch.empty_like(y)
+    bq.bq_butterfly_inv(layer, y, xb)
+    torch.cuda.synchronize()
+    ref_inv = ob.kron_inverse(theta, O.astype(np.float64), H.host(y).astype(np.float64), m)
+    H.assert_f32_close(H.host(xb), ref_inv, x.astype(np.float64))
+
+
+def test_bf16_io(bq):
+    torch = H.torch()
+    w = wl.act_4096(rows=24)
+    layer = make_layer(bq, w.theta)
+    x = H.dev_bf16_bits(w.x)
+    xf = H.input_f64(w.x, "bf16")
+    ref = ob.forward(w.theta, xf)
+    y32 = run_fwd(bq, layer, x, torch.float32)
+    H.assert_f32_close(H.host(y32), ref, xf)
+    y16 = run_fwd(bq, layer, x, torch.bfloat16)
+    H.assert_bf16_within_ulp(H.host(y16), ref)
+    # in place, bf16 -> bf16
+    xi = x.clone()
+    bq.bq_butterfly_fwd(layer, xi, xi)
+    torch.cuda.synchronize()
+    assert torch.equal(xi.view(torch.int16), y16.view(torch.int16))
+    # inverse from bf16 back to fp32
+    back = torch.empty((24, 4096), dtype=torch.float32, device="cuda")
+    bq.bq_butterfly_inv(layer, y16, back)
+    torch.cuda.synchronize()
+    H.assert_f32_close(H.host(back), ob.inverse(w.theta, H.input_f64(H.host(y16), "bf16")), xf)
+
+
+def test_zero_angles_is_exact_identity(bq):
+    torch = H.torch()
+    for m in (8, 256, 4096):
+        theta = np.zeros((m.bit_length() - 1, m // 2), np.float32)
+        x = np.random.default_rng(m).standard_normal((5, m)).astype(np.float32)
+        y = run_fwd(bq, make_layer(bq, theta), H.dev_f32(x), torch.float32)
+        assert np.array_equal(H.host(y), x)
+
+
+def test_hadamard_angles_match_fwht(bq):
+    scipy_linalg = pytest.importorskip("scipy.linalg")
+    torch = H.torch()
+    for m in (16, 1024):
+        L = m.bit_length() - 1
+        theta = np.full((L, m // 2), np.pi / 4, np.float32)
+        x = np.random.default_rng(1).standard_normal((4, m)).astype(np.float32)
+        y = run_fwd(bq, make_layer(bq, theta), H.dev_f32(x), torch.float32)
+        d = np.array([1.0])
+        for _ in range(L):
+            d = np.kron(d, [1.0, -1.0])
+        Hm = scipy_linalg.hadamard(m) * d[None, :] / np.sqrt(m)   # Q = H diag(d) / sqrt(n)
+        H.assert_f32_close(H.host(y), x.astype(np.float64) @ Hm.T, x.astype(np.float64), tol=1e-5)
+
+
+def test_tiny_workload(bq):
+    """n = 256: Qx, Q^T(Qx), W Q^T then 2-bit RTN in groups of 64."""
+    torch = H.torch()
+    w = wl.tiny()
+    layer = make_layer(bq, w.theta)
+    y = run_fwd(bq, layer, H.dev_f32(w.x), torch.float32)
+    H.assert_f32_close(H.host(y), ob.forward(w.theta, w.x.astype(np.float64)), w.x.astype(np.float64))
+    xb = torch.empty_like(y)
+    bq.bq_butterfly_inv(layer, y, xb)
+    torch.cuda.synchronize()
+    H.assert_f32_close(H.host(xb), w.x.astype(np.float64), w.x.astype(np.float64))
+    check_quant(bq, layer, H.dev_f32(w.w), w.w.astype(np.float64), w.theta, 2, 64, weight=True)
+
+
+# --------------------------------------------------------------------------- quantization
+
+def check_quant(bq, layer, x_dev, x_f64, theta, bits, group, weight=False, O=None, m=None, sample=None):
+    """Bit-exact against the oracle quantizer on the GPU's float32 output; end to end
+    against the float64 oracle within one level on at most 1e-4 of the entries."""
+    torch = H.torch()
+    rows = x_dev.shape[0]
+    n = x_dev.shape[1]
+    codes, scale, zero = bq.quant_outputs(rows, n, bits, group, "cuda")
+    fn = bq.bq_weight_rotate_pack if weight else bq.bq_transform_quantize
+    fn(layer, x_dev, bits, group, codes, scale, zero)
+    y32 = run_fwd(bq, layer, x_dev, torch.float32)
+    torch.cuda.synchronize()
+    idx = np.arange(rows) if sample is None else sample
+    y_gpu = H.host(y32)[idx]
+    c_gpu, s_gpu, z_gpu = H.host(codes)[idx], H.host(scale)[idx].view(np.uint16), H.host(zero)[idx].view(np.uint16)
+    c_ref, s_ref, z_ref = oq.quantize_pack(y_gpu, bits, group)
+    assert np.array_equal(s_gpu, s_ref), "scales differ from the oracle quantizer on identical input"
+    assert np.array_equal(z_gpu, z_ref), "zero points differ from the oracle quantizer on identical input"
+    assert np.array_equal(c_gpu, c_ref), "codes differ from the oracle quantizer on identical input"
+    # end to end against the float64 transform
+    xs = x_f64[idx]
+    ref = ob.forward(theta, xs) if O is None else ob.kron_forward(theta, O, xs, m)
+    H.assert_f32_close(y_gpu, ref, xs)
+    q_e2e, _, _ = oq.quantize_codes(ref.astype(np.float32), bits, group)
+    q_gpu = oq.unpack(c_gpu, bits, n)
+    d = H.ordered_diff_codes(q_gpu, q_e2e)
+    assert d.max() <= 1 and (d > 0).mean() <= 1e-4, f"end-to-end code mismatch: max {d.max()}, frac {(d > 0).mean()}"
+    return c_gpu
+
+
+@pytest.mark.parametrize("bits,group", [(4, 128), (2, 128), (4, 64), (2, 64), (4, 32), (2, 32), (4, 256), (2, 256)])
+def test_quant_settings_small(bq, bits, group):
+    rng = np.random.default_rng(bits * 1000 + group)
+    m = 1024
+    theta = wl.uniform_angles(rng, m)
+    x = (rng.standard_normal((19, m)) * 3).astype(np.float32)
+    layer = make_layer(bq, theta)
+    check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, bits, group)
+
+
+def test_quant_degenerate_groups(bq):
+    """theta = 0 keeps a constant row constant: every group takes the hi == lo branch."""
+    torch = H.torch()
+    m = 256
+    theta = np.zeros((8, 128), np.float32)
+    x = np.full((3, m), 1.75, np.float32)
+    x[1] = 0.0
+    x[2, :64] = -3.0
+    layer = make_layer(bq, theta)
+    codes, scale, zero = bq.quant_outputs(3, m, 4, 64, "cuda")
+    bq.bq_transform_quantize(layer, H.dev_f32(x), 4, 64, codes, scale, zero)
+    torch.cuda.synchronize()
+    c_ref, s_ref, z_ref = oq.quantize_pack(x, 4, 64)
+    assert np.array_equal(H.host(codes), c_ref)
+    assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
+    assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
+
+
+def test_weight_side_matches_activation_side(bq):
+    torch = H.torch()
+    w = wl.weight_4096(rows=40)
+    layer = make_layer(bq, w.theta)
+    x = H.dev_bf16_bits(w.w)
+    a = bq.quant_outputs(40, 4096, 2, 128, "cuda")
+    b = bq.quant_outputs(40, 4096, 2, 128, "cuda")
+    bq.bq_transform_quantize(layer, x, 2, 128, *a)
+    bq.bq_weight_rotate_pack(layer, x, 2, 128, *b)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+# --------------------------------------------------------------------------- full workload sizes
+
+def _sample(rows, k, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, rows - 1], rng.choice(rows, size=k, replace=False)]))
+
+
+def test_full_act_4096_int4(bq):
+    w = wl.act_4096()
+    layer = make_layer(bq, w.theta)
+    check_quant(bq, layer, H.dev_bf16_bits(w.x), H.input_f64(w.x, "bf16"), w.theta, 4, 128,
+                sample=_sample(2048, 96, 1))
+
+
+def test_full_weight_4096_int2(bq):
+    w = wl.weight_4096()
+    layer = make_layer(bq, w.theta)
+    check_quant(bq, layer, H.dev_bf16_bits(w.w), H.input_f64(w.w, "bf16"), w.theta, 2, 128, weight=True,
+                sample=_sample(11008, 96, 2))
+
+
+def test_full_act_5120_kron_int4(bq):
+    w = wl.act_5120()
+    layer = make_layer(bq, w.theta, w.O)
+    check_quant(bq, layer, H.dev_bf16_bits(w.x), H.input_f64(w.x, "bf16"), w.theta, 4, 128,
+                O=w.O.astype(np.float64), m=w.m, sample=_sample(8192, 64, 3))
+
+
+# --------------------------------------------------------------------------- backward
+
+def run_bwd(bq, layers, x_dev, dy_dev, y_dtype):
+    torch = H.torch()
+    nl, rows, m = x_dev.shape
+    y = torch.empty((nl, rows, m), dtype=y_dtype, device="cuda")
+    dx = torch.empty((nl, rows, m), dtype=torch.float32, device="cuda")
+    L = m.bit_length() - 1
+    dth = torch.empty((nl, L * m // 2), dtype=torch.float32, device="cuda")
+    ws = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, nl, rows), dtype=torch.uint8, device="cuda")
+    bq.bq_butterfly_bwd(layers, x_dev, y, dy_dev, dx, dth, ws)
+    torch.cuda.synchronize()
+    return y, dx, dth
+
+
+def check_dtheta(dth_gpu, dth_ref, A):
+    bound = 2e-4 * A + 1e-6 * A.max()
+    err = np.abs(dth_gpu - dth_ref)
+    assert np.all(err <= bound), f"dtheta error {err.max():.3e} (bound at worst {bound.ravel()[np.argmax(err - bound)]:.3e})"
+
+
+@pytest.mark.parametrize("m,layers,rows", [(8, 1, 5), (16, 3, 7), (64, 2, 33), (256, 4, 50), (4096, 2, 9)])
+def test_bwd_small(bq, m, layers, rows):
+    torch = H.torch()
+    rng = np.random.default_rng(m + layers + rows)
+    thetas = [wl.uniform_angles(rng, m) for _ in range(layers)]
+    x = rng.standard_normal((layers, rows, m)).astype(np.float32)
+    dy = rng.standard_normal((layers, rows, m)).astype(np.float32)
+    L = [make_layer(bq, t) for t in thetas]
+    y, dx, dth = run_bwd(bq, L, H.dev_f32(x), H.dev_f32(dy), torch.float32)
+    for l in range(layers):
+        xr, dyr = x[l].astype(np.float64), dy[l].astype(np.float64)
+        yr, dxr, dthr = ob.backward(thetas[l], xr, dyr)
+        H.assert_f32_close(H.host(y)[l], yr, xr)
+        H.assert_f32_close(H.host(dx)[l], dxr, dyr)
+        check_dtheta(H.host(dth)[l].reshape(dthr.shape), dthr, ob.backward_abs_scale(thetas[l], xr, dyr))
+    # bitwise reproducible
+    _, dx2, dth2 = run_bwd(bq, L, H.dev_f32(x), H.dev_f32(dy), torch.float32)
+    assert torch.equal(dth, dth2) and torch.equal(dx, dx2)
+
+
+def test_bwd_bf16_io(bq):
+    torch = H.torch()
+    w = wl.backward_layer_host(0, 300, m=4096)
+    layer = make_layer(bq, w.theta)
+    x = H.dev_bf16_bits(w.x)[None]
+    dy = H.dev_f32(w.dy)[None]
+    y, dx, dth = run_bwd(bq, [layer], x, dy, torch.bfloat16)
+    xf = H.input_f64(w.x, "bf16")
+    yr, dxr, dthr = ob.backward(w.theta, xf, w.dy.astype(np.float64))
+    H.assert_bf16_within_ulp(H.host(y)[0], yr)
+    H.assert_f32_close(H.host(dx)[0], dxr, w.dy.astype(np.float64))
+    check_dtheta(H.host(dth)[0].reshape(dthr.shape), dthr, ob.backward_abs_scale(w.theta, xf, w.dy.astype(np.float64)))
