@@ -107,12 +107,13 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_id: str):
         self.proc = None
+        self.raw = ""
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", str(gpu_index),
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-i", gpu_id,
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True)
         except (OSError, FileNotFoundError):
             self.proc = None
 
@@ -121,10 +122,11 @@ class ClockSampler:
             return None
         self.proc.terminate()
         try:
-            out, _ = self.proc.communicate(timeout=5)
+            out, err = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-            out, _ = self.proc.communicate()
+            out, err = self.proc.communicate()
+        self.raw = (out or "")[-2000:] + (err or "")[-500:]
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in out.strip().splitlines():
@@ -139,8 +141,18 @@ class ClockSampler:
                 if v.lower().startswith("active"):
                     reasons.add(nm)
         if not sm:
-            return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+            return {"error": "no nvidia-smi samples", "raw": self.raw[-300:]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm),
+                "window": "from 0.5 s of continuous steps before the timed region to its end"}
+
+
+def gpu_id_for(device) -> str:
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(device).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(device.index if hasattr(device, "index") else 0)
 
 
 def cpu_oracle_rate(w, rows_target_s: float, max_rows: int):
@@ -210,10 +222,18 @@ def run_ours(args, spec, rank, world, local_rank):
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    # the clock sampler needs more time than the timed region takes: keep the GPU
+    # busy with identical steps for 0.5 s while it starts
+    sampler = ClockSampler(gpu_id_for(dev))
+    t_busy = time.perf_counter()
+    while time.perf_counter() - t_busy < 0.5:
+        for _ in range(20):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    sampler = ClockSampler(local_rank)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     wall0 = time.perf_counter()
     for s, e in evs:

@@ -36,6 +36,8 @@ bq_status transform(const bq_layer* layer, const void* x, bq_dtype xt, void* y, 
   if (rows == 0) return BQ_OK;
   if (x == y && xt != yt) return BQ_ERR_INVALID_ARG;
   const KLayer L = make_klayer(*layer);
+  if (!inverse && fast4096_supports(L, nullptr))
+    return launch_fast4096(L, x, xt, y, yt, rows, nullptr, static_cast<cudaStream_t>(stream));
   return launch_generic(L, x, xt, y, yt, rows, inverse, nullptr, static_cast<cudaStream_t>(stream));
 }
 
@@ -52,6 +54,8 @@ bq_status quantize(const bq_layer* layer, const void* x, bq_dtype xt, int64_t ro
   if (!aligned16(x) || !aligned16(codes) || !aligned16(scale) || !aligned16(zero)) return BQ_ERR_INVALID_ARG;
   const KLayer L = make_klayer(*layer);
   QuantArgs q{bits, group, codes, scale, zero};
+  if (fast4096_supports(L, &q))
+    return launch_fast4096(L, x, xt, nullptr, BQ_F32, rows, &q, static_cast<cudaStream_t>(stream));
   return launch_generic(L, x, xt, nullptr, BQ_F32, rows, false, &q, static_cast<cudaStream_t>(stream));
 }
 

@@ -23,10 +23,16 @@ constexpr int kMaxGroup = 256;     // largest quantization group
 //   fast   [L][m]      per-position coefficient of the scaled form: at stage s
 //                      position i is updated as a_i += fast[s][i] * a_{i ^ 2^s}
 //   sigma  [m]         per-position output scale of the scaled form
+//   image  [128][416]  (m == 4096 only) tensor-memory image of the specialised
+//                      n = 4096 kernel: lane t, column c holds the coefficient
+//                      thread t needs at that column (see bq_fast4096.cu)
 struct TableLayout {
   int m, L;
-  size_t off_cs, off_fast, off_sigma, total;
+  size_t off_cs, off_fast, off_sigma, off_image, total;
 };
+
+constexpr int kImageLanes = 128;
+constexpr int kImageCols = 416;
 
 __host__ __device__ inline int ilog2(int v) {
   int l = 0;
@@ -43,7 +49,8 @@ __host__ __device__ inline TableLayout table_layout(int m) {
   t.off_cs = 16;
   t.off_fast = t.off_cs + round4(size_t(t.L) * m);
   t.off_sigma = t.off_fast + round4(size_t(t.L) * m);
-  t.total = t.off_sigma + round4(size_t(m));
+  t.off_image = t.off_sigma + round4(size_t(m));
+  t.total = t.off_image + (m == 4096 ? size_t(kImageLanes) * kImageCols : 0);
   return t;
 }
 
@@ -54,6 +61,7 @@ struct KLayer {
   const float* fast;    // [L][m]
   const float* sigma;   // [m]
   const float* hdr;     // header (flag at hdr[0])
+  const float* image;   // tensor-memory image (m == 4096) or nullptr
   const float* O;       // [r][r] or nullptr
 };
 
@@ -65,6 +73,7 @@ inline KLayer make_klayer(const bq_layer& l) {
   k.fast = l.table + t.off_fast;
   k.sigma = l.table + t.off_sigma;
   k.hdr = l.table;
+  k.image = l.m == 4096 ? l.table + t.off_image : nullptr;
   k.O = l.O;
   return k;
 }
@@ -78,6 +87,9 @@ struct QuantArgs {
 
 // Launchers (defined in the .cu files).  Each returns BQ_OK or BQ_ERR_CUDA.
 bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t st);
+bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
+                          const QuantArgs* q, cudaStream_t st);
+bool fast4096_supports(const KLayer& L, const QuantArgs* q);
 bq_status launch_generic(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt,
                          int64_t rows, bool inverse, const QuantArgs* q, cudaStream_t st);
 bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt,

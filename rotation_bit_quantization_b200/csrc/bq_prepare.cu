@@ -76,6 +76,54 @@ __global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ t
   }
 }
 
+// Position held in register slot e by thread t of a 128-thread row group, for
+// the three passes of the specialised n = 4096 kernel (see bq_fast4096.cu).
+__device__ __forceinline__ int pos_pass(int pass, int t, int e) {
+  if (pass == 0) return t * 32 + e;
+  if (pass == 1) return (t & 31) | (e << 5) | ((t >> 5) << 10);
+  return (e & 7) | (t << 3) | ((e >> 3) << 10);
+}
+
+// Tensor-memory image of the n = 4096 kernel: lane t, column c.
+//   columns [0,160):   pass 0 stages 0..4   (32 columns per stage)
+//   columns [160,320): pass 1 stages 5..9
+//   columns [320,384): pass 2 stages 10, 11
+//   columns [384,416): output scale of the 32 positions thread t ends with
+// Inside a stage block, column 4q + e (e = 0, 1) is the coefficient of the low
+// element of the thread's (2q + e)-th pair and column 4q + 2 + e that of its
+// high element: (alpha, beta) of the scaled form, or (cos, sin) when the
+// scaled form is out of range (header flag 0; the output scale is then 1).
+__global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= kImageLanes * kImageCols) return;
+  const int t = idx / kImageCols, col = idx % kImageCols;
+  const bool scaled = table[0] == 1.f;
+  const float2* cs = reinterpret_cast<const float2*>(table + tl.off_cs);
+  const float* fast = table + tl.off_fast;
+  const float* sigma = table + tl.off_sigma;
+  float v;
+  if (col >= 384) {
+    v = scaled ? sigma[pos_pass(2, t, col - 384)] : 1.f;
+  } else {
+    int pass, stage, sb;
+    if (col < 160) { pass = 0; stage = col / 32; sb = stage; }
+    else if (col < 320) { pass = 1; stage = 5 + (col - 160) / 32; sb = stage - 5; }
+    else { pass = 2; stage = 10 + (col - 320) / 32; sb = stage - 7; }
+    const int w = col & 31, q = w >> 2, high = (w >> 1) & 1, e = w & 1;
+    const int k = 2 * q + e;
+    const int j = ((k >> sb) << (sb + 1)) | (k & ((1 << sb) - 1));
+    const int low = pos_pass(pass, t, j);
+    if (scaled) {
+      v = fast[size_t(stage) * tl.m + (high ? pos_pass(pass, t, j | (1 << sb)) : low)];
+    } else {
+      const int p = ((low >> (stage + 1)) << stage) | (low & ((1 << stage) - 1));
+      const float2 c = cs[size_t(stage) * (tl.m >> 1) + p];
+      v = high ? c.y : c.x;
+    }
+  }
+  table[tl.off_image + idx] = v;
+}
+
 }  // namespace
 
 bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t st) {
@@ -86,6 +134,10 @@ bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t s
       return BQ_ERR_CUDA;
   }
   k_prepare<<<1, 1024, smem, st>>>(theta, table, tl);
+  if (m == 4096) {
+    const int total = kImageLanes * kImageCols;
+    k_image4096<<<(total + 255) / 256, 256, 0, st>>>(table, tl);
+  }
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 

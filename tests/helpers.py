@@ -2,7 +2,9 @@
 
 Comparison rules (per the accuracy bounds of the transform path):
 * float32 outputs: per row, max |y_gpu - y_oracle| <= 2e-5 * ||x||_2;
-* bfloat16 outputs: the GPU value is RN(oracle) or one of its bf16 neighbours;
+* bfloat16 outputs: bitwise the round-to-nearest-even of the GPU's own float32
+  output, and within one bf16 ulp of the oracle plus the float32 bound (a
+  literal one-ulp bound is unreachable for elements much smaller than 2e-5 ||x||);
 * quantized codes, scales and zero points computed from identical float32
   inputs are bit-exact; end to end, codes may differ by one level in at most
   1e-4 of the entries;
@@ -58,11 +60,23 @@ def _ordered(bits):
     return np.where(b & 0x8000, -(b & 0x7FFF), b)
 
 
-def assert_bf16_within_ulp(bits_gpu, y_ref):
+def bf16_ulp(v):
+    v = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def assert_bf16_output(bits_gpu, y32_gpu, y_ref, x_ref, tol=F32_TOL):
+    """bf16 output = RN(GPU float32 output) bitwise; |bf16 - oracle| <= ulp(oracle) + tol * ||x||."""
+    bits_gpu = np.asarray(bits_gpu, np.uint16).reshape(y_ref.shape)
+    assert np.array_equal(bits_gpu, wl.bf16_bits_from_f32(np.asarray(y32_gpu, np.float32).reshape(y_ref.shape))), \
+        "bf16 output is not the rounding of the float32 output"
+    v = wl.f32_from_bf16_bits(bits_gpu).astype(np.float64)
+    bound = bf16_ulp(y_ref) + tol * np.linalg.norm(x_ref, axis=-1, keepdims=True)
+    err = np.abs(v - y_ref)
+    assert np.all(err <= bound), f"bf16 error {err.max():.3e} above bound"
     ref_bits = wl.bf16_bits_from_f32(np.asarray(y_ref, np.float64).astype(np.float32))
-    d = np.abs(_ordered(np.asarray(bits_gpu, np.uint16).reshape(ref_bits.shape)) - _ordered(ref_bits))
-    assert d.max() <= 1, f"bf16 off by {d.max()} ulp"
-    return float((d > 0).mean())
+    return float((np.abs(_ordered(bits_gpu) - _ordered(ref_bits)) > 1).mean())
 
 
 def ordered_diff_codes(a, b):

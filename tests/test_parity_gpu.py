@@ -87,7 +87,7 @@ def test_bf16_io(bq):
     y32 = run_fwd(bq, layer, x, torch.float32)
     H.assert_f32_close(H.host(y32), ref, xf)
     y16 = run_fwd(bq, layer, x, torch.bfloat16)
-    H.assert_bf16_within_ulp(H.host(y16), ref)
+    H.assert_bf16_output(H.host(y16), H.host(y32), ref, xf)
     # in place, bf16 -> bf16
     xi = x.clone()
     bq.bq_butterfly_fwd(layer, xi, xi)
@@ -287,8 +287,52 @@ def test_bwd_bf16_io(bq):
     x = H.dev_bf16_bits(w.x)[None]
     dy = H.dev_f32(w.dy)[None]
     y, dx, dth = run_bwd(bq, [layer], x, dy, torch.bfloat16)
+    y32, _, _ = run_bwd(bq, [layer], x, dy, torch.float32)
     xf = H.input_f64(w.x, "bf16")
     yr, dxr, dthr = ob.backward(w.theta, xf, w.dy.astype(np.float64))
-    H.assert_bf16_within_ulp(H.host(y)[0], yr)
+    H.assert_bf16_output(H.host(y)[0], H.host(y32)[0], yr, xf)
     H.assert_f32_close(H.host(dx)[0], dxr, w.dy.astype(np.float64))
     check_dtheta(H.host(dth)[0].reshape(dthr.shape), dthr, ob.backward_abs_scale(w.theta, xf, w.dy.astype(np.float64)))
+
+
+# --------------------------------------------------------------------------- specialised n = 4096 kernel
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (2, 64), (4, 128), (2, 128), (4, 256), (2, 256), (4, 32)])
+@pytest.mark.parametrize("rows", [1, 2, 5, 37])
+def test_quant_4096_groups_and_ragged_rows(bq, bits, group, rows):
+    rng = np.random.default_rng(bits * 7 + group + rows)
+    theta = wl.uniform_angles(rng, 4096)
+    x = (rng.standard_t(3, (rows, 4096)) * 0.5).astype(np.float32)
+    layer = make_layer(bq, theta)
+    check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, bits, group)
+
+
+def test_fallback_when_scaled_form_out_of_range(bq):
+    """Angles at the float32 value nearest pi/2 drive the scaled form's scales below 2^-60:
+    the n = 4096 kernel must switch to the plain cos/sin rotation."""
+    torch = H.torch()
+    theta = np.full((12, 2048), np.float32(np.pi / 2), np.float32)
+    theta[:, ::3] = np.float32(0.3)
+    layer = make_layer(bq, theta)
+    assert not layer.fast_form
+    x = np.random.default_rng(0).standard_normal((9, 4096)).astype(np.float32)
+    y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+    H.assert_f32_close(H.host(y), ob.forward(theta, x.astype(np.float64)), x.astype(np.float64))
+    check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, 4, 128)
+
+
+def test_scaled_form_is_used_for_uniform_angles(bq):
+    for cfg in (wl.act_4096(rows=1), wl.weight_4096(rows=1)):
+        assert make_layer(bq, cfg.theta).fast_form
+
+
+def test_many_rows_all_grid_slots(bq):
+    """More rows than row groups of one wave, odd total: every slot runs pairs and a tail."""
+    torch = H.torch()
+    rng = np.random.default_rng(5)
+    theta = wl.uniform_angles(rng, 4096)
+    rows = 148 * 4 * 3 + 7
+    x = rng.standard_normal((rows, 4096)).astype(np.float32)
+    y = run_fwd(bq, make_layer(bq, theta), H.dev_f32(x), torch.float32)
+    idx = _sample(rows, 64, 9)
+    H.assert_f32_close(H.host(y)[idx], ob.forward(theta, x[idx].astype(np.float64)), x[idx].astype(np.float64))
