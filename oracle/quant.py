@@ -17,7 +17,8 @@ that codes, scales and zero points can be compared bit for bit:
    uses s = float32(scale16) so that dequantizing from the stored values is
    self-consistent;
 4. degenerate groups: if hi == lo or s == 0 (fp16 underflow), s = 1.0;
-   z = clamp(rint(-lo / s), 0, qmax);  q = clamp(rint(x / s) + z, 0, qmax);
+   z = clamp(rint(-lo / s), 0, qmax), an integer stored as fp16 (a zero
+   point of 0 is +0.0);  q = clamp(rint(x / s) + z, 0, qmax);
    rint rounds half to even; the divisions are IEEE float32 divisions (never a
    reciprocal multiply);
 5. packing is little-endian inside a byte, lowest element index in the lowest
@@ -59,7 +60,9 @@ def group_params(y32, bits: int, group: int):
     degenerate = (hi == lo) | (s == np.float32(0))
     s = np.where(degenerate, np.float32(1.0), s).astype(np.float32)
     scale16 = np.where(degenerate, np.float16(1.0), scale16).astype(np.float16)
-    z = np.clip(np.rint(-lo / s), np.float32(0), qmax).astype(np.float32)
+    # the zero point is an integer; +0.0 makes a zero point of 0 encode as +0
+    # (rint(-lo/s) of lo = 0 is -0.0, which the clamp may pass through)
+    z = (np.clip(np.rint(-lo / s), np.float32(0), qmax) + np.float32(0)).astype(np.float32)
     return scale16.view(np.uint16), z.astype(np.float16).view(np.uint16), s, z
 
 

@@ -354,6 +354,13 @@ def test_quant_degenerate_and_underflow():
     assert s2.view(np.float16)[0, 0] == 1.0
 
 
+def test_zero_point_zero_is_positive_zero():
+    # lo = 0 gives rint(-0/s) = -0.0; the zero point is the integer 0, encoded +0
+    y = np.array([[0.0, 1.0, 2.0, 3.0], [0.0, 0.0, 0.0, 0.0]], dtype=np.float32)
+    _, _, z16 = oq.quantize_codes(y, 2, 4)
+    assert z16.tolist() == [[0], [0]]
+
+
 def test_pack_layout():
     c4 = np.array([[1, 2, 15, 0]], dtype=np.uint8)
     assert oq.pack(c4, 4).tolist() == [[0x21, 0x0F]]
