@@ -239,7 +239,46 @@ __device__ __forceinline__ int bitrev(int k) {
   return r;
 }
 
+__device__ __forceinline__ float min3(float a, float b, float c) {
+  float d;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Codes of 8 values by IEEE division, for sets where the fast path below cannot
+// prove its result (kept out of line: it runs for roughly one set in 10^4).
+template <int BITS>
+__device__ __noinline__ uint32_t codes_by_division(float y0, float y1, float y2, float y3, float y4, float y5,
+                                                    float y6, float y7, float s, float z) {
+  const float qmax = static_cast<float>((1 << BITS) - 1);
+  const float y[8] = {y0, y1, y2, y3, y4, y5, y6, y7};
+  uint32_t word = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float t = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(y[e], s)), z), 0.f), qmax);
+    word |= static_cast<uint32_t>(t) << (BITS * e);
+  }
+  return word;
+}
+
 // Per-group asymmetric RTN of the R rows held in pass-C layout, packing and stores.
+//
+// Codes are q = clamp(rint(y / s) + z, 0, qmax) with y / s the correctly rounded
+// float32 quotient.  Fast path: v = y * inv with inv = 1 / s correctly rounded,
+// so |v - y/s| <= 2^-23 |y/s| and |v - RN(y/s)| <= 1.5 * 2^-23 |y/s|.  When v is
+// farther than vmax * 2^-20 from every half-integer (vmax bounds |v| over the
+// group; the factor 2^-20 also absorbs the rounding of the threshold itself),
+// RN(y/s) lies on the same side of the same half-integer and
+// rint(RN(y/s)) = rint(v) exactly.  rint(v) is
+// taken with the float32 magic constant 1.5 * 2^23 (round-half-even addition),
+// whose bit pattern then carries the integer, so adding z and clamping happen
+// on integers.  A set of 8 values with any element too close to a tie (or with
+// |v| >= 2^22) is redone with IEEE division.
 template <int BITS, int GLANES, int R>
 __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const FastArgs& A, long long row0, int tau,
                                                int lane) {
@@ -248,19 +287,15 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
   constexpr int LOGG = clog2<0>(GLANES);  // lanes sharing one group
   constexpr int GROUP = 8 * GLANES;
   constexpr int GPR = M / GROUP;          // groups per row
-  const float qmax = static_cast<float>((1 << BITS) - 1);
+  constexpr int QMAX = (1 << BITS) - 1;
+  const float qmax = static_cast<float>(QMAX);
   float mn[S], mx[S];
 #pragma unroll
   for (int k = 0; k < S; ++k) {
     const int r = k >> 2, h = k & 3;
-    float lo = fminf(a[r][4 * h].x, a[r][4 * h].y), hi = fmaxf(a[r][4 * h].x, a[r][4 * h].y);
-#pragma unroll
-    for (int q = 1; q < 4; ++q) {
-      lo = fminf(lo, fminf(a[r][4 * h + q].x, a[r][4 * h + q].y));
-      hi = fmaxf(hi, fmaxf(a[r][4 * h + q].x, a[r][4 * h + q].y));
-    }
-    mn[k] = lo;
-    mx[k] = hi;
+    const float2 p0 = a[r][4 * h], p1 = a[r][4 * h + 1], p2 = a[r][4 * h + 2], p3 = a[r][4 * h + 3];
+    mn[k] = fminf(min3(p0.x, p0.y, p1.x), min3(p1.y, p2.x, min3(p2.y, p3.x, p3.y)));
+    mx[k] = fmaxf(max3(p0.x, p0.y, p1.x), max3(p1.y, p2.x, max3(p2.y, p3.x, p3.y)));
   }
   // recursive halving over lane bits 0..LOGS-1: afterwards lane l holds set bitrev(l & (S-1))
 #pragma unroll
@@ -287,7 +322,11 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
     s = 1.f;
     h16 = __float2half_rn(1.f);
   }
-  const float z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax);
+  const float z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax), 0.f);  // +0 for a zero point of 0
+  const float inv = __fdiv_rn(1.f, s);
+  // tie margin for the whole group: every |v| <= max(|lo|, |hi|) * inv * (1 + 2^-22)
+  const float vmax = fmaxf(fabsf(lo), fabsf(hi)) * inv * 1.000001f;
+  const float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
   {
     const int k = bitrev<S>(lane & (S - 1));
     if (((lane >> LOGS) & ((1 << (LOGG - LOGS)) - 1)) == 0) {
@@ -297,20 +336,36 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
       A.zero[row * GPR + g] = __half_as_ushort(__float2half_rn(z));
     }
   }
+  const float kMagic = 12582912.f;  // 1.5 * 2^23
 #pragma unroll
   for (int k = 0; k < S; ++k) {
     const int src = (lane & ~(S - 1)) | bitrev<S>(k);
+    const float invk = __shfl_sync(0xffffffffu, inv, src);
+    const float thrk = __shfl_sync(0xffffffffu, thr, src);
+    const int zk = static_cast<int>(__shfl_sync(0xffffffffu, z, src));
     const float sk = __shfl_sync(0xffffffffu, s, src);
-    const float zk = __shfl_sync(0xffffffffu, z, src);
     const int r = k >> 2, h = k & 3;
+    const float2 iv = make_float2(invk, invk), mg = make_float2(kMagic, kMagic);
+    const float2 nmg = make_float2(-kMagic, -kMagic), neg1 = make_float2(-1.f, -1.f);
+    bool exact = true;
     uint32_t word = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float v0 = a[r][4 * h + q].x, v1 = a[r][4 * h + q].y;
-      const float t0 = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v0, sk)), zk), 0.f), qmax);
-      const float t1 = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(v1, sk)), zk), 0.f), qmax);
-      word |= static_cast<uint32_t>(t0) << (BITS * (2 * q));
-      word |= static_cast<uint32_t>(t1) << (BITS * (2 * q + 1));
+      const float2 v = __fmul2_rn(a[r][4 * h + q], iv);
+      const float2 t = __fadd2_rn(v, mg);
+      const float2 e = __ffma2_rn(__fadd2_rn(t, nmg), neg1, v);  // v - rint(v), exact
+      exact = exact && fabsf(e.x) < thrk && fabsf(e.y) < thrk;
+      int c0 = static_cast<int>(__float_as_uint(t.x)) - 0x4B400000 + zk;
+      int c1 = static_cast<int>(__float_as_uint(t.y)) - 0x4B400000 + zk;
+      c0 = min(max(c0, 0), QMAX);
+      c1 = min(max(c1, 0), QMAX);
+      word |= static_cast<uint32_t>(c0) << (BITS * (2 * q));
+      word |= static_cast<uint32_t>(c1) << (BITS * (2 * q + 1));
+    }
+    if (!exact) {
+      word = codes_by_division<BITS>(a[r][4 * h].x, a[r][4 * h].y, a[r][4 * h + 1].x, a[r][4 * h + 1].y,
+                                     a[r][4 * h + 2].x, a[r][4 * h + 2].y, a[r][4 * h + 3].x, a[r][4 * h + 3].y,
+                                     sk, static_cast<float>(zk));
     }
     const long long row = row0 + r;
     if constexpr (BITS == 4) {
@@ -470,19 +525,44 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
   {
+    // each thread copies its lane's share of the image: two batches of loads in
+    // flight, then the tensor-memory stores
     const float4* src = reinterpret_cast<const float4*>(A.image + tau * kImageCols + slot * kFillPerSlot);
-#pragma unroll 1
-    for (int c = 0; c < kFillPerSlot; c += 16) {
-      uint32_t v[16];
+    constexpr int kChunks = kFillPerSlot / 16;  // 13 chunks of 16 columns
+    constexpr int kFirst = 7;
+    {
+      float4 f[kFirst * 4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 f = src[c / 4 + i];
-        v[4 * i] = __float_as_uint(f.x);
-        v[4 * i + 1] = __float_as_uint(f.y);
-        v[4 * i + 2] = __float_as_uint(f.z);
-        v[4 * i + 3] = __float_as_uint(f.w);
+      for (int i = 0; i < kFirst * 4; ++i) f[i] = src[i];
+#pragma unroll
+      for (int c = 0; c < kFirst; ++c) {
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[4 * i] = __float_as_uint(f[4 * c + i].x);
+          v[4 * i + 1] = __float_as_uint(f[4 * c + i].y);
+          v[4 * i + 2] = __float_as_uint(f[4 * c + i].z);
+          v[4 * i + 3] = __float_as_uint(f[4 * c + i].w);
+        }
+        tmem_st16(tb + slot * kFillPerSlot + 16 * c, v);
       }
-      tmem_st16(tb + slot * kFillPerSlot + c, v);
+    }
+    {
+      float4 f[(kChunks - kFirst) * 4];
+#pragma unroll
+      for (int i = 0; i < (kChunks - kFirst) * 4; ++i) f[i] = src[kFirst * 4 + i];
+#pragma unroll
+      for (int c = 0; c < kChunks - kFirst; ++c) {
+        uint32_t v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[4 * i] = __float_as_uint(f[4 * c + i].x);
+          v[4 * i + 1] = __float_as_uint(f[4 * c + i].y);
+          v[4 * i + 2] = __float_as_uint(f[4 * c + i].z);
+          v[4 * i + 3] = __float_as_uint(f[4 * c + i].w);
+        }
+        tmem_st16(tb + slot * kFillPerSlot + 16 * (kFirst + c), v);
+      }
     }
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
   }

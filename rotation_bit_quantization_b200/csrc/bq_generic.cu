@@ -139,7 +139,7 @@ __device__ void quant_row(const float* buf, int n, const QuantArgs& qa, long lon
       s = 1.f;
       h = __float2half_rn(1.f);
     }
-    const float z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax);
+    const float z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax), 0.f);  // +0 for a zero point of 0
     uint32_t word = 0;
 #pragma unroll
     for (int c = 0; c < 8; ++c) {

@@ -336,3 +336,35 @@ def test_many_rows_all_grid_slots(bq):
     y = run_fwd(bq, make_layer(bq, theta), H.dev_f32(x), torch.float32)
     idx = _sample(rows, 64, 9)
     H.assert_f32_close(H.host(y)[idx], ob.forward(theta, x[idx].astype(np.float64)), x[idx].astype(np.float64))
+
+
+def test_quant_exact_ties_and_near_ties(bq):
+    """theta = 0 makes y = x exactly, so quotients y / s can be placed on and next to
+    half-integers: the fused codes must match IEEE float32 division bit for bit."""
+    torch = H.torch()
+    theta = np.zeros((12, 2048), np.float32)
+    layer = make_layer(bq, theta)
+    rng = np.random.default_rng(11)
+    rows = []
+    for lo, hi in ((-0.5, 0.4375), (-0.7, 0.8), (-3.1, 0.2), (-0.05, 1.9), (-1e-3, 1e-3)):
+        s = np.float32(np.float16(np.float32(np.float32(hi) - np.float32(lo)) / np.float32(15)))
+        row = rng.uniform(lo, hi, 4096).astype(np.float32)
+        k = rng.integers(-16, 16, 4096).astype(np.float32)
+        ties = ((k + np.float32(0.5)) * s).astype(np.float32)
+        sel = rng.integers(0, 3, 4096)
+        ties = np.where(sel == 1, np.nextafter(ties, np.float32(np.inf)), ties)
+        ties = np.where(sel == 2, np.nextafter(ties, np.float32(-np.inf)), ties)
+        ties = np.clip(ties, np.float32(lo), np.float32(hi))
+        row[1::2] = ties[1::2]
+        row[::128] = np.float32(lo)
+        row[1::128] = np.float32(hi)
+        rows.append(row)
+    x = np.stack(rows).astype(np.float32)
+    for bits in (4, 2):
+        codes, scale, zero = bq.quant_outputs(x.shape[0], 4096, bits, 128, "cuda")
+        bq.bq_transform_quantize(layer, H.dev_f32(x), bits, 128, codes, scale, zero)
+        torch.cuda.synchronize()
+        c_ref, s_ref, z_ref = oq.quantize_pack(x, bits, 128)
+        assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
+        assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
+        assert np.array_equal(H.host(codes), c_ref)
