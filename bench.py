@@ -44,6 +44,9 @@ def workload_spec(name: str):
     if name == "act4096":
         return dict(make=lambda rank: wl.act_4096(2048, seed_offset=rank), kind="quant", rows=2048, n=4096,
                     bits=4, group=128, label="act n=4096 rows=2048 bf16 -> Qx + INT4 RTN g128 (LLaMA-2-7B activation shape)")
+    if name == "fwd4096":
+        return dict(make=lambda rank: wl.act_4096(2048, seed_offset=rank), kind="fwd", rows=2048, n=4096,
+                    bits=4, group=128, label="act n=4096 rows=2048 bf16 -> Qx float32 (forward only)")
     if name == "weight4096":
         return dict(make=lambda rank: wl.weight_4096(11008), kind="quant", rows=11008, n=4096, bits=2, group=128,
                     label="weight n=4096 rows=11008 bf16 -> W Q^T + INT2 RTN g128 (W2A16)")
@@ -212,11 +215,15 @@ def run_ours(args, spec, rank, world, local_rank):
     O = None if w.O is None else torch.from_numpy(w.O).to(dev)
     layer = bq.Layer(theta, O)
     codes, scale, zero = bq.quant_outputs(rows, n, bits, group, dev)
+    yf = torch.empty((rows, n), dtype=torch.float32, device=dev) if spec["kind"] == "fwd" else None
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step():
-        bq.bq_transform_quantize(layer, x, bits, group, codes, scale, zero)
+        if yf is not None:
+            bq.bq_butterfly_fwd(layer, x, yf)
+        else:
+            bq.bq_transform_quantize(layer, x, bits, group, codes, scale, zero)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -258,7 +265,7 @@ def run_ours(args, spec, rank, world, local_rank):
 
     # end to end through the public API with host buffers: H2D input, kernel, D2H codes/scale/zero
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and yf is None:
         x_pin = x_host.pin_memory()
         c_pin = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
         s_pin = torch.empty(scale.shape, dtype=scale.dtype).pin_memory()
@@ -294,7 +301,7 @@ def run_ours(args, spec, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     fl_launch = flops_per_row(w.m, w.r) * rows
-    by_launch = bytes_per_row(n, 2, bits, group) * rows
+    by_launch = (bytes_per_row(n, 2, bits, group) if yf is None else n * (2 + 4)) * rows
     avg_launch_s = (total_ms / args.steps) * 1e-3
     achieved_tf = fl_launch / avg_launch_s / 1e12
     traffic, traffic_kernel = recorded_traffic(args.workload)
@@ -387,7 +394,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="act4096", choices=["act4096", "weight4096", "act5120"])
+    ap.add_argument("--workload", default="act4096", choices=["act4096", "fwd4096", "weight4096", "act5120"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

@@ -12,9 +12,8 @@
 //    bq_precompute_cs) into its 128 TMEM lanes x 416 columns at start-up, and
 //    every thread reads its own lane with tcgen05.ld, a path separate from
 //    shared memory.
-//  * 128 threads (one warpgroup, thread t <-> TMEM lane t) own a row group;
-//    each thread holds 32 elements of 2 rows (R = 2; a 1-row tail handles odd
-//    counts), so each coefficient load serves two rows.  The 12 stages run in
+//  * 128 threads (one warpgroup, thread t <-> TMEM lane t) own a row at a
+//    time; each thread holds 32 of its elements.  The 12 stages run in
 //    three passes with the in-register index bits
 //        pass A: position bits {0..4}    stages 0..4
 //        pass B: position bits {5..9}    stages 5..9
@@ -29,9 +28,10 @@
 //    fma.rn.f32x2 where two pairs sit in adjacent registers; when the layer's
 //    scaled form is out of range (table header flag 0) the same kernel runs the
 //    plain cos/sin rotation instead.
-//  * One CTA per SM (all 512 TMEM columns, 128 KB shared memory), two row
-//    groups per CTA for latency hiding; inputs of the next row pair are
-//    prefetched into registers while the current pair is processed.
+//  * One CTA per SM (all 512 TMEM columns), three row groups per CTA sharing
+//    the tensor-memory image (warps w, w+4, w+8 use the same lanes) for
+//    latency hiding; the next row's input is prefetched into registers while
+//    the current row is processed.
 #include <cfloat>
 
 #include "bq_internal.cuh"
@@ -41,10 +41,10 @@ namespace {
 
 constexpr int M = 4096;
 constexpr int kGroupThreads = 128;
-constexpr int kSlots = 2;
+constexpr int kSlots = 3;
 constexpr int kThreads = kSlots * kGroupThreads;
 constexpr int kColB = 160, kColC = 320, kColS = 384;
-constexpr int kFillPerSlot = kImageCols / kSlots;  // 208 columns per slot
+constexpr int kFillChunks = kImageCols / 16;  // 26 chunks of 16 columns, dealt round-robin to the slots
 
 enum Mode { kOutF32 = 0, kOutBF16 = 1, kQuant = 2 };
 
@@ -250,6 +250,13 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
+// Inserts the low `len` bits of `a` into `b` at bit `pos`.
+__device__ __forceinline__ uint32_t bfi(uint32_t a, uint32_t b, int pos, int len) {
+  uint32_t d;
+  asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(pos), "r"(len));
+  return d;
+}
+
 // Codes of 8 values by IEEE division, for sets where the fast path below cannot
 // prove its result (kept out of line: it runs for roughly one set in 10^4).
 template <int BITS>
@@ -276,9 +283,10 @@ __device__ __noinline__ uint32_t codes_by_division(float y0, float y1, float y2,
 // RN(y/s) lies on the same side of the same half-integer and
 // rint(RN(y/s)) = rint(v) exactly.  rint(v) is
 // taken with the float32 magic constant 1.5 * 2^23 (round-half-even addition),
-// whose bit pattern then carries the integer, so adding z and clamping happen
-// on integers.  A set of 8 values with any element too close to a tie (or with
-// |v| >= 2^22) is redone with IEEE division.
+// with z folded into the constant (no tie can occur on the fast path, so
+// rint(v) + z = RN(v + z) there); the bit pattern then carries the code.  A set of
+// 8 values with any element too close to a tie (or |v| >= 2^22), or whose group
+// would need clamping, is redone with IEEE division and clamping.
 template <int BITS, int GLANES, int R>
 __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const FastArgs& A, long long row0, int tau,
                                                int lane) {
@@ -324,9 +332,12 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
   }
   const float z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax), 0.f);  // +0 for a zero point of 0
   const float inv = __fdiv_rn(1.f, s);
-  // tie margin for the whole group: every |v| <= max(|lo|, |hi|) * inv * (1 + 2^-22)
+  // tie margin for the whole group: every |v| <= max(|lo|, |hi|) * inv * (1 + 2^-20)
   const float vmax = fmaxf(fabsf(lo), fabsf(hi)) * inv * 1.000001f;
   const float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
+  // codes are monotone in y: when the group's extremes quantize inside [0, qmax]
+  // (checked with IEEE division), no element needs clamping
+  const bool inrange = __fadd_rn(rintf(__fdiv_rn(lo, s)), z) >= 0.f && __fadd_rn(rintf(__fdiv_rn(hi, s)), z) <= qmax;
   {
     const int k = bitrev<S>(lane & (S - 1));
     if (((lane >> LOGS) & ((1 << (LOGG - LOGS)) - 1)) == 0) {
@@ -336,36 +347,35 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
       A.zero[row * GPR + g] = __half_as_ushort(__float2half_rn(z));
     }
   }
-  const float kMagic = 12582912.f;  // 1.5 * 2^23
+  // rint(v) + z as the bit pattern of v + (1.5 * 2^23 + z): valid because the fast
+  // path only accepts v away from half-integers (no rounding tie can occur)
+  const float mz = __fadd_rn(12582912.f, z);
 #pragma unroll
   for (int k = 0; k < S; ++k) {
     const int src = (lane & ~(S - 1)) | bitrev<S>(k);
     const float invk = __shfl_sync(0xffffffffu, inv, src);
     const float thrk = __shfl_sync(0xffffffffu, thr, src);
-    const int zk = static_cast<int>(__shfl_sync(0xffffffffu, z, src));
+    const float mzk = __shfl_sync(0xffffffffu, mz, src);
     const float sk = __shfl_sync(0xffffffffu, s, src);
+    const bool ink = __shfl_sync(0xffffffffu, static_cast<int>(inrange), src) != 0;
     const int r = k >> 2, h = k & 3;
-    const float2 iv = make_float2(invk, invk), mg = make_float2(kMagic, kMagic);
-    const float2 nmg = make_float2(-kMagic, -kMagic), neg1 = make_float2(-1.f, -1.f);
-    bool exact = true;
+    const float2 iv = make_float2(invk, invk), m2 = make_float2(mzk, mzk);
+    const float2 nm2 = make_float2(-mzk, -mzk), neg1 = make_float2(-1.f, -1.f);
+    bool exact = ink;
     uint32_t word = 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 v = __fmul2_rn(a[r][4 * h + q], iv);
-      const float2 t = __fadd2_rn(v, mg);
-      const float2 e = __ffma2_rn(__fadd2_rn(t, nmg), neg1, v);  // v - rint(v), exact
+      const float2 t = __fadd2_rn(v, m2);
+      const float2 e = __ffma2_rn(__fadd2_rn(t, nm2), neg1, v);  // v - rint(v), exact
       exact = exact && fabsf(e.x) < thrk && fabsf(e.y) < thrk;
-      int c0 = static_cast<int>(__float_as_uint(t.x)) - 0x4B400000 + zk;
-      int c1 = static_cast<int>(__float_as_uint(t.y)) - 0x4B400000 + zk;
-      c0 = min(max(c0, 0), QMAX);
-      c1 = min(max(c1, 0), QMAX);
-      word |= static_cast<uint32_t>(c0) << (BITS * (2 * q));
-      word |= static_cast<uint32_t>(c1) << (BITS * (2 * q + 1));
+      word = bfi(__float_as_uint(t.x), word, BITS * (2 * q), BITS);
+      word = bfi(__float_as_uint(t.y), word, BITS * (2 * q + 1), BITS);
     }
     if (!exact) {
       word = codes_by_division<BITS>(a[r][4 * h].x, a[r][4 * h].y, a[r][4 * h + 1].x, a[r][4 * h + 1].y,
                                      a[r][4 * h + 2].x, a[r][4 * h + 2].y, a[r][4 * h + 3].x, a[r][4 * h + 3].y,
-                                     sk, static_cast<float>(zk));
+                                     sk, __fadd_rn(mzk, -12582912.f));
     }
     const long long row = row0 + r;
     if constexpr (BITS == 4) {
@@ -488,16 +498,10 @@ template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
 __device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long long re, int slot, int tau, int lane,
                                          uint32_t tb, float* bufAB, float* bufBC, Prefetch<TI>& pre,
                                          uint32_t (&c0)[32], uint32_t (&c1)[32]) {
-  for (long long row = rb; row < re;) {
-    const int cnt = (re - row >= 2) ? 2 : 1;
-    const long long nrow = row + cnt;
-    const int ncnt = re - nrow >= 2 ? 2 : static_cast<int>(re - nrow);
-    if (cnt == 2)
-      process<TI, MODE, BITS, GLANES, SCALED, 2>(A, row, nrow, ncnt, slot, tau, lane, tb, bufAB, bufBC, pre, c0, c1);
-    else
-      process<TI, MODE, BITS, GLANES, SCALED, 1>(A, row, nrow, ncnt, slot, tau, lane, tb, bufAB, bufBC, pre, c0, c1);
-    row = nrow;
-  }
+#pragma unroll 1
+  for (long long row = rb; row < re; ++row)
+    process<TI, MODE, BITS, GLANES, SCALED, 1>(A, row, row + 1, row + 1 < re ? 1 : 0, slot, tau, lane, tb, bufAB,
+                                               bufBC, pre, c0, c1);
 }
 
 template <typename TI, int MODE, int BITS, int GLANES>
@@ -506,14 +510,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __shared__ uint32_t s_tmem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
-  float* bufAB = smem + slot * (4 * M);
-  float* bufBC = bufAB + 2 * M;
+  float* bufAB = smem + slot * (2 * M);
+  float* bufBC = bufAB + M;
   const long long G = static_cast<long long>(gridDim.x) * kSlots;
   const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
 
   Prefetch<TI> pre;
-  prefetch(pre, static_cast<const TI*>(A.x), rb, re - rb >= 2 ? 2 : static_cast<int>(re - rb), tau);
+  prefetch(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
 
   if (warp == 0) {
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
@@ -525,43 +529,32 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
   {
-    // each thread copies its lane's share of the image: two batches of loads in
-    // flight, then the tensor-memory stores
-    const float4* src = reinterpret_cast<const float4*>(A.image + tau * kImageCols + slot * kFillPerSlot);
-    constexpr int kChunks = kFillPerSlot / 16;  // 13 chunks of 16 columns
-    constexpr int kFirst = 7;
-    {
-      float4 f[kFirst * 4];
+    // each thread copies its lane's share of the image (16-column chunks dealt
+    // round-robin to the slots): all loads in flight first, then the stores
+    const float4* src = reinterpret_cast<const float4*>(A.image + tau * kImageCols);
+    constexpr int kMine = (kFillChunks + kSlots - 1) / kSlots;
+    float4 f[kMine * 4];
 #pragma unroll
-      for (int i = 0; i < kFirst * 4; ++i) f[i] = src[i];
+    for (int i = 0; i < kMine; ++i) {
+      const int c = slot + i * kSlots;
+      if (c < kFillChunks) {
 #pragma unroll
-      for (int c = 0; c < kFirst; ++c) {
-        uint32_t v[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[4 * i] = __float_as_uint(f[4 * c + i].x);
-          v[4 * i + 1] = __float_as_uint(f[4 * c + i].y);
-          v[4 * i + 2] = __float_as_uint(f[4 * c + i].z);
-          v[4 * i + 3] = __float_as_uint(f[4 * c + i].w);
-        }
-        tmem_st16(tb + slot * kFillPerSlot + 16 * c, v);
+        for (int j = 0; j < 4; ++j) f[4 * i + j] = src[4 * c + j];
       }
     }
-    {
-      float4 f[(kChunks - kFirst) * 4];
 #pragma unroll
-      for (int i = 0; i < (kChunks - kFirst) * 4; ++i) f[i] = src[kFirst * 4 + i];
-#pragma unroll
-      for (int c = 0; c < kChunks - kFirst; ++c) {
+    for (int i = 0; i < kMine; ++i) {
+      const int c = slot + i * kSlots;
+      if (c < kFillChunks) {
         uint32_t v[16];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[4 * i] = __float_as_uint(f[4 * c + i].x);
-          v[4 * i + 1] = __float_as_uint(f[4 * c + i].y);
-          v[4 * i + 2] = __float_as_uint(f[4 * c + i].z);
-          v[4 * i + 3] = __float_as_uint(f[4 * c + i].w);
+        for (int j = 0; j < 4; ++j) {
+          v[4 * j] = __float_as_uint(f[4 * i + j].x);
+          v[4 * j + 1] = __float_as_uint(f[4 * i + j].y);
+          v[4 * j + 2] = __float_as_uint(f[4 * i + j].z);
+          v[4 * j + 3] = __float_as_uint(f[4 * i + j].w);
         }
-        tmem_st16(tb + slot * kFillPerSlot + 16 * (kFirst + c), v);
+        tmem_st16(tb + 16 * c, v);
       }
     }
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -590,13 +583,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
 template <typename TI, int MODE, int BITS, int GLANES>
 bq_status launch(const FastArgs& A, cudaStream_t st) {
   auto kern = k_fast4096<TI, MODE, BITS, GLANES>;
-  const int smem = kSlots * 4 * M * static_cast<int>(sizeof(float));
+  const int smem = kSlots * 2 * M * static_cast<int>(sizeof(float));
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return BQ_ERR_CUDA;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long long grid = (A.rows + 2 * kSlots - 1) / (2 * kSlots);
+  long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(A);
