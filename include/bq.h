@@ -16,7 +16,8 @@
  * ---------------------------------------
  *  - All data pointers are DEVICE pointers unless stated; the caller owns
  *    every buffer.  The library never allocates device memory and keeps no
- *    global state; calls on different streams are independent.
+ *    global state (the one exception is the fixed scratch array of
+ *    bq_butterfly_bwd_noalloc); calls on different streams are independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream; an error status is
  *    returned before anything is launched when host-side validation fails.
@@ -113,6 +114,36 @@ bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers,
                            const float* dy, float* dx, float* dtheta,
                            int64_t rows_per_layer, void* workspace,
                            size_t workspace_bytes, void* stream);
+
+/* Size in bytes of the fixed device scratch that bq_butterfly_bwd_noalloc uses. */
+#define BQ_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* bq_butterfly_bwd without a workspace argument, for callers that cannot
+ * allocate device memory when they run the backward: code running while
+ * another framework owns the device allocator, real-time loops that must not
+ * block in an allocator, or processes whose device memory is fully reserved
+ * by a pool.  The paper has no counterpart to this entry point.
+ *
+ * Arguments, results and the deterministic dtheta reduction are those of
+ * bq_butterfly_bwd; y and dx are bitwise identical to it.  dtheta is summed
+ * in possibly fewer, larger token chunks (so possibly in a different order):
+ * the library's scratch is one file-scope device array of
+ * BQ_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library
+ * keeps until the process exits, and the chunk count is reduced until the
+ * partial sums fit in it.  If even one chunk per layer does not fit
+ * (num_layers * log2(m) * m/2 * 4 bytes + 512 > BQ_NOALLOC_SCRATCH_BYTES,
+ * e.g. more than 85 layers of width 4096) it returns BQ_ERR_WORKSPACE and
+ * launches nothing.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call shares the one array and clears the part that must
+ * start at zero itself; calls whose executions overlap on the GPU (different
+ * streams, or concurrent host threads) race on it and must be serialised by
+ * the caller. */
+bq_status bq_butterfly_bwd_noalloc(const bq_layer* layers, int32_t num_layers,
+                                   const void* x, bq_dtype xt, void* y, bq_dtype yt,
+                                   const float* dy, float* dx, float* dtheta,
+                                   int64_t rows_per_layer, void* stream);
 
 /* Fused Q x followed by per-group asymmetric round-to-nearest quantization and
  * packing (2-bit weights: explainer article, section "training & results";

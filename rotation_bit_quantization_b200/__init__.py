@@ -9,6 +9,7 @@ from ._lib import (  # noqa: F401
     BQError,
     Layer,
     bq_butterfly_bwd,
+    bq_butterfly_bwd_noalloc,
     bq_butterfly_bwd_workspace_size,
     bq_butterfly_fwd,
     bq_butterfly_inv,

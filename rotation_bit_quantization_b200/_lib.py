@@ -25,6 +25,7 @@ EXPORTED = (
     "bq_butterfly_inv",
     "bq_butterfly_bwd_workspace_size",
     "bq_butterfly_bwd",
+    "bq_butterfly_bwd_noalloc",
     "bq_transform_quantize",
     "bq_weight_rotate_pack",
     "bq_status_string",
@@ -64,6 +65,7 @@ def load(path: str | None = None):
         "bq_butterfly_inv": (i32, [lp, vp, i32, vp, i32, i64, vp]),
         "bq_butterfly_bwd_workspace_size": (sz, [i32, i32, i64]),
         "bq_butterfly_bwd": (i32, [lp, i32, vp, i32, vp, i32, vp, vp, vp, i64, vp, sz, vp]),
+        "bq_butterfly_bwd_noalloc": (i32, [lp, i32, vp, i32, vp, i32, vp, vp, vp, i64, vp]),
         "bq_transform_quantize": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
         "bq_weight_rotate_pack": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
@@ -187,6 +189,17 @@ def bq_butterfly_bwd(layers, x, y, dy, dx, dtheta, workspace, stream=None):
                                                         _dtype_code(y), _ptr(dy), _ptr(dx), _ptr(dtheta), rows,
                                                         _ptr(workspace), workspace.numel() * workspace.element_size(),
                                                         _stream(stream)))
+
+
+def bq_butterfly_bwd_noalloc(layers, x, y, dy, dx, dtheta, stream=None):
+    """Like bq_butterfly_bwd, with the library's fixed device scratch instead of a workspace."""
+    arr = (BQLayer * len(layers))(*[l.c for l in layers])
+    for t, nm in ((x, "x"), (y, "y"), (dy, "dy"), (dx, "dx"), (dtheta, "dtheta")):
+        _dev(t, nm)
+    rows = x.numel() // (len(layers) * layers[0].n)
+    _check("bq_butterfly_bwd_noalloc",
+           load().bq_butterfly_bwd_noalloc(arr, len(layers), _ptr(x), _dtype_code(x), _ptr(y), _dtype_code(y),
+                                           _ptr(dy), _ptr(dx), _ptr(dtheta), rows, _stream(stream)))
 
 
 def _quant(name, layer, x, bits, group, codes, scale, zero, stream):
