@@ -81,10 +81,11 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files) -> str:
+    """Hash of the CUDA sources a profiled kernel is built from (paths relative to csrc/)."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "rotation_bit_quantization_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
+    for f in sorted(files):
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode()); h.update(fh.read())
     return h.hexdigest()[:16]
@@ -98,7 +99,7 @@ def recorded_traffic(workload: str):
         return None, None
     with open(p) as f:
         rec = json.load(f).get(workload)
-    if not rec or rec.get("source_hash") != kernel_source_hash():
+    if not rec or rec.get("source_hash") != kernel_source_hash(rec.get("sources", [])):
         return None, None
     return rec.get("dram_bytes_per_launch"), rec.get("kernel")
 
