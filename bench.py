@@ -50,6 +50,9 @@ def workload_spec(name: str):
     if name == "weight4096":
         return dict(make=lambda rank: wl.weight_4096(11008), kind="quant", rows=11008, n=4096, bits=2, group=128,
                     label="weight n=4096 rows=11008 bf16 -> W Q^T + INT2 RTN g128 (W2A16)")
+    if name == "bwd":
+        return dict(make=None, kind="bwd", rows=65536, n=4096, bits=0, group=0, layers=32,
+                    label="calibration backward: 32 layers x 65536 tokens x n=4096, X bf16, dY fp32 -> Y bf16, dX fp32, dtheta (one launch)")
     if name == "act5120":
         return dict(make=lambda rank: wl.act_5120(8192), kind="quant", rows=8192, n=5120, bits=4, group=128,
                     label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> INT4 RTN g128 (LLaMA-2-13B shape)")
@@ -352,6 +355,70 @@ def run_ours(args, spec, rank, world, local_rank):
     return result
 
 
+def run_bwd_bench(args, spec, rank, world, local_rank):
+    """The calibration backward: one bq_butterfly_bwd launch over all layers per step."""
+    import torch
+    import torch.distributed as dist
+
+    import rotation_bit_quantization_b200 as bq
+    from rotation_bit_quantization_b200 import build as bq_build
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    bq_build.build()
+    bq.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    L, T, m = spec["layers"], spec["rows"], spec["n"]
+    thetas = wl.backward_angles(L, m)
+    layers = [bq.Layer(torch.from_numpy(thetas[l]).to(dev)) for l in range(L)]
+    x, dy = wl.backward_inputs_device(L, T, m, dev, seed=5 + rank)
+    y = torch.empty((L, T, m), dtype=torch.bfloat16, device=dev)
+    dx = torch.empty((L, T, m), dtype=torch.float32, device=dev)
+    dth = torch.empty((L, 12 * m // 2), dtype=torch.float32, device=dev)
+    ws = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, L, T), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bq.bq_butterfly_bwd(layers, x, y, dy, dx, dth, ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id_for(dev))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s_, e_ in evs:
+        s_.record(stream)
+        step()
+        e_.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = float(sum(s_.elapsed_time(e_) for s_, e_ in evs))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / args.steps
+    tokens = L * T
+    by_tok = m * (2 + 2 + 4 + 4)
+    peaks, peak_src = load_peaks()
+    achieved = tokens * by_tok / (ms * 1e-3) / 1e9
+    return {
+        "metric": "butterfly backward tokens/s (Y, dX, dtheta), n=4096", "value": tokens * world / (ms * 1e-3),
+        "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded on device)", "config": {"workload": spec["label"], "layers": L, "tokens_per_layer": T,
+                                                           "l2": "inputs 103 GB, far larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "algorithmic_bytes_per_token": by_tok, "algorithmic_flops_per_token": 368640},
+        "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, spec):
@@ -395,7 +462,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="act4096", choices=["act4096", "fwd4096", "weight4096", "act5120"])
+    ap.add_argument("--workload", default="act4096", choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -407,6 +474,8 @@ def main():
     spec = workload_spec(args.workload)
 
     if args.impl == "reference":
+        if spec["kind"] == "bwd":
+            raise SystemExit("--impl reference covers the transform + quantize workloads only")
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args, spec)))
@@ -421,7 +490,10 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res = run_ours(args, spec, rank, world, local_rank)
+        if spec["kind"] == "bwd":
+            res = run_bwd_bench(args, spec, rank, world, local_rank)
+        else:
+            res = run_ours(args, spec, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -368,3 +368,71 @@ def test_quant_exact_ties_and_near_ties(bq):
         assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
         assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
         assert np.array_equal(H.host(codes), c_ref)
+
+
+# --------------------------------------------------------------------------- backward at full size
+
+@pytest.mark.slow
+def test_full_backward_32_layers(bq):
+    """32 layers x 65536 tokens x 4096, one launch (the calibration backward workload).
+
+    dtheta sums over every token, so it cannot be sampled: two 2048-token slices of
+    layer 0 are checked against the oracle, and the full-size dtheta is checked to be
+    the sum of the kernel's own dtheta over the 32 disjoint slices (additivity).  Y
+    and dX are compared with the oracle on sampled tokens, and every layer must
+    satisfy sum <dY, Y> = sum <dX, X> (Q orthogonal)."""
+    torch = H.torch()
+    L, T, m = 32, 65536, 4096
+    free, _ = torch.cuda.mem_get_info()
+    if free < 115 * 2 ** 30:
+        pytest.skip("needs ~110 GB of free device memory")
+    thetas = wl.backward_angles(L, m)
+    layers = [make_layer(bq, thetas[l]) for l in range(L)]
+    x, dy = wl.backward_inputs_device(L, T, m, "cuda")
+    y = torch.empty((L, T, m), dtype=torch.bfloat16, device="cuda")
+    dx = torch.empty((L, T, m), dtype=torch.float32, device="cuda")
+    dth = torch.empty((L, 12 * m // 2), dtype=torch.float32, device="cuda")
+    ws = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, L, T), dtype=torch.uint8, device="cuda")
+    bq.bq_butterfly_bwd(layers, x, y, dy, dx, dth, ws)
+    torch.cuda.synchronize()
+    # invariant per layer (float64 reductions on the device)
+    for l in range(L):
+        a = (dy[l].double() * y[l].double()).sum().item()
+        b = (dx[l].double() * x[l].double()).sum().item()
+        scale = (dy[l].double().abs() * y[l].double().abs()).sum().item()
+        assert abs(a - b) <= 1e-3 * scale, f"layer {l}: {a} vs {b}"
+    # sampled tokens of layers 0 and 31 against the oracle
+    rng = np.random.default_rng(0)
+    for l in (0, 31):
+        idx = np.sort(rng.choice(T, 48, replace=False))
+        ti = torch.from_numpy(idx).cuda()
+        xs = H.host(x[l][ti]).reshape(48, m)
+        xf = H.input_f64(xs, "bf16")
+        dys = H.host(dy[l][ti]).astype(np.float64)
+        yr, dxr, _ = ob.backward(thetas[l], xf, dys)
+        H.assert_f32_close(H.host(dx[l][ti]), dxr, dys)
+        ybits = H.host(y[l][ti])
+        v = wl.f32_from_bf16_bits(ybits).astype(np.float64)
+        bound = H.bf16_ulp(yr) + H.F32_TOL * np.linalg.norm(xf, axis=-1, keepdims=True)
+        assert np.all(np.abs(v - yr) <= bound)
+    # additivity over 32 disjoint slices of layer 0, and two slices against the oracle
+    S = T // 32
+    parts = torch.zeros((12 * m // 2,), dtype=torch.float64, device="cuda")
+    ws1 = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, 1, S), dtype=torch.uint8, device="cuda")
+    ys = torch.empty((1, S, m), dtype=torch.bfloat16, device="cuda")
+    dxs = torch.empty((1, S, m), dtype=torch.float32, device="cuda")
+    dths = torch.empty((1, 12 * m // 2), dtype=torch.float32, device="cuda")
+    for k in range(32):
+        xk = x[0][k * S:(k + 1) * S].contiguous()[None]
+        dyk = dy[0][k * S:(k + 1) * S].contiguous()[None]
+        bq.bq_butterfly_bwd([layers[0]], xk, ys, dyk, dxs, dths, ws1)
+        torch.cuda.synchronize()
+        parts += dths[0].double()
+        if k in (0, 17):
+            xf = H.input_f64(H.host(xk[0]), "bf16")
+            dyf = H.host(dyk[0]).astype(np.float64)
+            _, _, dthr = ob.backward(thetas[0], xf, dyf)
+            check_dtheta(H.host(dths[0]).reshape(dthr.shape), dthr, ob.backward_abs_scale(thetas[0], xf, dyf))
+    full = dth[0].double()
+    absmax = parts.abs().max().item()
+    assert (full - parts).abs().max().item() <= 1e-4 * absmax + 1e-3
