@@ -530,8 +530,9 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
   {
     // each thread copies its lane's share of the image (16-column chunks dealt
-    // round-robin to the slots): all loads in flight first, then the stores
-    const float4* src = reinterpret_cast<const float4*>(A.image + tau * kImageCols);
+    // round-robin to the slots): all loads in flight first (each warp load is one
+    // contiguous 512-byte run of the [column/4][lane] image), then the stores
+    const float4* src = reinterpret_cast<const float4*>(A.image) + tau;  // block q of lane tau at [q * 128]
     constexpr int kMine = (kFillChunks + kSlots - 1) / kSlots;
     float4 f[kMine * 4];
 #pragma unroll
@@ -539,7 +540,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
       const int c = slot + i * kSlots;
       if (c < kFillChunks) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) f[4 * i + j] = src[4 * c + j];
+        for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
       }
     }
 #pragma unroll
@@ -584,11 +585,18 @@ template <typename TI, int MODE, int BITS, int GLANES>
 bq_status launch(const FastArgs& A, cudaStream_t st) {
   auto kern = k_fast4096<TI, MODE, BITS, GLANES>;
   const int smem = kSlots * 2 * M * static_cast<int>(sizeof(float));
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return BQ_ERR_CUDA;
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
+  // per device: the shared-memory opt-in and the SM count, set up on first use
+  static int sms_of[64] = {};
+  if (sms_of[dev] == 0) {
+    int sms = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return BQ_ERR_CUDA;
+    sms_of[dev] = sms;
+  }
+  const int sms = sms_of[dev];
   long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;

@@ -23,9 +23,10 @@ constexpr int kMaxGroup = 256;     // largest quantization group
 //   fast   [L][m]      per-position coefficient of the scaled form: at stage s
 //                      position i is updated as a_i += fast[s][i] * a_{i ^ 2^s}
 //   sigma  [m]         per-position output scale of the scaled form
-//   image  [128][416]  (m == 4096 only) tensor-memory image of the specialised
-//                      n = 4096 kernel: lane t, column c holds the coefficient
-//                      thread t needs at that column (see bq_fast4096.cu)
+//   image  [104][128][4] (m == 4096 only) tensor-memory image of the specialised
+//                      n = 4096 kernel: lane t, column c (float4 block c/4 of
+//                      lane t) holds the coefficient thread t needs at that
+//                      column (see bq_fast4096.cu)
 struct TableLayout {
   int m, L;
   size_t off_cs, off_fast, off_sigma, off_image, total;

@@ -84,7 +84,9 @@ __device__ __forceinline__ int pos_pass(int pass, int t, int e) {
   return (e & 7) | (t << 3) | ((e >> 3) << 10);
 }
 
-// Tensor-memory image of the n = 4096 kernel: lane t, column c.
+// Tensor-memory image of the n = 4096 kernel: lane t, column c, stored as float4
+// blocks [c / 4][t] so that a warp filling four consecutive columns of its 32
+// lanes reads one contiguous 512-byte run.
 //   columns [0,160):   pass 0 stages 0..4   (32 columns per stage)
 //   columns [160,320): pass 1 stages 5..9
 //   columns [320,384): pass 2 stages 10, 11
@@ -121,7 +123,7 @@ __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
       v = high ? c.y : c.x;
     }
   }
-  table[tl.off_image + idx] = v;
+  table[tl.off_image + (size_t(col >> 2) * kImageLanes + t) * 4 + (col & 3)] = v;
 }
 
 }  // namespace
