@@ -19,7 +19,9 @@
 //        pass B: position bits {5..9}    stages 5..9
 //        pass C: position bits {0,1,2,10,11}  stages 10, 11
 //    and two swizzled shared-memory transposes between them (conflict-free:
-//    one side uses 16-byte vectors, the other 4-byte scalars).  Pass C's
+//    one side uses 16-byte vectors, the other 4-byte scalars).  The A -> B
+//    exchange stays inside each warp (bits 10, 11 are the warp index of both
+//    layouts); only B -> C needs the row group's barrier.  Pass C's
 //    layout keeps 8 consecutive positions per thread, so the RTN epilogue
 //    (group statistics, packing, coalesced stores) runs in place without a
 //    third transpose.
@@ -250,13 +252,6 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// Inserts the low `len` bits of `a` into `b` at bit `pos`.
-__device__ __forceinline__ uint32_t bfi(uint32_t a, uint32_t b, int pos, int len) {
-  uint32_t d;
-  asm("bfi.b32 %0, %1, %2, %3, %4;" : "=r"(d) : "r"(a), "r"(b), "r"(pos), "r"(len));
-  return d;
-}
-
 // Codes of 8 values by IEEE division, for sets where the fast path below cannot
 // prove its result (kept out of line: it runs for roughly one set in 10^4).
 template <int BITS>
@@ -330,14 +325,18 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
     s = 1.f;
     h16 = __float2half_rn(1.f);
   }
-  const float z = __fadd_rn(fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), qmax), 0.f);  // +0 for a zero point of 0
+  const float zraw = rintf(__fdiv_rn(-lo, s));
+  const float z = __fadd_rn(fminf(fmaxf(zraw, 0.f), qmax), 0.f);  // +0 for a zero point of 0
   const float inv = __fdiv_rn(1.f, s);
   // tie margin for the whole group: every |v| <= max(|lo|, |hi|) * inv * (1 + 2^-20)
   const float vmax = fmaxf(fabsf(lo), fabsf(hi)) * inv * 1.000001f;
   const float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
-  // codes are monotone in y: when the group's extremes quantize inside [0, qmax]
-  // (checked with IEEE division), no element needs clamping
-  const bool inrange = __fadd_rn(rintf(__fdiv_rn(lo, s)), z) >= 0.f && __fadd_rn(rintf(__fdiv_rn(hi, s)), z) <= qmax;
+  // codes are monotone in y: when the group's extremes quantize inside [0, qmax],
+  // no element needs clamping.  Division and rint are both odd functions, so the
+  // code of lo is z - rint(-lo/s) exactly: in range at the bottom iff
+  // rint(-lo/s) <= qmax.  The top is checked with one IEEE division.
+  const bool inrange = zraw <= qmax && __fadd_rn(rintf(__fdiv_rn(hi, s)), z) <= qmax;
+  const float thr_in = inrange ? thr : -1.f;  // -1 sends the whole set to the slow path
   {
     const int k = bitrev<S>(lane & (S - 1));
     if (((lane >> LOGS) & ((1 << (LOGG - LOGS)) - 1)) == 0) {
@@ -348,29 +347,40 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
     }
   }
   // rint(v) + z as the bit pattern of v + (1.5 * 2^23 + z): valid because the fast
-  // path only accepts v away from half-integers (no rounding tie can occur)
+  // path only accepts v away from half-integers (no rounding tie can occur).  The
+  // code sits in the low bits (the constant's bits start at bit 22), so
+  // bits(t0) + bits(t1) << BITS ... has the packed byte in its low byte.
   const float mz = __fadd_rn(12582912.f, z);
 #pragma unroll
   for (int k = 0; k < S; ++k) {
     const int src = (lane & ~(S - 1)) | bitrev<S>(k);
     const float invk = __shfl_sync(0xffffffffu, inv, src);
-    const float thrk = __shfl_sync(0xffffffffu, thr, src);
+    const float thrk = __shfl_sync(0xffffffffu, thr_in, src);
     const float mzk = __shfl_sync(0xffffffffu, mz, src);
     const float sk = __shfl_sync(0xffffffffu, s, src);
-    const bool ink = __shfl_sync(0xffffffffu, static_cast<int>(inrange), src) != 0;
     const int r = k >> 2, h = k & 3;
     const float2 iv = make_float2(invk, invk), m2 = make_float2(mzk, mzk);
     const float2 nm2 = make_float2(-mzk, -mzk), neg1 = make_float2(-1.f, -1.f);
-    bool exact = ink;
-    uint32_t word = 0;
+    bool exact = true;
+    uint32_t b[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float2 v = __fmul2_rn(a[r][4 * h + q], iv);
       const float2 t = __fadd2_rn(v, m2);
       const float2 e = __ffma2_rn(__fadd2_rn(t, nm2), neg1, v);  // v - rint(v), exact
-      exact = exact && fabsf(e.x) < thrk && fabsf(e.y) < thrk;
-      word = bfi(__float_as_uint(t.x), word, BITS * (2 * q), BITS);
-      word = bfi(__float_as_uint(t.y), word, BITS * (2 * q + 1), BITS);
+      exact = exact & (fabsf(e.x) < thrk) & (fabsf(e.y) < thrk);
+      b[2 * q] = __float_as_uint(t.x);
+      b[2 * q + 1] = __float_as_uint(t.y);
+    }
+    uint32_t word;
+    if constexpr (BITS == 4) {
+      const uint32_t p0 = b[0] + (b[1] << 4), p1 = b[2] + (b[3] << 4);
+      const uint32_t p2 = b[4] + (b[5] << 4), p3 = b[6] + (b[7] << 4);
+      word = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040), 0x5410);
+    } else {
+      const uint32_t p0 = b[0] + (b[1] << 2) + (b[2] << 4) + (b[3] << 6);
+      const uint32_t p1 = b[4] + (b[5] << 2) + (b[6] << 4) + (b[7] << 6);
+      word = __byte_perm(p0, p1, 0x0040) & 0xffffu;
     }
     if (!exact) {
       word = codes_by_division<BITS>(a[r][4 * h].x, a[r][4 * h].y, a[r][4 * h + 1].x, a[r][4 * h + 1].y,
@@ -435,7 +445,10 @@ __device__ __forceinline__ void process(const FastArgs& A, long long row0, long 
     for (int c = 0; c < 8; ++c)
       *reinterpret_cast<float4*>(bufAB + r * M + tau * 32 + 4 * (c ^ (tau & 7))) =
           make_float4(a[r][2 * c].x, a[r][2 * c].y, a[r][2 * c + 1].x, a[r][2 * c + 1].y);
-  group_sync(slot);
+  // pass-A thread t writes row t (positions 32t..32t+31); pass-B thread t reads rows
+  // 32(t >> 5) .. 32(t >> 5) + 31: position bits 10, 11 are the warp index in both
+  // layouts, so this exchange stays inside the warp
+  __syncwarp();
   {
     const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
 #pragma unroll
@@ -498,10 +511,13 @@ template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
 __device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long long re, int slot, int tau, int lane,
                                          uint32_t tb, float* bufAB, float* bufBC, Prefetch<TI>& pre,
                                          uint32_t (&c0)[32], uint32_t (&c1)[32]) {
+  // the B -> C buffer alternates between rows: with only a warp-level sync before
+  // the next row's B -> C writes, row i's readers and row i+2's writers are kept
+  // apart by row i+1's row-group barrier
 #pragma unroll 1
   for (long long row = rb; row < re; ++row)
     process<TI, MODE, BITS, GLANES, SCALED, 1>(A, row, row + 1, row + 1 < re ? 1 : 0, slot, tau, lane, tb, bufAB,
-                                               bufBC, pre, c0, c1);
+                                               bufBC + ((row - rb) & 1) * M, pre, c0, c1);
 }
 
 template <typename TI, int MODE, int BITS, int GLANES>
@@ -510,8 +526,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __shared__ uint32_t s_tmem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
-  float* bufAB = smem + slot * (2 * M);
-  float* bufBC = bufAB + M;
+  float* bufAB = smem + slot * (3 * M);
+  float* bufBC = bufAB + M;  // two buffers, used alternately
   const long long G = static_cast<long long>(gridDim.x) * kSlots;
   const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
@@ -584,7 +600,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
 template <typename TI, int MODE, int BITS, int GLANES>
 bq_status launch(const FastArgs& A, cudaStream_t st) {
   auto kern = k_fast4096<TI, MODE, BITS, GLANES>;
-  const int smem = kSlots * 2 * M * static_cast<int>(sizeof(float));
+  const int smem = kSlots * 3 * M * static_cast<int>(sizeof(float));
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
   // per device: the shared-memory opt-in and the SM count, set up on first use
