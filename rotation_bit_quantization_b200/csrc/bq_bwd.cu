@@ -238,7 +238,7 @@ bq_status run_bwd(const BwdArgs& A, cudaStream_t st) {
 }  // namespace
 
 int bwd_chunks(int m, int num_layers, int64_t rows) {
-  (void)m;
+  if (m == 4096) return bwd4096_chunks(num_layers, rows);
   const int target_blocks = 148 * 4;
   long long c = (target_blocks + num_layers - 1) / num_layers;
   if (c > rows) c = rows;
@@ -254,6 +254,8 @@ size_t bwd_workspace_bytes(int m, int num_layers, int chunks) {
 bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt, void* y, bq_dtype yt,
                      const float* dy, float* dx, float* dtheta, int64_t rows, void* ws, int chunks,
                      cudaStream_t st) {
+  if (layers[0].m == 4096)
+    return launch_bwd4096(layers, num_layers, x, xt, y, yt, dy, dx, dtheta, rows, ws, chunks, st);
   BwdArgs A;
   A.m = layers[0].m;
   A.L = layers[0].L;

@@ -96,6 +96,10 @@ bq_status launch_generic(const KLayer& L, const void* x, bq_dtype xt, void* y, b
 bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt,
                      void* y, bq_dtype yt, const float* dy, float* dx, float* dtheta,
                      int64_t rows, void* ws, int chunks, cudaStream_t st);
+bq_status launch_bwd4096(const KLayer* layers, int num_layers, const void* x, bq_dtype xt, void* y, bq_dtype yt,
+                         const float* dy, float* dx, float* dtheta, int64_t rows, void* ws, int chunks,
+                         cudaStream_t st);
+int bwd4096_chunks(int num_layers, int64_t rows);
 int bwd_chunks(int m, int num_layers, int64_t rows);
 size_t bwd_workspace_bytes(int m, int num_layers, int chunks);
 

@@ -280,6 +280,38 @@ def test_bwd_small(bq, m, layers, rows):
     assert torch.equal(dth, dth2) and torch.equal(dx, dx2)
 
 
+@pytest.mark.parametrize("layers,rows,io", [(5, 203, "f32"), (3, 1500, "bf16"), (1, 2400, "bf16_x_f32_y")])
+def test_bwd_4096_many_chunks(bq, layers, rows, io):
+    """n = 4096 backward across many token chunks: several chunks per CTA, CTAs that move
+    between layers (new cos/sin gathered mid-launch), ragged chunk boundaries, and the
+    per-layer ticket reduction; every layer compared with the float64 oracle in full."""
+    torch = H.torch()
+    ws = [wl.backward_layer_host(l, rows, m=4096) for l in range(layers)]
+    L = [make_layer(bq, w.theta) for w in ws]
+    if io == "f32":
+        xs = [H.input_f64(w.x, "bf16").astype(np.float32) for w in ws]
+        x = H.dev_f32(np.stack(xs))
+        ydt = torch.float32
+    else:
+        x = H.dev_bf16_bits(np.stack([w.x for w in ws]))
+        ydt = torch.bfloat16 if io == "bf16" else torch.float32
+    dy = H.dev_f32(np.stack([w.dy for w in ws]))
+    y, dx, dth = run_bwd(bq, L, x, dy, ydt)
+    for l, w in enumerate(ws):
+        xf = H.input_f64(w.x, "bf16")
+        dyf = w.dy.astype(np.float64)
+        yr, dxr, dthr = ob.backward(w.theta, xf, dyf)
+        if ydt == torch.float32:
+            H.assert_f32_close(H.host(y)[l], yr, xf)
+        else:
+            y32, _, _ = run_bwd(bq, [L[l]], x[l:l + 1].contiguous(), dy[l:l + 1].contiguous(), torch.float32)
+            H.assert_bf16_output(H.host(y)[l], H.host(y32)[0], yr, xf)
+        H.assert_f32_close(H.host(dx)[l], dxr, dyf)
+        check_dtheta(H.host(dth)[l].reshape(dthr.shape), dthr, ob.backward_abs_scale(w.theta, xf, dyf))
+    _, dx2, dth2 = run_bwd(bq, L, x, dy, ydt)
+    assert torch.equal(dth, dth2) and torch.equal(dx, dx2)
+
+
 def test_bwd_bf16_io(bq):
     torch = H.torch()
     w = wl.backward_layer_host(0, 300, m=4096)
