@@ -237,22 +237,45 @@ __device__ __forceinline__ void get(const float* buf, int base, float2 (&a)[4]) 
 
 // ------------------------------------------------------------------ token I/O
 
-__device__ __forceinline__ void load_x(const float* x, int tau, uint4 (&p)[2]) {
-  const uint4* s = reinterpret_cast<const uint4*>(x + 8 * tau);
-  p[0] = s[0];
-  p[1] = s[1];
+// The next token's X and dY are copied into shared memory with cp.async while the
+// current token runs.  Thread tau copies the 16-byte pieces at byte offsets
+// 16 (tau + 512 q) of each row: for X these are its own pass-0 elements (bf16:
+// one piece, fp32: two), for dY it is a share that other threads read in pass 3,
+// after a barrier.
+__device__ __forceinline__ void cp16(void* dst, const void* src) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
 }
-__device__ __forceinline__ void load_x(const __nv_bfloat16* x, int tau, uint4 (&p)[2]) {
-  p[0] = *reinterpret_cast<const uint4*>(x + 8 * tau);
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename TI>
+__device__ __forceinline__ void issue_token(const TI* x, const float* dy, float* xs, float* dys, int tau) {
+  const char* xb = reinterpret_cast<const char*>(x);
+  char* xd = reinterpret_cast<char*>(xs);
+  if constexpr (sizeof(TI) == 4) {
+    cp16(xd + 32 * tau, xb + 32 * tau);
+    cp16(xd + 32 * tau + 16, xb + 32 * tau + 16);
+  } else {
+    cp16(xd + 16 * tau, xb + 16 * tau);
+  }
+  const char* yb = reinterpret_cast<const char*>(dy);
+  char* yd = reinterpret_cast<char*>(dys);
+  cp16(yd + 16 * tau, yb + 16 * tau);
+  cp16(yd + 16 * (tau + 512), yb + 16 * (tau + 512));
 }
-__device__ __forceinline__ void unpack_x(const uint4 (&p)[2], float2 (&a)[4], float) {
-  a[0] = make_float2(__uint_as_float(p[0].x), __uint_as_float(p[0].y));
-  a[1] = make_float2(__uint_as_float(p[0].z), __uint_as_float(p[0].w));
-  a[2] = make_float2(__uint_as_float(p[1].x), __uint_as_float(p[1].y));
-  a[3] = make_float2(__uint_as_float(p[1].z), __uint_as_float(p[1].w));
+
+__device__ __forceinline__ void read_x(const float* xs, int tau, float2 (&a)[4], float) {
+  const float4 u = reinterpret_cast<const float4*>(xs)[2 * tau];
+  const float4 v = reinterpret_cast<const float4*>(xs)[2 * tau + 1];
+  a[0] = make_float2(u.x, u.y);
+  a[1] = make_float2(u.z, u.w);
+  a[2] = make_float2(v.x, v.y);
+  a[3] = make_float2(v.z, v.w);
 }
-__device__ __forceinline__ void unpack_x(const uint4 (&p)[2], float2 (&a)[4], __nv_bfloat16) {
-  const uint32_t w[4] = {p[0].x, p[0].y, p[0].z, p[0].w};
+__device__ __forceinline__ void read_x(const float* xs, int tau, float2 (&a)[4], __nv_bfloat16) {
+  const uint4 p = reinterpret_cast<const uint4*>(xs)[tau];
+  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
 #pragma unroll
   for (int k = 0; k < 4; ++k) a[k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
 }
@@ -295,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd4096(const __grid_constant__
   float* E3 = E2 + kBuf;   // v after stage 8  (pass 2 -> 3)
   float* Ga = E3 + kBuf;   // g: reverse pass 3 -> 2 and 1 -> 0
   float* Gb = Ga + kBuf;   // g: reverse pass 2 -> 1
+  float* Xs = Gb + kBuf;   // [2][M] floats: X of the current / next token (bf16 uses half)
+  float* Ds = Xs + 2 * M;  // [2][M]: dY of the current / next token
   const int tau = threadIdx.x, w = tau >> 5;
   const Bases B = make_bases(tau);
 
@@ -344,21 +369,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd4096(const __grid_constant__
 #pragma unroll
     for (int s = 0; s < kStages; ++s) acc[s][0] = acc[s][1] = make_float2(0.f, 0.f);
 
-    uint4 px[2];
-    load_x(X + t0 * M, tau, px);
+    issue_token(X + t0 * M, DY + t0 * M, Xs + (t0 & 1) * M, Ds + (t0 & 1) * M, tau);
+    cp_commit();
     uint32_t ca[8], cn[8];
     tld8(tb, ca);
     twait(ca);
 
 #pragma unroll 1
     for (long long t = t0; t < t1; ++t) {
+      const int par = static_cast<int>(t & 1);
+      cp_wait_all();  // this thread's copies of token t have landed
       float2 v[4];
-      unpack_x(px, v, TI());
-      float dyv[8];
-      const float* dyt = DY + t * M + B.p3;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) dyv[e] = dyt[512 * e];
-      if (t + 1 < t1) load_x(X + (t + 1) * M, tau, px);
+      read_x(Xs + par * M, tau, v, TI());
+      if (t + 1 < t1) issue_token(X + (t + 1) * M, DY + (t + 1) * M, Xs + (par ^ 1) * M, Ds + (par ^ 1) * M, tau);
+      cp_commit();
 
       // ---------------- forward: v <- Q v, leaving v at the ends of passes 0..2 in E1..E3
       tld8(tb + 8, cn);  rotate<0, false>(v, ca); twait(cn);
@@ -387,7 +411,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd4096(const __grid_constant__
       // ---------------- reverse sweep: s = 11 .. 0
       float2 g[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) g[k] = make_float2(dyv[2 * k], dyv[2 * k + 1]);
+      for (int k = 0; k < 4; ++k) {
+        // dY of token t: every thread's copies landed before the pass 2 -> 3 barrier
+        const float* d = Ds + par * M + B.p3;
+        g[k] = make_float2(d[512 * (2 * k)], d[512 * (2 * k + 1)]);
+      }
       // pass 3
       tld8(tb + 80, ca);
       accumulate<2>(acc[11], v, g); rotate<2, true>(g, cn); rotate<2, true>(v, cn);
@@ -462,21 +490,19 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd4096(const __grid_constant__
       __threadfence();
       const float* base = A.part + static_cast<size_t>(layer) * A.chunks * (kAcc * kThreads) + tau;
       float* out = A.dtheta + static_cast<size_t>(layer) * (kStages * (M / 2));
-#pragma unroll 1
-      for (int k0 = 0; k0 < kAcc; k0 += 4) {
-        float sum[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
-        for (int c = 0; c < A.chunks; ++c) {
-          const float* q = base + static_cast<size_t>(c) * (kAcc * kThreads) + k0 * kThreads;
+      // one chunk per step, all 48 of its loads independent (the reduction is
+      // latency-bound otherwise: it runs on one CTA per layer)
+      float sum[kAcc];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) sum[i] += __ldcg(q + i * kThreads);
-        }
+      for (int k = 0; k < kAcc; ++k) sum[k] = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < A.chunks; ++c) {
+        const float* q = base + static_cast<size_t>(c) * (kAcc * kThreads);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int k = k0 + i, s = k >> 2, pr = k & 3;
-          out[s * (M / 2) + pair_index(tau, s, pr)] = sum[i];
-        }
+        for (int k = 0; k < kAcc; ++k) sum[k] += __ldcg(q + k * kThreads);
       }
+#pragma unroll
+      for (int k = 0; k < kAcc; ++k) out[(k >> 2) * (M / 2) + pair_index(tau, k >> 2, k & 3)] = sum[k];
       if (tau == 0) A.counters[layer] = 0u;
     }
   }
@@ -488,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_bwd4096(const __grid_constant__
 template <typename TI, typename TO>
 bq_status run(const B4Args& A, cudaStream_t st) {
   auto kern = k_bwd4096<TI, TO>;
-  constexpr int smem = 5 * kBuf * static_cast<int>(sizeof(float));
+  constexpr int smem = (5 * kBuf + 4 * M) * static_cast<int>(sizeof(float));
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
   static int sms_of[64] = {};
