@@ -38,6 +38,8 @@ bq_status transform(const bq_layer* layer, const void* x, bq_dtype xt, void* y, 
   const KLayer L = make_klayer(*layer);
   if (!inverse && fast4096_supports(L, nullptr))
     return launch_fast4096(L, x, xt, y, yt, rows, nullptr, static_cast<cudaStream_t>(stream));
+  if (!inverse && kron1024_supports(L, nullptr))
+    return launch_kron1024(L, x, xt, y, yt, rows, nullptr, static_cast<cudaStream_t>(stream));
   return launch_generic(L, x, xt, y, yt, rows, inverse, nullptr, static_cast<cudaStream_t>(stream));
 }
 
@@ -56,6 +58,8 @@ bq_status quantize(const bq_layer* layer, const void* x, bq_dtype xt, int64_t ro
   QuantArgs q{bits, group, codes, scale, zero};
   if (fast4096_supports(L, &q))
     return launch_fast4096(L, x, xt, nullptr, BQ_F32, rows, &q, static_cast<cudaStream_t>(stream));
+  if (kron1024_supports(L, &q))
+    return launch_kron1024(L, x, xt, nullptr, BQ_F32, rows, &q, static_cast<cudaStream_t>(stream));
   return launch_generic(L, x, xt, nullptr, BQ_F32, rows, false, &q, static_cast<cudaStream_t>(stream));
 }
 

@@ -91,6 +91,9 @@ bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t s
 bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool fast4096_supports(const KLayer& L, const QuantArgs* q);
+bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
+                          const QuantArgs* q, cudaStream_t st);
+bool kron1024_supports(const KLayer& L, const QuantArgs* q);
 bq_status launch_generic(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt,
                          int64_t rows, bool inverse, const QuantArgs* q, cudaStream_t st);
 bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt,

@@ -468,3 +468,89 @@ def test_full_backward_32_layers(bq):
     full = dth[0].double()
     absmax = parts.abs().max().item()
     assert (full - parts).abs().max().item() <= 1e-4 * absmax + 1e-3
+
+
+# --------------------------------------------------------------------------- specialised n = 5120 = 1024 x 5 kernel
+
+def _kron_case(seed, rows, scale=1.0):
+    rng = np.random.default_rng(seed)
+    theta = wl.uniform_angles(rng, 1024)
+    O = wl.random_orthogonal(rng, 5)
+    x = (rng.standard_normal((rows, 5120)) * scale).astype(np.float32)
+    return theta, O, x
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_kron5120_fwd_many_rows(bq, io):
+    """More rows than one wave of row CTAs (3 per SM): every CTA takes several rows
+    with the next row's input prefetched; bf16 and float32 input and output."""
+    torch = H.torch()
+    rows = 148 * 3 * 2 + 5
+    theta, O, x = _kron_case(21, rows)
+    layer = make_layer(bq, theta, O)
+    idx = _sample(rows, 48, 22)
+    if io == "f32":
+        y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+        xs = x[idx].astype(np.float64)
+        H.assert_f32_close(H.host(y)[idx], ob.kron_forward(theta, O.astype(np.float64), xs, 1024), xs)
+    else:
+        xb = wl.bf16_bits_from_f32(x)
+        xd = H.dev_bf16_bits(xb)
+        y = run_fwd(bq, layer, xd, torch.bfloat16)
+        y32 = run_fwd(bq, layer, xd, torch.float32)
+        xs = H.input_f64(xb, "bf16")[idx]
+        H.assert_bf16_output(H.host(y)[idx], H.host(y32)[idx], ob.kron_forward(theta, O.astype(np.float64), xs, 1024), xs)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 64), (2, 64), (4, 128), (2, 128), (4, 256), (2, 256)])
+def test_kron5120_quant_groups(bq, bits, group):
+    theta, O, x = _kron_case(bits * 7 + group, 37, scale=2.0)
+    layer = make_layer(bq, theta, O)
+    check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, bits, group, O=O.astype(np.float64), m=1024)
+
+
+def test_kron5120_plain_form_fallback(bq):
+    """Angles whose scaled form leaves its range: the kernel's cos/sin path."""
+    torch = H.torch()
+    theta = np.full((10, 512), np.float32(np.pi / 2), np.float32)
+    theta[:, ::3] = np.float32(0.3)
+    O = wl.random_orthogonal(np.random.default_rng(3), 5)
+    layer = make_layer(bq, theta, O)
+    assert not layer.fast_form
+    x = np.random.default_rng(4).standard_normal((11, 5120)).astype(np.float32)
+    y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+    ref = ob.kron_forward(theta, O.astype(np.float64), x.astype(np.float64), 1024)
+    H.assert_f32_close(H.host(y), ref, x.astype(np.float64))
+    check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, 4, 128, O=O.astype(np.float64), m=1024)
+
+
+def test_kron5120_exact_ties(bq):
+    """theta = 0 and O = I make y = x exactly: quotients on and next to half-integers
+    must give the codes of IEEE float32 division in the fused kernel too."""
+    torch = H.torch()
+    layer = make_layer(bq, np.zeros((10, 512), np.float32), np.eye(5, dtype=np.float32))
+    rng = np.random.default_rng(12)
+    rows = []
+    for lo, hi in ((-0.5, 0.4375), (-0.7, 0.8), (-3.1, 0.2), (-1e-3, 1e-3)):
+        s = np.float32(np.float16(np.float32(np.float32(hi) - np.float32(lo)) / np.float32(15)))
+        row = rng.uniform(lo, hi, 5120).astype(np.float32)
+        k = rng.integers(-16, 16, 5120).astype(np.float32)
+        ties = ((k + np.float32(0.5)) * s).astype(np.float32)
+        sel = rng.integers(0, 3, 5120)
+        ties = np.where(sel == 1, np.nextafter(ties, np.float32(np.inf)), ties)
+        ties = np.where(sel == 2, np.nextafter(ties, np.float32(-np.inf)), ties)
+        row[1::2] = np.clip(ties, np.float32(lo), np.float32(hi))[1::2]
+        row[::128] = np.float32(lo)
+        row[1::128] = np.float32(hi)
+        rows.append(row)
+    x = np.stack(rows).astype(np.float32)
+    y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
+    assert np.array_equal(H.host(y), x)
+    for bits in (4, 2):
+        codes, scale, zero = bq.quant_outputs(x.shape[0], 5120, bits, 128, "cuda")
+        bq.bq_transform_quantize(layer, H.dev_f32(x), bits, 128, codes, scale, zero)
+        torch.cuda.synchronize()
+        c_ref, s_ref, z_ref = oq.quantize_pack(x, bits, 128)
+        assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
+        assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
+        assert np.array_equal(H.host(codes), c_ref)
