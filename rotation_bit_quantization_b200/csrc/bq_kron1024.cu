@@ -40,6 +40,7 @@ namespace {
 constexpr int M1 = 1024;
 constexpr int kT = 128;
 constexpr int kPlane = 1168;  // exchange-buffer floats per i2 plane
+constexpr int kRed = 688;     // chunk-extreme slots: cg * S <= 672 for n = 5120
 
 enum KMode { kKF32 = 0, kKBF16 = 1, kKQuant = 2 };
 
@@ -201,16 +202,18 @@ __device__ __forceinline__ void kunpack(const KPre<TI, R>& p, float2 (&a)[R][4])
 // where x' is the partner element in lane l ^ 16.
 
 template <typename TI, int MODE, int BITS, int R>
-__global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
+__global__ void __launch_bounds__(kT, 4) k_kron1024(const KronArgs A) {
   constexpr int N = M1 * R;
   constexpr float kQmax = static_cast<float>((1 << BITS) - 1);
   extern __shared__ __align__(16) float smem[];
   __shared__ uint32_t s_tmem;
-  float* bufA = smem;                  // [R][kPlane]: pass 0 -> 1
-  float* bufB = bufA + R * kPlane;     // [R][kPlane]: pass 1 -> 2
-  float* nat = bufB + R * kPlane;      // [N + 16]: the row in element order
-  float2* red = reinterpret_cast<float2*>(nat + N + 16);  // [N / 8] chunk (min, max)
-  float4* par = reinterpret_cast<float4*>(red + N / 8);   // [N / 64] group parameters
+  // one exchange buffer serves pass 0 -> 1 and pass 1 -> 2: warp w only touches
+  // positions with i1 bits 8, 9 = w until the pass 1 -> 2 barrier
+  float* bufA = smem;                  // [R][kPlane]
+  float* bufB = bufA;
+  float* nat = bufA + R * kPlane;      // [N + 16]: the row in element order
+  float2* red = reinterpret_cast<float2*>(nat + N + 16);  // [kRed] chunk (min, max), transposed
+  float4* par = reinterpret_cast<float4*>(red + kRed);    // [N / 64] group parameters
   const int tau = threadIdx.x, l = tau & 31, w = tau >> 5;
   const bool scaled = A.hdr[0] == 1.f;
 
@@ -319,6 +322,7 @@ __global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
       for (int k = 0; k < 4; ++k)
         a[r][k] = make_float2(bufA[r * kPlane + b1 + xoff<1>(2 * k)], bufA[r * kPlane + b1 + xoff<1>(2 * k + 1)]);
     KSTEP(3, 0, cn, ca); KSTEP(4, 1, ca, cn); KSTEP(5, 2, cn, ca);
+    __syncwarp();  // every lane's pass-1 reads precede the writes into the same region
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
@@ -399,7 +403,11 @@ __global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
       }
     } else {
       // per-chunk extremes -> per-group parameters (one thread per group) -> codes
-      const int cg = A.group >> 3, G = N / A.group;
+      // chunk c of group g = c / cg, j = c % cg sits at red[j * S + g]: S odd for
+      // cg >= 16 and S = 2 (mod 16) for cg = 8 keep both the writes (16 lanes per
+      // phase) and the reducers' reads conflict-free
+      const int cg = A.group >> 3, G = N / A.group, lcg = 31 - __clz(cg);
+      const int S = cg == 8 ? G + 2 : G + 1;
 #pragma unroll
       for (int q = 0; q < R; ++q) {
         float mn = fminf(yv[q][0].x, yv[q][0].y), mx = fmaxf(yv[q][0].x, yv[q][0].y);
@@ -408,13 +416,14 @@ __global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
           mn = fminf(mn, fminf(yv[q][k].x, yv[q][k].y));
           mx = fmaxf(mx, fmaxf(yv[q][k].x, yv[q][k].y));
         }
-        red[tau + kT * q] = make_float2(mn, mx);
+        const int c = tau + kT * q;
+        red[(c & (cg - 1)) * S + (c >> lcg)] = make_float2(mn, mx);
       }
       __syncthreads();
       if (tau < G) {
         float lo = FLT_MAX, hi = -FLT_MAX;
         for (int j = 0; j < cg; ++j) {
-          const float2 t = red[tau * cg + j];
+          const float2 t = red[j * S + tau];
           lo = fminf(lo, t.x);
           hi = fmaxf(hi, t.y);
         }
@@ -427,7 +436,7 @@ __global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
 #pragma unroll
       for (int q = 0; q < R; ++q) {
         const int c = tau + kT * q;
-        const float4 p = par[c / cg];
+        const float4 p = par[c >> lcg];
         const uint32_t word = rtn_codes8<BITS>(yv[q], p.x, p.y, p.z, p.w);
         if constexpr (BITS == 4) {
           *reinterpret_cast<uint32_t*>(A.codes + row * (N / 2) + 4 * c) = word;
@@ -445,7 +454,7 @@ __global__ void __launch_bounds__(kT, 3) k_kron1024(const KronArgs A) {
 
 template <int R>
 constexpr int kron_smem_bytes() {
-  return static_cast<int>(sizeof(float)) * (2 * R * kPlane + M1 * R + 16 + 2 * (M1 * R / 8) + 4 * (M1 * R / 64));
+  return static_cast<int>(sizeof(float)) * (R * kPlane + M1 * R + 16 + 2 * kRed + 4 * (M1 * R / 64));
 }
 
 template <typename TI, int MODE, int BITS, int R>
@@ -462,7 +471,7 @@ bq_status kron_launch(const KronArgs& A, cudaStream_t st) {
       return BQ_ERR_CUDA;
     sms_of[dev] = sms;
   }
-  long long grid = static_cast<long long>(sms_of[dev]) * 3;  // three row CTAs per SM
+  long long grid = static_cast<long long>(sms_of[dev]) * 4;  // four row CTAs per SM
   if (grid > A.rows) grid = A.rows;
   if (grid < 1) grid = 1;
   kern<<<static_cast<unsigned>(grid), kT, smem, st>>>(A);
