@@ -520,6 +520,41 @@ __device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long l
                                                bufBC + ((row - rb) & 1) * M, pre, c0, c1);
 }
 
+// Copies this thread's share of a tensor-memory image (NCHUNK chunks of 16
+// columns, dealt round-robin to the slots) into its lane: all loads in flight
+// first (each warp load is one contiguous 512-byte run of the [column/4][lane]
+// image), then the stores.
+template <int NCHUNK>
+__device__ __forceinline__ void fill_tmem(const float* image, uint32_t tb, int slot, int tau) {
+  const float4* src = reinterpret_cast<const float4*>(image) + tau;  // block q of lane tau at [q * 128]
+  constexpr int kMine = (NCHUNK + kSlots - 1) / kSlots;
+  float4 f[kMine * 4];
+#pragma unroll
+  for (int i = 0; i < kMine; ++i) {
+    const int c = slot + i * kSlots;
+    if (c < NCHUNK) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kMine; ++i) {
+    const int c = slot + i * kSlots;
+    if (c < NCHUNK) {
+      uint32_t v[16];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[4 * j] = __float_as_uint(f[4 * i + j].x);
+        v[4 * j + 1] = __float_as_uint(f[4 * i + j].y);
+        v[4 * j + 2] = __float_as_uint(f[4 * i + j].z);
+        v[4 * j + 3] = __float_as_uint(f[4 * i + j].w);
+      }
+      tmem_st16(tb + 16 * c, v);
+    }
+  }
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 template <typename TI, int MODE, int BITS, int GLANES>
 __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   extern __shared__ __align__(16) float smem[];
@@ -544,38 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  {
-    // each thread copies its lane's share of the image (16-column chunks dealt
-    // round-robin to the slots): all loads in flight first (each warp load is one
-    // contiguous 512-byte run of the [column/4][lane] image), then the stores
-    const float4* src = reinterpret_cast<const float4*>(A.image) + tau;  // block q of lane tau at [q * 128]
-    constexpr int kMine = (kFillChunks + kSlots - 1) / kSlots;
-    float4 f[kMine * 4];
-#pragma unroll
-    for (int i = 0; i < kMine; ++i) {
-      const int c = slot + i * kSlots;
-      if (c < kFillChunks) {
-#pragma unroll
-        for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
-      }
-    }
-#pragma unroll
-    for (int i = 0; i < kMine; ++i) {
-      const int c = slot + i * kSlots;
-      if (c < kFillChunks) {
-        uint32_t v[16];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          v[4 * j] = __float_as_uint(f[4 * i + j].x);
-          v[4 * j + 1] = __float_as_uint(f[4 * i + j].y);
-          v[4 * j + 2] = __float_as_uint(f[4 * i + j].z);
-          v[4 * j + 3] = __float_as_uint(f[4 * i + j].w);
-        }
-        tmem_st16(tb + 16 * c, v);
-      }
-    }
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-  }
+  fill_tmem<kFillChunks>(A.image, tb, slot, tau);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -632,6 +636,208 @@ bq_status dispatch_quant(const FastArgs& A, int bits, int group, cudaStream_t st
   return launch<TI, kQuant, 2, 32>(A, st);
 }
 
+
+// ------------------------------------------------------------------ inverse
+//
+// x = Q^T y: stages 11 .. 0, each the transpose [[c, s], [-s, c]] of its rotation,
+// in the forward's thread layouts visited backwards (pass C, then B, then A) with
+// the two transposes reversed.  Coefficients: the plain (cos, sin) image, whose
+// stage-s block sits at column 32 s; the scaled form's [[1, alpha], [beta, 1]]
+// steps do not invert into steps of the same shape.
+
+template <int SB>
+__device__ __forceinline__ void stage_inv(float2 (&a)[2][16], const uint32_t (&c)[32]) {
+  if constexpr (SB == 0) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int k = 2 * q + e;
+        const float cl = u2f(c[4 * q + e]), ch = u2f(c[4 * q + 2 + e]);
+        const float lo = a[0][k].x, hi = a[0][k].y;
+        a[0][k].x = fmaf(ch, hi, cl * lo);
+        a[0][k].y = fmaf(-ch, lo, cl * hi);
+      }
+  } else {
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      constexpr int kHalf = 1 << (SB - 1);
+      const int lq = low_slot<SB>(2 * q) >> 1;
+      const int hq = lq + kHalf;
+      const float2 cl = make_float2(u2f(c[4 * q]), u2f(c[4 * q + 1]));
+      const float2 ch = make_float2(u2f(c[4 * q + 2]), u2f(c[4 * q + 3]));
+      const float2 lo = a[0][lq], hi = a[0][hq];
+      a[0][lq] = __ffma2_rn(ch, hi, __fmul2_rn(cl, lo));
+      a[0][hq] = __ffma2_rn(make_float2(-ch.x, -ch.y), lo, __fmul2_rn(cl, hi));
+    }
+  }
+}
+
+// stage S of the inverse from `cur`, while the block of stage S - 1 streams into `nxt`
+template <int S, int SB>
+__device__ __forceinline__ void inv_step(float2 (&a)[2][16], uint32_t (&cur)[32], uint32_t (&nxt)[32], uint32_t tb) {
+  if constexpr (S > 0) tmem_ld32(tb + 32 * (S - 1), nxt);
+  stage_inv<SB>(a, cur);
+  if constexpr (S > 0) tmem_wait(nxt);
+}
+
+// Pass-C layout input: thread tau holds positions 8 tau + 1024 h + (0..7), h < 4.
+template <typename TI>
+__device__ __forceinline__ void prefetch_c(Prefetch<TI>& p, const TI* x, long long row, int cnt, int tau) {
+  if (cnt > 0) {
+    constexpr int kPer = Prefetch<TI>::kVec / 4;  // 16-byte vectors per group of 8 elements
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + row * M + h * 1024 + tau * 8);
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) p.v[0][kPer * h + i] = src[i];
+    }
+  }
+}
+
+template <typename TI, typename TO>
+__device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int ncnt, int slot, int tau, uint32_t tb,
+                                        float* bufAB, float* bufBC, Prefetch<TI>& pre, uint32_t (&c0)[32],
+                                        uint32_t (&c1)[32]) {
+  float2 a[2][16];
+  unpack_input<1>(pre, a);
+  prefetch_c(pre, static_cast<const TI*>(A.x), row + 1, ncnt, tau);
+  // pass C: stages 11, 10 (slot bits 4, 3); c0 holds block 11 on entry
+  inv_step<11, 4>(a, c0, c1, tb);
+  inv_step<10, 3>(a, c1, c0, tb);
+  {
+    const int sw = (tau >> 2) & 1;
+#pragma unroll
+    for (int h = 0; h < 4; ++h)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        *reinterpret_cast<float4*>(bufBC + h * 1024 + tau * 8 + 4 * (hh ^ sw)) =
+            make_float4(a[0][4 * h + 2 * hh].x, a[0][4 * h + 2 * hh].y, a[0][4 * h + 2 * hh + 1].x,
+                        a[0][4 * h + 2 * hh + 1].y);
+  }
+  group_sync(slot);
+  {
+    const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
+#pragma unroll
+    for (int rb = 0; rb < 32; rb += 2)
+      a[0][rb >> 1] = make_float2(bufBC[base + 32 * rb + 4 * sw], bufBC[base + 32 * (rb + 1) + 4 * (sw ^ 1)]);
+  }
+  // pass B: stages 9 .. 5
+  inv_step<9, 4>(a, c0, c1, tb);
+  inv_step<8, 3>(a, c1, c0, tb);
+  inv_step<7, 2>(a, c0, c1, tb);
+  inv_step<6, 1>(a, c1, c0, tb);
+  inv_step<5, 0>(a, c0, c1, tb);
+  {
+    const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
+#pragma unroll
+    for (int rb = 0; rb < 32; rb += 2) {
+      bufAB[base + 32 * rb + 4 * (cq ^ (rb & 7))] = a[0][rb >> 1].x;
+      bufAB[base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))] = a[0][rb >> 1].y;
+    }
+  }
+  __syncwarp();  // the B -> A exchange stays inside the warp (position bits 10, 11)
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 v = *reinterpret_cast<const float4*>(bufAB + tau * 32 + 4 * (c ^ (tau & 7)));
+    a[0][2 * c] = make_float2(v.x, v.y);
+    a[0][2 * c + 1] = make_float2(v.z, v.w);
+  }
+  // pass A: stages 4 .. 0, then block 11 again for the next row
+  inv_step<4, 4>(a, c1, c0, tb);
+  inv_step<3, 3>(a, c0, c1, tb);
+  inv_step<2, 2>(a, c1, c0, tb);
+  inv_step<1, 1>(a, c0, c1, tb);
+  tmem_ld32(tb + 32 * 11, c0);
+  stage_inv<0>(a, c1);
+  // pass-A layout output: 32 consecutive positions at 32 tau
+  const long long off = row * M + tau * 32;
+  if constexpr (sizeof(TO) == 4) {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(A.y) + off);
+#pragma unroll
+    for (int c = 0; c < 8; ++c) dst[c] = make_float4(a[0][2 * c].x, a[0][2 * c].y, a[0][2 * c + 1].x, a[0][2 * c + 1].y);
+  } else {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(A.y) + off);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        __nv_bfloat162 b = __floats2bfloat162_rn(a[0][4 * c + k].x, a[0][4 * c + k].y);
+        w[k] = *reinterpret_cast<uint32_t*>(&b);
+      }
+      dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  tmem_wait(c0);
+}
+
+template <typename TI, typename TO>
+__global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
+  extern __shared__ __align__(16) float smem[];
+  __shared__ uint32_t s_tmem;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
+  float* bufAB = smem + slot * (3 * M);
+  float* bufBC = bufAB + M;  // two buffers, used alternately
+  const long long G = static_cast<long long>(gridDim.x) * kSlots;
+  const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
+  const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
+
+  Prefetch<TI> pre;
+  prefetch_c(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
+  if (warp == 0) {
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(dst) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  fill_tmem<kImageInvCols / 16>(A.image, tb, slot, tau);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  uint32_t c0[32], c1[32];
+  tmem_ld32(tb + 32 * 11, c0);
+  tmem_wait(c0);
+  // the C -> B buffer alternates between rows (row i's readers and row i+2's
+  // writers are kept apart by row i+1's barrier)
+#pragma unroll 1
+  for (long long row = rb; row < re; ++row)
+    inv_row<TI, TO>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * M, pre, c0, c1);
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(s_tmem) : "memory");
+  }
+}
+
+template <typename TI, typename TO>
+bq_status launch_inv(const FastArgs& A, cudaStream_t st) {
+  auto kern = k_inv4096<TI, TO>;
+  const int smem = kSlots * 3 * M * static_cast<int>(sizeof(float));
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
+  static int sms_of[64] = {};
+  if (sms_of[dev] == 0) {
+    int sms = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return BQ_ERR_CUDA;
+    sms_of[dev] = sms;
+  }
+  long long grid = (A.rows + kSlots - 1) / kSlots;
+  if (grid > sms_of[dev]) grid = sms_of[dev];
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(A);
+  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 }  // namespace
 
 bool fast4096_supports(const KLayer& L, const QuantArgs* q) {
@@ -658,6 +864,21 @@ bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, 
   if (xt == BQ_F32)
     return yt == BQ_F32 ? launch<float, kOutF32, 4, 16>(A, st) : launch<float, kOutBF16, 4, 16>(A, st);
   return yt == BQ_F32 ? launch<__nv_bfloat16, kOutF32, 4, 16>(A, st) : launch<__nv_bfloat16, kOutBF16, 4, 16>(A, st);
+}
+
+bq_status launch_inv4096(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
+                         cudaStream_t st) {
+  FastArgs A;
+  A.x = y;  // the kernel reads A.x and writes A.y
+  A.y = x;
+  A.rows = rows;
+  A.image = L.image_inv;
+  A.hdr = L.hdr;
+  A.codes = nullptr;
+  A.scale = nullptr;
+  A.zero = nullptr;
+  if (yt == BQ_F32) return xt == BQ_F32 ? launch_inv<float, float>(A, st) : launch_inv<float, __nv_bfloat16>(A, st);
+  return xt == BQ_F32 ? launch_inv<__nv_bfloat16, float>(A, st) : launch_inv<__nv_bfloat16, __nv_bfloat16>(A, st);
 }
 
 }  // namespace bq

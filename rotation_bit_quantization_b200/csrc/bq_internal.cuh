@@ -27,13 +27,16 @@ constexpr int kMaxGroup = 256;     // largest quantization group
 //                      n = 4096 kernel: lane t, column c (float4 block c/4 of
 //                      lane t) holds the coefficient thread t needs at that
 //                      column (see bq_fast4096.cu)
+//   image_inv [96][128][4] (m == 4096 only) the same lanes and stage columns
+//                      holding plain (cos, sin) for the inverse kernel
 struct TableLayout {
   int m, L;
-  size_t off_cs, off_fast, off_sigma, off_image, total;
+  size_t off_cs, off_fast, off_sigma, off_image, off_image_inv, total;
 };
 
 constexpr int kImageLanes = 128;
 constexpr int kImageCols = 416;
+constexpr int kImageInvCols = 384;
 
 __host__ __device__ inline int ilog2(int v) {
   int l = 0;
@@ -51,7 +54,8 @@ __host__ __device__ inline TableLayout table_layout(int m) {
   t.off_fast = t.off_cs + round4(size_t(t.L) * m);
   t.off_sigma = t.off_fast + round4(size_t(t.L) * m);
   t.off_image = t.off_sigma + round4(size_t(m));
-  t.total = t.off_image + (m == 4096 ? size_t(kImageLanes) * kImageCols : 0);
+  t.off_image_inv = t.off_image + (m == 4096 ? size_t(kImageLanes) * kImageCols : 0);
+  t.total = t.off_image_inv + (m == 4096 ? size_t(kImageLanes) * kImageInvCols : 0);
   return t;
 }
 
@@ -63,6 +67,7 @@ struct KLayer {
   const float* sigma;   // [m]
   const float* hdr;     // header (flag at hdr[0])
   const float* image;   // tensor-memory image (m == 4096) or nullptr
+  const float* image_inv;  // plain-form image for the inverse (m == 4096) or nullptr
   const float* O;       // [r][r] or nullptr
 };
 
@@ -75,6 +80,7 @@ inline KLayer make_klayer(const bq_layer& l) {
   k.sigma = l.table + t.off_sigma;
   k.hdr = l.table;
   k.image = l.m == 4096 ? l.table + t.off_image : nullptr;
+  k.image_inv = l.m == 4096 ? l.table + t.off_image_inv : nullptr;
   k.O = l.O;
   return k;
 }
@@ -91,6 +97,8 @@ bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t s
 bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool fast4096_supports(const KLayer& L, const QuantArgs* q);
+bq_status launch_inv4096(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
+                         cudaStream_t st);
 bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool kron1024_supports(const KLayer& L, const QuantArgs* q);

@@ -95,11 +95,15 @@ __device__ __forceinline__ int pos_pass(int pass, int t, int e) {
 // element of the thread's (2q + e)-th pair and column 4q + 2 + e that of its
 // high element: (alpha, beta) of the scaled form, or (cos, sin) when the
 // scaled form is out of range (header flag 0; the output scale is then 1).
+// The inverse image (columns [0, 384) only) always holds (cos, sin).
 __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= kImageLanes * kImageCols) return;
-  const int t = idx / kImageCols, col = idx % kImageCols;
-  const bool scaled = table[0] == 1.f;
+  int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  const bool inv = idx >= kImageLanes * kImageCols;
+  if (inv) idx -= kImageLanes * kImageCols;
+  if (idx >= kImageLanes * (inv ? kImageInvCols : kImageCols)) return;
+  const int ncol = inv ? kImageInvCols : kImageCols;
+  const int t = idx / ncol, col = idx % ncol;
+  const bool scaled = !inv && table[0] == 1.f;
   const float2* cs = reinterpret_cast<const float2*>(table + tl.off_cs);
   const float* fast = table + tl.off_fast;
   const float* sigma = table + tl.off_sigma;
@@ -123,7 +127,7 @@ __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
       v = high ? c.y : c.x;
     }
   }
-  table[tl.off_image + (size_t(col >> 2) * kImageLanes + t) * 4 + (col & 3)] = v;
+  table[(inv ? tl.off_image_inv : tl.off_image) + (size_t(col >> 2) * kImageLanes + t) * 4 + (col & 3)] = v;
 }
 
 }  // namespace
@@ -137,7 +141,7 @@ bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t s
   }
   k_prepare<<<1, 1024, smem, st>>>(theta, table, tl);
   if (m == 4096) {
-    const int total = kImageLanes * kImageCols;
+    const int total = kImageLanes * (kImageCols + kImageInvCols);
     k_image4096<<<(total + 255) / 256, 256, 0, st>>>(table, tl);
   }
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;

@@ -554,3 +554,56 @@ def test_kron5120_exact_ties(bq):
         assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
         assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
         assert np.array_equal(H.host(codes), c_ref)
+
+
+# --------------------------------------------------------------------------- specialised n = 4096 inverse
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_inv4096_many_rows(bq, io):
+    """x = Q^T y on more rows than one wave of row groups (every group takes several
+    rows, with the next row prefetched), bf16 and float32, and in place."""
+    torch = H.torch()
+    rng = np.random.default_rng(31)
+    theta = wl.uniform_angles(rng, 4096)
+    layer = make_layer(bq, theta)
+    rows = 148 * 3 * 2 + 7
+    y = rng.standard_normal((rows, 4096)).astype(np.float32)
+    idx = _sample(rows, 40, 32)
+    if io == "f32":
+        yd = H.dev_f32(y)
+        x = torch.empty_like(yd)
+        bq.bq_butterfly_inv(layer, yd, x)
+        torch.cuda.synchronize()
+        ys = y[idx].astype(np.float64)
+        H.assert_f32_close(H.host(x)[idx], ob.inverse(theta, ys), ys)
+        bq.bq_butterfly_inv(layer, yd, yd)   # in place
+        torch.cuda.synchronize()
+        assert torch.equal(yd, x)
+    else:
+        yb = wl.bf16_bits_from_f32(y)
+        yd = H.dev_bf16_bits(yb)
+        x16 = torch.empty_like(yd)
+        x32 = torch.empty(yd.shape, dtype=torch.float32, device="cuda")
+        bq.bq_butterfly_inv(layer, yd, x16)
+        bq.bq_butterfly_inv(layer, yd, x32)
+        torch.cuda.synchronize()
+        ys = H.input_f64(yb, "bf16")[idx]
+        ref = ob.inverse(theta, ys)
+        H.assert_f32_close(H.host(x32)[idx], ref, ys)
+        H.assert_bf16_output(H.host(x16)[idx], H.host(x32)[idx], ref, ys)
+
+
+def test_inv4096_round_trip_full_rows(bq):
+    """Q^T (Q x) = x at the act n = 4096 workload size (2048 rows), forward on the
+    scaled form and inverse on the plain form."""
+    torch = H.torch()
+    w = wl.act_4096()
+    layer = make_layer(bq, w.theta)
+    assert layer.fast_form
+    xd = H.dev_bf16_bits(w.x)
+    y = run_fwd(bq, layer, xd, torch.float32)
+    back = torch.empty_like(y)
+    bq.bq_butterfly_inv(layer, y, back)
+    torch.cuda.synchronize()
+    xf = H.input_f64(w.x, "bf16")
+    H.assert_f32_close(H.host(back), xf, xf)
