@@ -36,7 +36,7 @@
 //    the current row is processed.
 #include <cfloat>
 
-#include "bq_internal.cuh"
+#include "bq_rtn.cuh"
 
 namespace bq {
 namespace {
@@ -252,36 +252,15 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// Codes of 8 values by IEEE division, for sets where the fast path below cannot
-// prove its result (kept out of line: it runs for roughly one set in 10^4).
-template <int BITS>
-__device__ __noinline__ uint32_t codes_by_division(float y0, float y1, float y2, float y3, float y4, float y5,
-                                                    float y6, float y7, float s, float z) {
-  const float qmax = static_cast<float>((1 << BITS) - 1);
-  const float y[8] = {y0, y1, y2, y3, y4, y5, y6, y7};
-  uint32_t word = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float t = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(y[e], s)), z), 0.f), qmax);
-    word |= static_cast<uint32_t>(t) << (BITS * e);
-  }
-  return word;
-}
-
 // Per-group asymmetric RTN of the R rows held in pass-C layout, packing and stores.
 //
-// Codes are q = clamp(rint(y / s) + z, 0, qmax) with y / s the correctly rounded
-// float32 quotient.  Fast path: v = y * inv with inv = 1 / s correctly rounded,
-// so |v - y/s| <= 2^-23 |y/s| and |v - RN(y/s)| <= 1.5 * 2^-23 |y/s|.  When v is
-// farther than vmax * 2^-20 from every half-integer (vmax bounds |v| over the
-// group; the factor 2^-20 also absorbs the rounding of the threshold itself),
-// RN(y/s) lies on the same side of the same half-integer and
-// rint(RN(y/s)) = rint(v) exactly.  rint(v) is
-// taken with the float32 magic constant 1.5 * 2^23 (round-half-even addition),
-// with z folded into the constant (no tie can occur on the fast path, so
-// rint(v) + z = RN(v + z) there); the bit pattern then carries the code.  A set of
-// 8 values with any element too close to a tie (or |v| >= 2^22), or whose group
-// would need clamping, is redone with IEEE division and clamping.
+// Group extremes: 3-input min / max over each 8-value set, then a recursive-halving
+// shuffle reduction after which lane l holds set bitrev(l & (S-1)) of its group.
+// Every lane computes that group's parameters (scale16, s, z, 1 / s and the tie
+// threshold, as in rtn_params); each set then takes them by shuffle from the lane
+// that holds them and is coded by rtn_codes8 (exact RTN: see bq_rtn.cuh).  One
+// reducing warp per row group with the parameters in shared memory issues fewer
+// instructions but adds two row-group barriers, and measured slower at 2048 rows.
 template <int BITS, int GLANES, int R>
 __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const FastArgs& A, long long row0, int tau,
                                                int lane) {
@@ -346,10 +325,7 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
       A.zero[row * GPR + g] = __half_as_ushort(__float2half_rn(z));
     }
   }
-  // rint(v) + z as the bit pattern of v + (1.5 * 2^23 + z): valid because the fast
-  // path only accepts v away from half-integers (no rounding tie can occur).  The
-  // code sits in the low bits (the constant's bits start at bit 22), so
-  // bits(t0) + bits(t1) << BITS ... has the packed byte in its low byte.
+  // codes of each set with its group's parameters (from the lane that reduced it)
   const float mz = __fadd_rn(12582912.f, z);
 #pragma unroll
   for (int k = 0; k < S; ++k) {
@@ -359,34 +335,8 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
     const float mzk = __shfl_sync(0xffffffffu, mz, src);
     const float sk = __shfl_sync(0xffffffffu, s, src);
     const int r = k >> 2, h = k & 3;
-    const float2 iv = make_float2(invk, invk), m2 = make_float2(mzk, mzk);
-    const float2 nm2 = make_float2(-mzk, -mzk), neg1 = make_float2(-1.f, -1.f);
-    bool exact = true;
-    uint32_t b[8];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const float2 v = __fmul2_rn(a[r][4 * h + q], iv);
-      const float2 t = __fadd2_rn(v, m2);
-      const float2 e = __ffma2_rn(__fadd2_rn(t, nm2), neg1, v);  // v - rint(v), exact
-      exact = exact & (fabsf(e.x) < thrk) & (fabsf(e.y) < thrk);
-      b[2 * q] = __float_as_uint(t.x);
-      b[2 * q + 1] = __float_as_uint(t.y);
-    }
-    uint32_t word;
-    if constexpr (BITS == 4) {
-      const uint32_t p0 = b[0] + (b[1] << 4), p1 = b[2] + (b[3] << 4);
-      const uint32_t p2 = b[4] + (b[5] << 4), p3 = b[6] + (b[7] << 4);
-      word = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040), 0x5410);
-    } else {
-      const uint32_t p0 = b[0] + (b[1] << 2) + (b[2] << 4) + (b[3] << 6);
-      const uint32_t p1 = b[4] + (b[5] << 2) + (b[6] << 4) + (b[7] << 6);
-      word = __byte_perm(p0, p1, 0x0040) & 0xffffu;
-    }
-    if (!exact) {
-      word = codes_by_division<BITS>(a[r][4 * h].x, a[r][4 * h].y, a[r][4 * h + 1].x, a[r][4 * h + 1].y,
-                                     a[r][4 * h + 2].x, a[r][4 * h + 2].y, a[r][4 * h + 3].x, a[r][4 * h + 3].y,
-                                     sk, __fadd_rn(mzk, -12582912.f));
-    }
+    const float2 y[4] = {a[r][4 * h], a[r][4 * h + 1], a[r][4 * h + 2], a[r][4 * h + 3]};
+    const uint32_t word = rtn_codes8<BITS>(y, invk, thrk, mzk, sk);
     const long long row = row0 + r;
     if constexpr (BITS == 4) {
       *reinterpret_cast<uint32_t*>(A.codes + row * (M / 2) + h * 512 + tau * 4) = word;

@@ -8,18 +8,24 @@
 //   q = clamp(rint(y / s) + z, 0, qmax)  with IEEE float32 division, rint
 //   half-to-even.
 //
-// Fast path: v = y * inv with inv = 1 / s correctly rounded, so
-// |v - RN(y / s)| <= 1.5 * 2^-23 |y / s|.  When v is farther than vmax * 2^-20
-// from every half-integer (vmax bounds |v| over the group), rint(RN(y / s)) =
-// rint(v).  rint(v) + z is taken as the bit pattern of v + (1.5 * 2^23 + z)
-// (round-half-even addition; no tie can occur on the fast path), so the code
-// sits in the low bits.  A set of 8 values with any element near a tie, or a
-// group whose extremes would need clamping, is redone with IEEE division.
+// Fast path: with inv = 1 / s correctly rounded, y * inv + (1.5 * 2^23 + z) is
+// rounded once to an integer whose low bits are the code; when y * inv is far
+// enough from every half-integer (relative to vmax, a bound on |y * inv| over
+// the group) that integer is rint(RN(y / s)) + z (see rtn_codes8).  A set of 8
+// values with any element near a tie (or a NaN), or a group whose extremes
+// would need clamping, is redone with IEEE division.
 #pragma once
 
 #include "bq_internal.cuh"
 
 namespace bq {
+
+// 3-input maximum that returns NaN if any input is NaN
+__device__ __forceinline__ float max_nan3(float a, float b, float c) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
 
 struct RtnParams {
   float inv;   // 1 / s, correctly rounded
@@ -71,18 +77,27 @@ __device__ __noinline__ uint32_t rtn_codes_by_division(float y0, float y1, float
 
 // Packed codes of 8 consecutive values (lowest element in the lowest bits):
 // INT4 -> 32 bits, INT2 -> 16 bits.
+//
+// With P = y * inv exact and |P| < 2^22: t = RN(P + mz) = mz + rint(P) (the sum
+// lies in (2^23, 2^24), where the float32 spacing is 1), r = t - mz = rint(P)
+// exactly, and e = RN(r - P) is within 2^-25 of r - P.  The threshold
+// thr = RN(0.5 - vmax 2^-20) then leaves P at least vmax 2^-20 - 2^-24 away
+// from every half-integer whenever |e| < thr, which exceeds
+// |RN(y / s) - P| <= 2^-23 vmax once vmax > 1/14; below that |P| and |y / s|
+// are both under 1/2 and every code is z.  So rint(RN(y / s)) = r on the
+// fast path, and t's low bits carry r + z.
 template <int BITS>
 __device__ __forceinline__ uint32_t rtn_codes8(const float2 (&y)[4], float inv, float thr, float mz, float s) {
-  const float2 iv = make_float2(inv, inv), m2 = make_float2(mz, mz);
-  const float2 nm2 = make_float2(-mz, -mz), neg1 = make_float2(-1.f, -1.f);
-  bool exact = true;
+  const float2 iv = make_float2(inv, inv), niv = make_float2(-inv, -inv);
+  const float2 m2 = make_float2(mz, mz), nm2 = make_float2(-mz, -mz);
   uint32_t b[8];
+  float emax = 0.f;
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    const float2 v = __fmul2_rn(y[q], iv);
-    const float2 t = __fadd2_rn(v, m2);
-    const float2 e = __ffma2_rn(__fadd2_rn(t, nm2), neg1, v);  // v - rint(v), exact
-    exact = exact & (fabsf(e.x) < thr) & (fabsf(e.y) < thr);
+    const float2 t = __ffma2_rn(y[q], iv, m2);        // mz + rint(y * inv)
+    const float2 r = __fadd2_rn(t, nm2);               // rint(y * inv), exact
+    const float2 e = __ffma2_rn(y[q], niv, r);         // r - y * inv, one rounding
+    emax = max_nan3(emax, fabsf(e.x), fabsf(e.y));  // a NaN goes to the slow path
     b[2 * q] = __float_as_uint(t.x);
     b[2 * q + 1] = __float_as_uint(t.y);
   }
@@ -96,7 +111,7 @@ __device__ __forceinline__ uint32_t rtn_codes8(const float2 (&y)[4], float inv, 
     const uint32_t p1 = b[4] + (b[5] << 2) + (b[6] << 4) + (b[7] << 6);
     word = __byte_perm(p0, p1, 0x0040) & 0xffffu;
   }
-  if (!exact)
+  if (!(emax < thr))
     word = rtn_codes_by_division<BITS>(y[0].x, y[0].y, y[1].x, y[1].y, y[2].x, y[2].y, y[3].x, y[3].y, s,
                                        __fadd_rn(mz, -12582912.f));
   return word;
