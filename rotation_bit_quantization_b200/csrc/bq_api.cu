@@ -40,6 +40,8 @@ bq_status transform(const bq_layer* layer, const void* x, bq_dtype xt, void* y, 
     return launch_fast4096(L, x, xt, y, yt, rows, nullptr, static_cast<cudaStream_t>(stream));
   if (inverse && fast4096_supports(L, nullptr))
     return launch_inv4096(L, x, xt, y, yt, rows, static_cast<cudaStream_t>(stream));
+  if (inverse && kron1024_supports(L, nullptr))
+    return launch_kron1024_inv(L, x, xt, y, yt, rows, static_cast<cudaStream_t>(stream));
   if (!inverse && kron1024_supports(L, nullptr))
     return launch_kron1024(L, x, xt, y, yt, rows, nullptr, static_cast<cudaStream_t>(stream));
   return launch_generic(L, x, xt, y, yt, rows, inverse, nullptr, static_cast<cudaStream_t>(stream));

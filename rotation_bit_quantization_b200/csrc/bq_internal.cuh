@@ -102,6 +102,8 @@ bq_status launch_inv4096(const KLayer& L, const void* y, bq_dtype yt, void* x, b
 bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool kron1024_supports(const KLayer& L, const QuantArgs* q);
+bq_status launch_kron1024_inv(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
+                              cudaStream_t st);
 bq_status launch_generic(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt,
                          int64_t rows, bool inverse, const QuantArgs* q, cudaStream_t st);
 bq_status launch_bwd(const KLayer* layers, int num_layers, const void* x, bq_dtype xt,

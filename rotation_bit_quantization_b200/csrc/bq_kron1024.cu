@@ -484,6 +484,277 @@ bq_status kron_dispatch(const KronArgs& A, bq_dtype yt, const QuantArgs* q, cuda
   return yt == BQ_F32 ? kron_launch<TI, kKF32, 4, R>(A, st) : kron_launch<TI, kKBF16, 4, R>(A, st);
 }
 
+
+// ------------------------------------------------------------------ inverse
+//
+// x = (B_1024^T (x) O_R^T) y: the forward's layouts visited backwards with plain
+// cos/sin (the scaled form's steps do not invert into steps of the same shape).
+// The row is read in element-order chunks into shared memory and picked up in
+// pass-2 layout; stage 9 runs across lanes, stages 8..0 in registers with the
+// exchanges reversed; O_R^T is applied in pass 0, which stores contiguously.
+// Tensor-memory columns: 8 s for register stage s (cos, sin), 72 + e / 80 + e the
+// stage-9 (cos, -+sin) of element e: y = k1 x + k2 x'.
+
+template <int SB, int R>
+__device__ __forceinline__ void stage_inv(float2 (&a)[R][4], const uint32_t (&c)[8]) {
+  if constexpr (SB == 0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float cl = u2f(c[k]), ch = u2f(c[4 + k]);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float lo = a[r][k].x, hi = a[r][k].y;
+        a[r][k].x = fmaf(ch, hi, cl * lo);
+        a[r][k].y = fmaf(-ch, lo, cl * hi);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int il = SB == 1 ? 2 * h : h, ih = SB == 1 ? 2 * h + 1 : h + 2;
+      const float2 cl = make_float2(u2f(c[2 * h]), u2f(c[2 * h + 1]));
+      const float2 ch = make_float2(u2f(c[4 + 2 * h]), u2f(c[5 + 2 * h]));
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float2 lo = a[r][il], hi = a[r][ih];
+        a[r][il] = __ffma2_rn(ch, hi, __fmul2_rn(cl, lo));
+        a[r][ih] = __ffma2_rn(make_float2(-ch.x, -ch.y), lo, __fmul2_rn(cl, hi));
+      }
+    }
+  }
+}
+
+// chunks c = tau + 128 q (q < R) of 8 consecutive elements, one row ahead
+template <typename TI, int R>
+__device__ __forceinline__ void kprefetch_chunks(KPre<TI, R>& p, const TI* row, int tau) {
+  constexpr int kPer = KPre<TI, R>::kVec / R;  // 16-byte vectors per chunk
+#pragma unroll
+  for (int q = 0; q < R; ++q) {
+    const uint4* s = reinterpret_cast<const uint4*>(row + 8 * (tau + kT * q));
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) p.v[kPer * q + i] = s[i];
+  }
+}
+
+template <typename TI, int R>
+__device__ __forceinline__ void kunpack_chunks(const KPre<TI, R>& p, float2 (&yv)[R][4]) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(p.v);
+#pragma unroll
+  for (int q = 0; q < R; ++q)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if constexpr (sizeof(TI) == 4) {
+        yv[q][k] = make_float2(__uint_as_float(w[8 * q + 2 * k]), __uint_as_float(w[8 * q + 2 * k + 1]));
+      } else {
+        const uint32_t u = w[4 * q + k];
+        yv[q][k] = make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+      }
+    }
+}
+
+template <typename TI, typename TO, int R>
+__global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
+  constexpr int N = M1 * R;
+  extern __shared__ __align__(16) float smem[];
+  __shared__ uint32_t s_tmem;
+  float* xbuf = smem;              // [R][kPlane]
+  float* nat = xbuf + R * kPlane;  // [N + 16]
+  const int tau = threadIdx.x, l = tau & 31, w = tau >> 5;
+
+  if (w == 0) {
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 128;" ::"r"(dst) : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  cta_sync();
+  const uint32_t tb = s_tmem + (static_cast<uint32_t>(32 * w) << 16);
+  {
+#pragma unroll 1
+    for (int s = 0; s < 9; ++s) {
+      const int P = s / 3, SB = s % 3;
+      uint32_t c[8];
+#pragma unroll
+      for (int pr = 0; pr < 4; ++pr) {
+        const int ilo = pos_pass(P, tau, e_low(pr, SB));
+        const float2 t = A.cs[s * (M1 / 2) + (((ilo >> (s + 1)) << s) | (ilo & ((1 << s) - 1)))];
+        c[pr] = __float_as_uint(t.x);
+        c[4 + pr] = __float_as_uint(t.y);
+      }
+      tst8(tb + 8 * s, c);
+    }
+    uint32_t k1[8], k2[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int i1 = pos_pass(2, tau, e);
+      const float2 t = A.cs[9 * (M1 / 2) + (i1 & 511)];
+      k1[e] = __float_as_uint(t.x);
+      k2[e] = __float_as_uint(((i1 >> 9) & 1) ? -t.y : t.y);
+    }
+    tst8(tb + 72, k1);
+    tst8(tb + 80, k2);
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+  }
+  cta_sync();
+
+  float o[R][R];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int q = 0; q < R; ++q) o[r][q] = A.O[r * R + q];
+
+  const int b0 = xbase(0, tau), b1 = xbase(1, tau), b2 = xbase(2, tau);
+  const int nb = pos_pass(2, tau, 0) * R + 16 * (l >> 4);
+  const int hsw = (tau >> 2) & 1;
+  const TI* Y = static_cast<const TI*>(A.x);
+
+  KPre<TI, R> pre;
+  if (blockIdx.x < A.rows) kprefetch_chunks<TI, R>(pre, Y + static_cast<long long>(blockIdx.x) * N, tau);
+  uint32_t ca[8], cn[8];
+  tld8(tb + 72, cn);
+  tld8(tb + 80, ca);
+  twait(cn);
+  twait(ca);
+
+#define KISTEP(S, SB, CUR, NXT) \
+  tld8(tb + 8 * ((S) - 1), NXT); stage_inv<SB, R>(a, CUR); twait(NXT)
+
+#pragma unroll 1
+  for (long long row = blockIdx.x; row < A.rows; row += gridDim.x) {
+    {
+      float2 yv[R][4];
+      kunpack_chunks<TI, R>(pre, yv);
+      if (row + gridDim.x < A.rows) kprefetch_chunks<TI, R>(pre, Y + (row + gridDim.x) * N, tau);
+#pragma unroll
+      for (int q = 0; q < R; ++q) {
+        const int c = tau + kT * q;
+        float* dst = nat + 8 * c + (8 * c >= 512 * R ? 16 : 0);
+        const float4 lo = make_float4(yv[q][0].x, yv[q][0].y, yv[q][1].x, yv[q][1].y);
+        const float4 hi = make_float4(yv[q][2].x, yv[q][2].y, yv[q][3].x, yv[q][3].y);
+        *reinterpret_cast<float4*>(dst + 4 * hsw) = hsw ? hi : lo;
+        *reinterpret_cast<float4*>(dst + 4 * (hsw ^ 1)) = hsw ? lo : hi;
+      }
+    }
+    __syncthreads();
+    float2 a[R][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const float x0 = nat[nb + 64 * R * (2 * k) + r], x1 = nat[nb + 64 * R * (2 * k + 1) + r];
+        const float p0 = __shfl_xor_sync(0xffffffffu, x0, 16), p1 = __shfl_xor_sync(0xffffffffu, x1, 16);
+        a[r][k] = make_float2(fmaf(u2f(ca[2 * k]), p0, u2f(cn[2 * k]) * x0),
+                              fmaf(u2f(ca[2 * k + 1]), p1, u2f(cn[2 * k + 1]) * x1));
+      }
+    tld8(tb + 64, ca);
+    twait(ca);
+    KISTEP(8, 2, ca, cn); KISTEP(7, 1, cn, ca); KISTEP(6, 0, ca, cn);
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        xbuf[r * kPlane + b2 + xoff<2>(2 * k)] = a[r][k].x;
+        xbuf[r * kPlane + b2 + xoff<2>(2 * k + 1)] = a[r][k].y;
+      }
+    __syncthreads();
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        a[r][k] = make_float2(xbuf[r * kPlane + b1 + xoff<1>(2 * k)], xbuf[r * kPlane + b1 + xoff<1>(2 * k + 1)]);
+    KISTEP(5, 2, cn, ca); KISTEP(4, 1, ca, cn); KISTEP(3, 0, cn, ca);
+    __syncwarp();  // every lane's pass-1 reads precede the writes into the same region
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        xbuf[r * kPlane + b1 + xoff<1>(2 * k)] = a[r][k].x;
+        xbuf[r * kPlane + b1 + xoff<1>(2 * k + 1)] = a[r][k].y;
+      }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const float4 u = *reinterpret_cast<const float4*>(xbuf + r * kPlane + b0);
+      const float4 v = *reinterpret_cast<const float4*>(xbuf + r * kPlane + b0 + 4);
+      a[r][0] = make_float2(u.x, u.y);
+      a[r][1] = make_float2(u.z, u.w);
+      a[r][2] = make_float2(v.x, v.y);
+      a[r][3] = make_float2(v.z, v.w);
+    }
+    KISTEP(2, 2, ca, cn); KISTEP(1, 1, cn, ca);
+    stage_inv<0, R>(a, ca);
+    tld8(tb + 72, cn);  // stage 9 of the next row
+    tld8(tb + 80, ca);
+
+    // O_R^T on every group of R, then the pass-0 elements (contiguous) to memory
+    float2 out[R][4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        float2 acc = __fmul2_rn(make_float2(o[0][r], o[0][r]), a[0][k]);
+#pragma unroll
+        for (int q = 1; q < R; ++q) acc = __ffma2_rn(make_float2(o[q][r], o[q][r]), a[q][k], acc);
+        out[r][k] = acc;
+      }
+    // element 8 R tau + j is (e, i2) = (j / R, j % R)
+    if constexpr (sizeof(TO) == 4) {
+      float* dst = static_cast<float*>(A.y) + row * N + 8 * R * tau;
+#pragma unroll
+      for (int v = 0; v < 2 * R; ++v) {
+        float f[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int j = 4 * v + t, e = j / R, r = j % R;
+          f[t] = (e & 1) ? out[r][e >> 1].y : out[r][e >> 1].x;
+        }
+        reinterpret_cast<float4*>(dst)[v] = make_float4(f[0], f[1], f[2], f[3]);
+      }
+    } else {
+      __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(A.y) + row * N + 8 * R * tau;
+#pragma unroll
+      for (int v = 0; v < R; ++v) {
+        uint32_t u[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int j0 = 8 * v + 2 * t, j1 = j0 + 1;
+          const float f0 = ((j0 / R) & 1) ? out[j0 % R][(j0 / R) >> 1].y : out[j0 % R][(j0 / R) >> 1].x;
+          const float f1 = ((j1 / R) & 1) ? out[j1 % R][(j1 / R) >> 1].y : out[j1 % R][(j1 / R) >> 1].x;
+          __nv_bfloat162 b = __floats2bfloat162_rn(f0, f1);
+          u[t] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        reinterpret_cast<uint4*>(dst)[v] = make_uint4(u[0], u[1], u[2], u[3]);
+      }
+    }
+    twait(cn);
+    twait(ca);
+  }
+#undef KISTEP
+
+  cta_sync();
+  if (w == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 128;" ::"r"(s_tmem) : "memory");
+}
+
+template <typename TI, typename TO, int R>
+bq_status kron_inv_launch(const KronArgs& A, cudaStream_t st) {
+  auto kern = k_kron1024_inv<TI, TO, R>;
+  constexpr int smem = kron_smem_bytes<R>();
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
+  static int sms_of[64] = {};
+  if (sms_of[dev] == 0) {
+    int sms = 0;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+      return BQ_ERR_CUDA;
+    sms_of[dev] = sms;
+  }
+  long long grid = static_cast<long long>(sms_of[dev]) * 4;
+  if (grid > A.rows) grid = A.rows;
+  if (grid < 1) grid = 1;
+  kern<<<static_cast<unsigned>(grid), kT, smem, st>>>(A);
+  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 }  // namespace
 
 bool kron1024_supports(const KLayer& L, const QuantArgs* q) {
@@ -508,6 +779,27 @@ bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, 
   A.zero = q ? q->zero : nullptr;
   A.group = q ? q->group : 128;
   return xt == BQ_F32 ? kron_dispatch<float, 5>(A, yt, q, st) : kron_dispatch<__nv_bfloat16, 5>(A, yt, q, st);
+}
+
+bq_status launch_kron1024_inv(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
+                              cudaStream_t st) {
+  KronArgs A;
+  A.x = y;  // the kernel reads A.x and writes A.y
+  A.y = x;
+  A.rows = rows;
+  A.fast = L.fast;
+  A.sigma = L.sigma;
+  A.cs = L.cs;
+  A.hdr = L.hdr;
+  A.O = L.O;
+  A.codes = nullptr;
+  A.scale = nullptr;
+  A.zero = nullptr;
+  A.group = 128;
+  if (yt == BQ_F32)
+    return xt == BQ_F32 ? kron_inv_launch<float, float, 5>(A, st) : kron_inv_launch<float, __nv_bfloat16, 5>(A, st);
+  return xt == BQ_F32 ? kron_inv_launch<__nv_bfloat16, float, 5>(A, st)
+                      : kron_inv_launch<__nv_bfloat16, __nv_bfloat16, 5>(A, st);
 }
 
 }  // namespace bq

@@ -607,3 +607,46 @@ def test_inv4096_round_trip_full_rows(bq):
     torch.cuda.synchronize()
     xf = H.input_f64(w.x, "bf16")
     H.assert_f32_close(H.host(back), xf, xf)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_kron5120_inverse_many_rows(bq, io):
+    """x = (B^T (x) O^T) y on more rows than one wave of row CTAs, bf16 and float32."""
+    torch = H.torch()
+    rows = 148 * 4 + 9
+    theta, O, y = _kron_case(41, rows)
+    layer = make_layer(bq, theta, O)
+    idx = _sample(rows, 40, 42)
+    if io == "f32":
+        yd = H.dev_f32(y)
+        x = torch.empty_like(yd)
+        bq.bq_butterfly_inv(layer, yd, x)
+        torch.cuda.synchronize()
+        ys = y[idx].astype(np.float64)
+        H.assert_f32_close(H.host(x)[idx], ob.kron_inverse(theta, O.astype(np.float64), ys, 1024), ys)
+    else:
+        yb = wl.bf16_bits_from_f32(y)
+        yd = H.dev_bf16_bits(yb)
+        x16 = torch.empty_like(yd)
+        x32 = torch.empty(yd.shape, dtype=torch.float32, device="cuda")
+        bq.bq_butterfly_inv(layer, yd, x16)
+        bq.bq_butterfly_inv(layer, yd, x32)
+        torch.cuda.synchronize()
+        ys = H.input_f64(yb, "bf16")[idx]
+        ref = ob.kron_inverse(theta, O.astype(np.float64), ys, 1024)
+        H.assert_f32_close(H.host(x32)[idx], ref, ys)
+        H.assert_bf16_output(H.host(x16)[idx], H.host(x32)[idx], ref, ys)
+
+
+def test_kron5120_round_trip_full_rows(bq):
+    """Q^T (Q x) = x at the act n = 5120 workload size (8192 rows)."""
+    torch = H.torch()
+    w = wl.act_5120()
+    layer = make_layer(bq, w.theta, w.O)
+    y = run_fwd(bq, layer, H.dev_bf16_bits(w.x), torch.float32)
+    back = torch.empty_like(y)
+    bq.bq_butterfly_inv(layer, y, back)
+    torch.cuda.synchronize()
+    idx = _sample(8192, 64, 43)
+    xf = H.input_f64(w.x, "bf16")[idx]
+    H.assert_f32_close(H.host(back)[idx], xf, xf)
