@@ -22,6 +22,14 @@ What it computes, and where the method is stated:
   technical summary, section 2 "method").  The pages give no formula; the
   readings taken are listed in the module docstring and in the design notes.
 
+* ``calib``      - the uniformity regulariser of calibration (abstract:
+  "uniformity regularization on post-transformation activations"; explainer
+  article, section "training & results": KL divergence between the rotated
+  activations' distribution and the uniform distribution over the quantization
+  intervals): a soft histogram over each group's RTN levels, its KL divergence
+  to uniform, and the gradient with respect to the activations.  The estimator
+  and smoothing are readings listed in the module docstring.
+
 Parity status: every function here is pinned by an independent check in
 ``tests/test_oracle_pins.py`` (closed forms, the Hadamard special case against
 ``scipy.linalg.hadamard``, explicit dense stage matrices, ``numpy.kron``, finite

@@ -1,0 +1,74 @@
+"""Float64 oracle of the uniformity regulariser used to calibrate the angles.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+The angles are learned with a loss that includes a uniformity regularisation of
+the post-transformation activations (ButterflyQuant abstract): the KL divergence
+between the distribution of the rotated activations and the uniform
+distribution over the quantization intervals, which pushes the transform to
+spread activations evenly over the levels of the quantizer (explainer article,
+section "training & results").  The pages give no estimator, smoothing or
+weighting.  The readings taken here:
+
+1. the bins of a group are the qmax + 1 levels of the group's own RTN grid: the
+   scale s and zero point z come from the quantizer (``quant.group_params``,
+   float32 steps on the float32 activations), and u = y / s + z is the real-valued
+   position of y on that grid;
+2. u is clamped to [0, qmax] and spread over the two nearest levels with a
+   triangular kernel, w_c = max(0, 1 - |u - c|): the soft histogram of a group
+   is p_c = (1/g) sum_i w_c(u_i), which sums to one;
+3. p is smoothed, p~_c = (p_c + eps) / (1 + B eps) with B = qmax + 1, so that
+   empty levels have a finite logarithm;
+4. the loss is the mean over all groups of all rows of KL(p~ || uniform) =
+   sum_c p~_c log(B p~_c);
+5. the gradient treats s and z as constants (they come from the group's min
+   and max), and a value with u outside (0, qmax) has zero gradient.  For u in
+   (k, k+1) only w_k and w_{k+1} move, so
+       dL/dy = (log p~_{k+1} - log p~_k) / (s g G (1 + B eps))
+   with G the number of groups (the +1 of d(p log p) cancels).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+from . import quant as oq
+
+
+def soft_histogram(y32, bits: int, group: int):
+    """(p, u, s) per group: p (rows, G, B) soft histogram, u (rows, G, g) the clamped
+    grid positions in float64, s (rows, G) float32 scales."""
+    y32 = np.asarray(y32, dtype=np.float32)
+    rows, n = y32.shape
+    _, _, s, z = oq.group_params(y32, bits, group)
+    qmax = 2 ** bits - 1
+    B = qmax + 1
+    v = y32.reshape(rows, n // group, group).astype(np.float64)
+    u = v / s.astype(np.float64)[..., None] + z.astype(np.float64)[..., None]
+    uc = np.clip(u, 0.0, float(qmax))
+    p = np.zeros((rows, n // group, B))
+    for c in range(B):
+        p[..., c] = np.maximum(0.0, 1.0 - np.abs(uc - c)).sum(axis=-1) / group
+    return p, u, s
+
+
+def uniformity_loss(y32, bits: int, group: int, eps: float):
+    """(loss, kl per group (rows, G), dloss/dy (rows, n)) in float64."""
+    y32 = np.asarray(y32, dtype=np.float32)
+    rows, n = y32.shape
+    qmax = 2 ** bits - 1
+    B = qmax + 1
+    G = rows * (n // group)
+    p, u, s = soft_histogram(y32, bits, group)
+    pt = (p + eps) / (1.0 + B * eps)
+    logs = np.log(B * pt)
+    kl = (pt * logs).sum(axis=-1)
+    loss = kl.mean()
+    # gradient: only the two levels around u move, with slopes -1 and +1
+    inside = (u > 0.0) & (u < qmax)
+    k = np.clip(np.floor(u), 0, qmax - 1).astype(np.int64)
+    lk = np.take_along_axis(logs, k, axis=-1)
+    lk1 = np.take_along_axis(logs, k + 1, axis=-1)
+    d = (lk1 - lk) / (s.astype(np.float64)[..., None] * group * G * (1.0 + B * eps))
+    dy = np.where(inside, d, 0.0).reshape(rows, n)
+    return loss, kl, dy
