@@ -171,6 +171,32 @@ bq_status bq_weight_rotate_pack(const bq_layer* layer, const void* w, bq_dtype w
                                 uint8_t* codes, uint16_t* scale_f16,
                                 uint16_t* zero_f16, void* stream);
 
+/* Uniformity regulariser of calibration and its gradient.  The angles are learned
+ * with a loss that includes a uniformity regularisation of the rotated
+ * activations (abstract): the KL divergence between their distribution and the
+ * uniform distribution over the quantization intervals (explainer article,
+ * section "training & results").  Per group of `group` contiguous values of a
+ * row of y (float32, [rows][n], e.g. the output of bq_butterfly_fwd):
+ *   s, z  the group's RTN scale and zero point (the rules of
+ *         bq_transform_quantize), B = 2^bits levels;
+ *   u     = y / s + z clamped to [0, 2^bits - 1], spread over its two nearest
+ *         levels with the triangular kernel max(0, 1 - |u - c|);
+ *   p_c   = mean over the group of those weights; p~ = (p + eps) / (1 + B eps);
+ *   KL    = sum_c p~_c log(B p~_c).
+ * kl_group: [rows][n/group] float32 per-group KL (device, written).
+ * dy: [rows][n] float32 gradient of the mean KL over all groups with s and z held
+ *   constant (zero where u is outside the open interval (0, 2^bits - 1)), or NULL.
+ * loss: one float32, the mean KL over all groups (summed in a fixed order), or
+ *   NULL.  bits: 2 or 4; group: 64, 128 or 256 dividing n; 0 < eps < 1.
+ * y and dy must be 16-byte aligned.  Results are bitwise reproducible. */
+bq_status bq_uniformity_loss(const float* y, int64_t rows, int32_t n, int32_t bits, int32_t group, float eps,
+                             float* kl_group, float* dy, float* loss, void* stream);
+
+/* One gradient step on the angles: theta[i] -= lr * dtheta[i] for i < count
+ * (device float32 arrays; rebuild the layer's table with bq_precompute_cs
+ * afterwards). */
+bq_status bq_angle_sgd(float* theta, const float* dtheta, int64_t count, float lr, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* bq_status_string(bq_status status);
 

@@ -16,6 +16,8 @@ from ._lib import (  # noqa: F401
     bq_precompute_cs,
     bq_transform_quantize,
     bq_weight_rotate_pack,
+    bq_uniformity_loss,
+    bq_angle_sgd,
     load,
     quant_outputs,
     status_string,

@@ -28,6 +28,8 @@ EXPORTED = (
     "bq_butterfly_bwd_noalloc",
     "bq_transform_quantize",
     "bq_weight_rotate_pack",
+    "bq_uniformity_loss",
+    "bq_angle_sgd",
     "bq_status_string",
 )
 
@@ -68,6 +70,8 @@ def load(path: str | None = None):
         "bq_butterfly_bwd_noalloc": (i32, [lp, i32, vp, i32, vp, i32, vp, vp, vp, i64, vp]),
         "bq_transform_quantize": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
         "bq_weight_rotate_pack": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+        "bq_uniformity_loss": (i32, [vp, i64, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp]),
+        "bq_angle_sgd": (i32, [vp, vp, i64, ctypes.c_float, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -226,3 +230,21 @@ def bq_transform_quantize(layer: Layer, x, bits: int, group: int, codes, scale, 
 
 def bq_weight_rotate_pack(layer: Layer, w, bits: int, group: int, codes, scale, zero, stream=None):
     return _quant("bq_weight_rotate_pack", layer, w, bits, group, codes, scale, zero, stream)
+
+
+def bq_uniformity_loss(y, bits: int, group: int, eps: float, kl_group, dy=None, loss=None, stream=None):
+    """y: float32 (rows, n); kl_group: float32 (rows, n/group); dy: float32 like y or None;
+    loss: float32 tensor of one element or None."""
+    _dev(y, "y"); _dev(kl_group, "kl_group")
+    if dy is not None:
+        _dev(dy, "dy")
+    rows, n = y.shape
+    _check("bq_uniformity_loss", load().bq_uniformity_loss(_ptr(y), rows, n, bits, group, float(eps), _ptr(kl_group),
+                                                            _ptr(dy), _ptr(loss), _stream(stream)))
+    return kl_group, dy, loss
+
+
+def bq_angle_sgd(theta, dtheta, lr: float, stream=None):
+    _dev(theta, "theta"); _dev(dtheta, "dtheta")
+    _check("bq_angle_sgd", load().bq_angle_sgd(_ptr(theta), _ptr(dtheta), theta.numel(), float(lr), _stream(stream)))
+    return theta

@@ -140,3 +140,26 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
     finally:
         _lib._lib = saved
+
+
+@pytest.mark.parametrize("bits,group,eps", [(3, 128, 1e-4), (4, 96, 1e-4), (4, 32, 1e-4), (2, 128, 0.0),
+                                            (2, 128, 1.0), (2, 128, float("nan"))])
+def test_uniformity_rejects_bad_settings(lib, bits, group, eps):
+    st = lib.bq_uniformity_loss(FAKE, 4, 4096, bits, group, eps, FAKE, FAKE, FAKE, None)
+    assert st == _lib.BQ_ERR_INVALID_ARG
+
+
+def test_uniformity_rejects_bad_buffers(lib):
+    assert lib.bq_uniformity_loss(None, 4, 4096, 4, 128, 1e-4, FAKE, FAKE, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_uniformity_loss(FAKE, 4, 4096, 4, 128, 1e-4, None, FAKE, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_uniformity_loss(FAKE + 4, 4, 4096, 4, 128, 1e-4, FAKE, FAKE, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_uniformity_loss(FAKE, 4, 4000, 4, 128, 1e-4, FAKE, FAKE, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_uniformity_loss(FAKE, -1, 4096, 4, 128, 1e-4, FAKE, FAKE, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_uniformity_loss(FAKE, 0, 4096, 4, 128, 1e-4, FAKE, FAKE, FAKE, None) == _lib.BQ_OK  # nothing to do
+
+
+def test_angle_sgd_rejects_bad_arguments(lib):
+    assert lib.bq_angle_sgd(None, FAKE, 8, 0.1, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_angle_sgd(FAKE, FAKE, -1, 0.1, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_angle_sgd(FAKE, FAKE, 8, float("nan"), None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_angle_sgd(FAKE, FAKE, 0, 0.1, None) == _lib.BQ_OK

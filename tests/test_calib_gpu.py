@@ -1,0 +1,109 @@
+"""Parity of the uniformity regulariser (bq_uniformity_loss) with the float64 oracle,
+and a short calibration loop (forward, regulariser gradient, backward, angle step)
+that lowers the regulariser on synthetic activations with outlier channels."""
+
+import numpy as np
+import pytest
+
+from oracle import calib as oc
+from rotation_bit_quantization_b200 import workloads as wl
+from tests import helpers as H
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def bq():
+    torch = pytest.importorskip("torch")
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import rotation_bit_quantization_b200 as bq_mod
+    from rotation_bit_quantization_b200 import build
+    build.build()
+    bq_mod.load()
+    return bq_mod
+
+
+def _acts(seed, rows, n):
+    rng = np.random.default_rng(seed)
+    y = (rng.standard_t(3.0, (rows, n)) * 0.5).astype(np.float32)
+    y[:, rng.choice(n, 6, replace=False)] *= 40.0          # outlier channels
+    return y
+
+
+def _run(bq, y, bits, group, eps):
+    torch = H.torch()
+    rows, n = y.shape
+    yd = H.dev_f32(y)
+    kl = torch.empty((rows, n // group), dtype=torch.float32, device="cuda")
+    dy = torch.empty_like(yd)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    bq.bq_uniformity_loss(yd, bits, group, eps, kl, dy, loss)
+    torch.cuda.synchronize()
+    return H.host(kl), H.host(dy), float(H.host(loss)[0])
+
+
+@pytest.mark.parametrize("bits,group", [(2, 64), (2, 128), (4, 128), (4, 256), (4, 64), (2, 256)])
+def test_uniformity_matches_oracle(bq, bits, group):
+    eps = 1e-4
+    y = _acts(bits * 100 + group, 37, 4096)
+    kl, dy, loss = _run(bq, y, bits, group, eps)
+    ref_loss, ref_kl, ref_dy = oc.uniformity_loss(y, bits, group, eps)
+    assert np.abs(kl - ref_kl).max() <= 2e-5 * (1 + np.abs(ref_kl).max())
+    assert abs(loss - ref_loss) <= 2e-5 * abs(ref_loss) + 1e-7
+    # the gradient jumps where u crosses a level: compare where u is clearly between
+    # two levels or clearly outside [0, qmax]
+    _, u, _ = oc.soft_histogram(y, bits, group)
+    u = u.reshape(y.shape)
+    qmax = 2 ** bits - 1
+    frac = u - np.floor(u)
+    clear = ((frac > 1e-3) & (frac < 1 - 1e-3) & (u > 1e-3) & (u < qmax - 1e-3)) | (u < -1e-3) | (u > qmax + 1e-3)
+    assert clear.mean() > 0.99
+    scale = np.abs(ref_dy).max()
+    err = np.abs(dy - ref_dy)[clear]
+    assert np.all(err <= 1e-4 * scale + 1e-4 * np.abs(ref_dy)[clear]), err.max() / scale
+    assert np.all(dy[(u < -1e-3) | (u > qmax + 1e-3)] == 0.0)
+    kl2, dy2, loss2 = _run(bq, y, bits, group, eps)
+    assert np.array_equal(kl, kl2) and np.array_equal(dy, dy2) and loss == loss2
+
+
+def test_uniformity_small_rows_and_degenerate_groups(bq):
+    y = _acts(7, 3, 1024)
+    y[1, :128] = 2.5                      # a constant group: hi == lo
+    y[2, 128:256] = 0.0
+    kl, dy, loss = _run(bq, y, 4, 128, 1e-3)
+    ref_loss, ref_kl, ref_dy = oc.uniformity_loss(y, 4, 128, 1e-3)
+    assert np.abs(kl - ref_kl).max() <= 2e-5 * (1 + np.abs(ref_kl).max())
+    assert abs(loss - ref_loss) <= 2e-5 * abs(ref_loss)
+
+
+def test_calibration_steps_lower_the_regulariser(bq):
+    """Forward -> regulariser gradient -> backward (dtheta) -> angle step, repeated:
+    the butterfly learns a rotation that spreads the outlier channels over the
+    quantizer's levels, so the regulariser must fall."""
+    torch = H.torch()
+    m, rows, bits, group, eps = 1024, 64, 4, 128, 1e-4
+    rng = np.random.default_rng(3)
+    theta = torch.from_numpy(wl.uniform_angles(rng, m)).cuda()
+    x = _acts(4, rows, m)
+    xd = H.dev_f32(x)[None]
+    y = torch.empty((rows, m), dtype=torch.float32, device="cuda")
+    kl = torch.empty((rows, m // group), dtype=torch.float32, device="cuda")
+    dy = torch.empty_like(y)
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    ybwd = torch.empty((1, rows, m), dtype=torch.float32, device="cuda")
+    dx = torch.empty((1, rows, m), dtype=torch.float32, device="cuda")
+    dth = torch.empty((1, theta.numel()), dtype=torch.float32, device="cuda")
+    ws = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, 1, rows), dtype=torch.uint8, device="cuda")
+    losses = []
+    for step in range(12):
+        layer = bq.Layer(theta)
+        bq.bq_butterfly_fwd(layer, xd[0], y)
+        bq.bq_uniformity_loss(y, bits, group, eps, kl, dy, loss)
+        bq.bq_butterfly_bwd([layer], xd, ybwd, dy[None], dx, dth, ws)
+        torch.cuda.synchronize()
+        losses.append(float(loss.item()))
+        lr = 0.02 / float(dth.abs().max().item())      # at most 0.02 rad per angle and step
+        bq.bq_angle_sgd(theta, dth.view(theta.shape), lr)
+    assert losses[-1] < 0.9 * losses[0], losses
+    assert all(np.isfinite(losses))
