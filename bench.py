@@ -53,6 +53,10 @@ def workload_spec(name: str):
     if name == "bwd":
         return dict(make=None, kind="bwd", rows=65536, n=4096, bits=0, group=0, layers=32,
                     label="calibration backward: 32 layers x 65536 tokens x n=4096, X bf16, dY fp32 -> Y bf16, dX fp32, dtheta (one launch)")
+    if name == "uniformity":
+        return dict(make=None, kind="uniformity", rows=65536, n=4096, bits=4, group=128, layers=1,
+                    label="uniformity regulariser: 65536 tokens x n=4096 float32 rotated activations -> "
+                          "per-group KL to uniform over the INT4 g128 levels + dL/dY (one calibration batch of one layer)")
     if name == "act5120":
         return dict(make=lambda rank: wl.act_5120(8192), kind="quant", rows=8192, n=5120, bits=4, group=128,
                     label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> INT4 RTN g128 (LLaMA-2-13B shape)")
@@ -421,6 +425,73 @@ def run_bwd_bench(args, spec, rank, world, local_rank):
     }
 
 
+def run_uniformity_bench(args, spec, rank, world, local_rank):
+    """The calibration regulariser: one bq_uniformity_loss over a batch of rotated activations."""
+    import torch
+    import torch.distributed as dist
+
+    import rotation_bit_quantization_b200 as bq
+    from rotation_bit_quantization_b200 import build as bq_build
+
+    bq_build.build()
+    bq.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    rows, n, bits, group = spec["rows"], spec["n"], spec["bits"], spec["group"]
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(11 + rank)
+    y = torch.randn((rows, n), generator=gen, device=dev) * 0.5
+    y[:, torch.randperm(n, generator=gen, device=dev)[:6]] *= 40.0     # outlier channels
+    kl = torch.empty((rows, n // group), dtype=torch.float32, device=dev)
+    dy = torch.empty_like(y)
+    loss = torch.empty(1, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bq.bq_uniformity_loss(y, bits, group, 1e-4, kl, dy, loss)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id_for(dev))
+    t_busy = time.perf_counter()
+    while time.perf_counter() - t_busy < 0.5:
+        for _ in range(10):
+            step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s_, e_ in evs:
+        s_.record(stream)
+        step()
+        e_.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    total_ms = float(sum(s_.elapsed_time(e_) for s_, e_ in evs))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / args.steps
+    by_row = 4 * n + 4 * n + 4 * (n // group)
+    peaks, peak_src = load_peaks()
+    achieved = rows * by_row / (ms * 1e-3) / 1e9
+    return {
+        "metric": "uniformity regulariser rows/s (per-group KL + dL/dY), n=4096 INT4 g128", "value": rows * world / (ms * 1e-3),
+        "unit": "rows/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded on device)", "config": {"workload": spec["label"], "rows": rows,
+                                                           "l2": "input 1 GiB, larger than L2"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "algorithmic_bytes_per_row": by_row},
+        "gpu_launches": 2 * args.steps, "clocks": clocks,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, spec):
@@ -464,7 +535,8 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="act4096", choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd"])
+    ap.add_argument("--workload", default="act4096",
+                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity"])
     ap.add_argument("--rows", type=int, default=0, help="override the workload's rows (tokens per layer for bwd)")
     ap.add_argument("--layers", type=int, default=0, help="override the backward workload's layer count")
     ap.add_argument("--no-e2e", action="store_true")
@@ -481,7 +553,7 @@ def main():
         # that has to fit the profiling size rules; never the bench line's size
         from rotation_bit_quantization_b200 import workloads as wl
         rows = args.rows or spec["rows"]
-        if spec["kind"] == "bwd":
+        if spec["kind"] in ("bwd", "uniformity"):
             spec = dict(spec, rows=rows, layers=args.layers or spec["layers"])
         else:
             base = {"act4096": lambda r, k: wl.act_4096(r, seed_offset=k), "fwd4096": lambda r, k: wl.act_4096(r, seed_offset=k),
@@ -491,7 +563,7 @@ def main():
             f", layers={spec['layers']}]" if spec["kind"] == "bwd" else "]")
 
     if args.impl == "reference":
-        if spec["kind"] == "bwd":
+        if spec["kind"] in ("bwd", "uniformity"):
             raise SystemExit("--impl reference covers the transform + quantize workloads only")
         if rank != 0:
             return 0
@@ -509,6 +581,8 @@ def main():
     try:
         if spec["kind"] == "bwd":
             res = run_bwd_bench(args, spec, rank, world, local_rank)
+        elif spec["kind"] == "uniformity":
+            res = run_uniformity_bench(args, spec, rank, world, local_rank)
         else:
             res = run_ours(args, spec, rank, world, local_rank)
     finally:

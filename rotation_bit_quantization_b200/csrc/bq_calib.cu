@@ -15,10 +15,11 @@
 // Gradient (s, z held constant; zero outside 0 < u < qmax): for u in (k, k+1)
 //   dloss/dy = (log p~_{k+1} - log p~_k) / (s g G (1 + B eps)),  G = number of groups.
 //
-// One warp per group.  Each lane accumulates its values' weights into its own
-// column of a per-warp [B][32] histogram in shared memory (no atomics: the sum
-// order is fixed, so results are reproducible), the columns are added in a fixed
-// order, and each level's logarithm is taken once and fetched by shuffle.
+// Each lane accumulates its values' weights into its own column of a per-warp
+// [B][32] histogram in shared memory (each address has one writer, so the order
+// of the additions is fixed and results are reproducible), a group's columns are
+// added in a fixed order, and each level's logarithm is taken once and read back
+// by each lane from its own column for the gradient.
 #include <cfloat>
 
 #include "bq_rtn.cuh"
@@ -28,37 +29,40 @@ namespace {
 
 constexpr int kCalWarps = 8;
 
+// Each warp handles NG = 32 / GL groups at once with GL = GROUP / 32 lanes per
+// group and 32 values per lane (float4 chunks GL j + q of the group for lane q),
+// so the per-group work (scale and zero point, the histogram's column sums, the
+// logarithms) is spread over the warp instead of repeated by all of its lanes.
 template <int BITS, int GROUP>
 __global__ void __launch_bounds__(32 * kCalWarps) k_uniformity(const float* __restrict__ y, long long groups,
                                                                float eps, float gscale, float* __restrict__ kl_group,
                                                                float* __restrict__ dy) {
-  constexpr int B = 1 << BITS, QMAX = B - 1, E = GROUP / 32;
+  constexpr int B = 1 << BITS, QMAX = B - 1, GL = GROUP / 32, NG = 32 / GL;
+  constexpr int BPL = B >= GL ? B / GL : 1;  // levels each lane of a group sums
   __shared__ float hist[kCalWarps][B][32];
   const int lane = threadIdx.x & 31, wl = threadIdx.x >> 5;
+  const int gi = lane / GL, q = lane % GL;
   const float qmax = static_cast<float>(QMAX);
-  const long long stride = static_cast<long long>(gridDim.x) * kCalWarps;
+  const long long stride = static_cast<long long>(gridDim.x) * kCalWarps * NG;
 #pragma unroll 1
-  for (long long g = static_cast<long long>(blockIdx.x) * kCalWarps + wl; g < groups; g += stride) {
-    const float* src = y + g * GROUP + lane * E;
-    float v[E];
+  for (long long g0 = (static_cast<long long>(blockIdx.x) * kCalWarps + wl) * NG; g0 < groups; g0 += stride) {
+    const long long g = g0 + gi;
+    const bool live = g < groups;  // the last warp may hold fewer than NG groups
+    const float* src = y + (live ? g : g0) * GROUP;
+    float v[32];
 #pragma unroll
-    for (int q = 0; q < E; q += (E >= 4 ? 4 : E)) {
-      if constexpr (E >= 4) {
-        const float4 t = *reinterpret_cast<const float4*>(src + q);
-        v[q] = t.x; v[q + 1] = t.y; v[q + 2] = t.z; v[q + 3] = t.w;
-      } else {
-        const float2 t = *reinterpret_cast<const float2*>(src + q);
-        v[q] = t.x; v[q + 1] = t.y;
-      }
+    for (int j = 0; j < 8; ++j) {
+      const float4 t = *reinterpret_cast<const float4*>(src + 4 * (GL * j + q));
+      v[4 * j] = t.x; v[4 * j + 1] = t.y; v[4 * j + 2] = t.z; v[4 * j + 3] = t.w;
     }
     float lo = v[0], hi = v[0];
 #pragma unroll
-    for (int q = 1; q < E; ++q) {
-      lo = fminf(lo, v[q]);
-      hi = fmaxf(hi, v[q]);
+    for (int e = 1; e < 32; ++e) {
+      lo = fminf(lo, v[e]);
+      hi = fmaxf(hi, v[e]);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
+    for (int o = GL / 2; o > 0; o >>= 1) {
       lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
       hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
     }
@@ -66,46 +70,62 @@ __global__ void __launch_bounds__(32 * kCalWarps) k_uniformity(const float* __re
     const float z = __fadd_rn(p.mz, -12582912.f);
 #pragma unroll
     for (int c = 0; c < B; ++c) hist[wl][c][lane] = 0.f;
-    float u[E];
-    int k[E];
+    __syncwarp();
+    // soft histogram: each lane adds into its own column (the only writer of those
+    // addresses, so a plain read-modify-write in program order)
 #pragma unroll
-    for (int q = 0; q < E; ++q) {
-      u[q] = fmaf(v[q], p.inv, z);
-      const float uc = fminf(fmaxf(u[q], 0.f), qmax);
-      k[q] = min(static_cast<int>(uc), QMAX - 1);  // uc >= 0: truncation is floor
-      const float f = uc - static_cast<float>(k[q]);
-      hist[wl][k[q]][lane] += 1.f - f;
-      hist[wl][k[q] + 1][lane] += f;
+    for (int e = 0; e < 32; ++e) {
+      const float uc = fminf(fmaxf(fmaf(v[e], p.inv, z), 0.f), qmax);
+      const int k = min(static_cast<int>(uc), QMAX - 1);  // uc >= 0: truncation is floor
+      const float f = uc - static_cast<float>(k);
+      hist[wl][k][lane] += 1.f - f;
+      hist[wl][k + 1][lane] += f;
     }
     __syncwarp();
-    // level c = lane % B: add the columns in a fixed order per level, level c starting
-    // at column c so that the lanes of one step hit distinct banks
-    const int c = lane % B;
-    float cnt = 0.f;
-#pragma unroll 8
-    for (int l = 0; l < 32; ++l) cnt += hist[wl][c][(l + c) & 31];
-    const float pt = (cnt * (1.f / static_cast<float>(GROUP)) + eps) / (1.f + static_cast<float>(B) * eps);
-    const float lg = logf(static_cast<float>(B) * pt);
-    float term = lane < B ? pt * lg : 0.f;
+    // levels q BPL .. q BPL + BPL - 1 of this lane's group: its GL columns, in a fixed
+    // order per level that starts at column q (the group's lanes hit distinct banks)
+    float term = 0.f, lgv[BPL];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
-    if (lane == 0) kl_group[g] = term;
-    if (dy) {
-      const float sc = gscale / p.s;
-      float d[E];
+    for (int b = 0; b < BPL; ++b) {
+      const int c = q * BPL + b;
+      lgv[b] = 0.f;
+      if (c < B) {
+        float cnt = 0.f;
 #pragma unroll
-      for (int q = 0; q < E; ++q) {
-        const float l0 = __shfl_sync(0xffffffffu, lg, k[q]), l1 = __shfl_sync(0xffffffffu, lg, k[q] + 1);
-        d[q] = (u[q] > 0.f && u[q] < qmax) ? (l1 - l0) * sc : 0.f;
-      }
-      float* dst = dy + g * GROUP + lane * E;
-#pragma unroll
-      for (int q = 0; q < E; q += (E >= 4 ? 4 : E)) {
-        if constexpr (E >= 4) *reinterpret_cast<float4*>(dst + q) = make_float4(d[q], d[q + 1], d[q + 2], d[q + 3]);
-        else *reinterpret_cast<float2*>(dst + q) = make_float2(d[q], d[q + 1]);
+        for (int l = 0; l < GL; ++l) cnt += hist[wl][c][gi * GL + ((l + q) & (GL - 1))];
+        const float pt = (cnt * (1.f / static_cast<float>(GROUP)) + eps) / (1.f + static_cast<float>(B) * eps);
+        lgv[b] = logf(static_cast<float>(B) * pt);
+        term = fmaf(pt, lgv[b], term);
       }
     }
-    __syncwarp();  // the histogram columns are reused by the next group
+#pragma unroll
+    for (int o = GL / 2; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
+    if (live && q == 0) kl_group[g] = term;
+    // every lane gets its group's B logarithms into its own column of the histogram
+    float lgc[B];
+#pragma unroll
+    for (int c = 0; c < B; ++c) lgc[c] = __shfl_sync(0xffffffffu, lgv[c % BPL], gi * GL + c / BPL);
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < B; ++c) hist[wl][c][lane] = lgc[c];
+    __syncwarp();
+    if (dy) {
+      const float sc = gscale / p.s;
+      float* dst = dy + (live ? g : g0) * GROUP;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float d[4];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const float u = fmaf(v[4 * j + t], p.inv, z);
+          const float uc = fminf(fmaxf(u, 0.f), qmax);
+          const int k = min(static_cast<int>(uc), QMAX - 1);
+          d[t] = (u > 0.f && u < qmax) ? (hist[wl][k + 1][lane] - hist[wl][k][lane]) * sc : 0.f;
+        }
+        if (live) *reinterpret_cast<float4*>(dst + 4 * (GL * j + q)) = make_float4(d[0], d[1], d[2], d[3]);
+      }
+    }
+    __syncwarp();  // the columns are reused by the next groups
   }
 }
 
@@ -134,7 +154,8 @@ bq_status run_uniformity(const float* y, long long groups, float eps, float gsca
                          cudaStream_t st) {
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  long long grid = (groups + kCalWarps - 1) / kCalWarps;
+  constexpr int kGroupsPerBlock = kCalWarps * (32 / (GROUP / 32));
+  long long grid = (groups + kGroupsPerBlock - 1) / kGroupsPerBlock;
   const long long cap = static_cast<long long>(sms) * 8;
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
