@@ -1,4 +1,5 @@
-"""Float64 oracle of the uniformity regulariser used to calibrate the angles.
+"""Float64 oracle of the calibration losses: the uniformity regulariser and the
+reconstruction loss with a straight-through estimator.
 
 TEST INFRASTRUCTURE ONLY (see the package docstring).
 
@@ -72,3 +73,33 @@ def uniformity_loss(y32, bits: int, group: int, eps: float):
     d = (lk1 - lk) / (s.astype(np.float64)[..., None] * group * G * (1.0 + B * eps))
     dy = np.where(inside, d, 0.0).reshape(rows, n)
     return loss, kl, dy
+
+
+def reconstruction_loss(theta, w, x, bits: int, group: int):
+    """Reconstruction loss of one linear layer under weight quantization, and its
+    gradient with a straight-through estimator (readings of the explainer article,
+    section "training & results": the quantized layer's output should match the
+    original one; the abstract's invariance y = W x = (W Q^T)(Q x)).
+
+    V = W Q^T (row o of V is Q w_o), W_hat = dequantize(RTN(V)) with the quantizer
+    of ``quant`` applied to V rounded to float32, x~ = Q x per token, and
+        r[t, o] = (W_hat x~_t)_o - (W x_t)_o,   loss = (1/T) sum_t ||r_t||^2.
+    The straight-through estimator takes dW_hat / dV as the identity, so
+        G_x = dloss/dx~ = (2/T) r W_hat,   G_v = dloss/dV = (2/T) r^T x~,
+    and dtheta adds the backward of the activation side (rows x, gradient G_x)
+    and of the weight side (rows w, gradient G_v).  Returns (loss, dtheta)."""
+    from . import butterfly as ob
+    w = np.asarray(w, dtype=np.float64)
+    x = np.asarray(x, dtype=np.float64)
+    T = x.shape[0]
+    v = ob.forward(theta, w)
+    codes, scale16, zero16 = oq.quantize_codes(v.astype(np.float32), bits, group)
+    w_hat = oq.dequantize(codes, scale16, zero16, group).astype(np.float64)
+    xt = ob.forward(theta, x)
+    r = xt @ w_hat.T - x @ w.T
+    loss = float((r * r).sum() / T)
+    g_x = (2.0 / T) * (r @ w_hat)
+    g_v = (2.0 / T) * (r.T @ xt)
+    _, _, dth_x = ob.backward(theta, x, g_x)
+    _, _, dth_v = ob.backward(theta, w, g_v)
+    return loss, dth_x + dth_v

@@ -94,3 +94,91 @@ def test_gradient_points_toward_emptier_levels():
     y = np.array([[0.0] * 60 + [0.3, 3.0, 3.0, 3.0]], np.float32)            # s = 1, z = 0
     loss, kl, dy = oc.uniformity_loss(y, 2, 64, 1e-4)
     assert dy[0, 60] < 0
+
+
+# --------------------------------------------------------------------------- reconstruction loss
+
+from oracle import butterfly as ob                    # noqa: E402
+from rotation_bit_quantization_b200 import workloads as wl  # noqa: E402
+
+
+def _recon_case(seed, m=16, out=12, T=9):
+    rng = np.random.default_rng(seed)
+    theta = wl.uniform_angles(rng, m)
+    w = rng.standard_normal((out, m)).astype(np.float32)
+    x = rng.standard_normal((T, m)).astype(np.float32)
+    return theta, w, x
+
+
+def _q64(th64, m):
+    """Dense Q from float64 angles (stage matrices), for finite differences in theta."""
+    q = np.eye(m)
+    for s in range(ob.num_stages(m)):
+        B = np.zeros((m, m))
+        half = 1 << s
+        for i in range(m):
+            if (i >> s) & 1:
+                continue
+            j = i + half
+            p = ((i >> (s + 1)) << s) | (i & (half - 1))
+            c, sn = np.cos(th64[s, p]), np.sin(th64[s, p])
+            B[i, i], B[i, j], B[j, i], B[j, j] = c, -sn, sn, c
+        q = B @ q
+    return q
+
+
+def _surrogate(th64, theta0, w, x, bits, group):
+    """The straight-through surrogate around theta0: W_hat(theta) = RTN(V0) + V(theta) - V0."""
+    m = w.shape[1]
+    w64, x64 = w.astype(np.float64), x.astype(np.float64)
+    v0 = ob.forward(theta0, w64)
+    codes, s16, z16 = oq.quantize_codes(v0.astype(np.float32), bits, group)
+    q = _q64(th64, m)
+    w_hat = oq.dequantize(codes, s16, z16, group).astype(np.float64) + w64 @ q.T - v0
+    r = (x64 @ q.T) @ w_hat.T - x64 @ w64.T
+    return (r * r).sum() / x.shape[0]
+
+
+def test_reconstruction_gradient_matches_surrogate_finite_differences():
+    theta, w, x = _recon_case(1)
+    loss, dth = oc.reconstruction_loss(theta, w, x, 2, 8)
+    th0 = theta.astype(np.float64)
+    assert abs(_surrogate(th0, theta, w, x, 2, 8) - loss) < 1e-10 * max(1.0, loss)
+    h = 1e-6
+    for s, p in ((0, 0), (1, 3), (2, 5), (3, 7)):
+        tp, tm = th0.copy(), th0.copy()
+        tp[s, p] += h
+        tm[s, p] -= h
+        fd = (_surrogate(tp, theta, w, x, 2, 8) - _surrogate(tm, theta, w, x, 2, 8)) / (2 * h)
+        assert abs(fd - dth[s, p]) <= 1e-6 * max(1.0, abs(fd)), (s, p, fd, dth[s, p])
+
+
+def test_reconstruction_planted_missing_weight_side_is_caught():
+    theta, w, x = _recon_case(2)
+    th0 = theta.astype(np.float64)
+    v = ob.forward(theta, w.astype(np.float64))
+    codes, s16, z16 = oq.quantize_codes(v.astype(np.float32), 2, 8)
+    w_hat = oq.dequantize(codes, s16, z16, 8).astype(np.float64)
+    xt = ob.forward(theta, x.astype(np.float64))
+    r = xt @ w_hat.T - x.astype(np.float64) @ w.astype(np.float64).T
+    _, _, wrong = ob.backward(theta, x, (2.0 / x.shape[0]) * (r @ w_hat))      # weight side dropped
+    h = 1e-6
+    tp, tm = th0.copy(), th0.copy()
+    tp[1, 2] += h
+    tm[1, 2] -= h
+    fd = (_surrogate(tp, theta, w, x, 2, 8) - _surrogate(tm, theta, w, x, 2, 8)) / (2 * h)
+    assert abs(fd - wrong[1, 2]) > 1e-4 * max(1.0, abs(fd))
+
+
+def test_reconstruction_is_zero_for_an_exactly_quantizable_layer():
+    # theta = 0 (Q = I) and weights on their groups' RTN grids: W_hat = W, r = 0
+    m, out, group = 16, 6, 8
+    rng = np.random.default_rng(4)
+    q = rng.integers(0, 4, (out, m))
+    q[:, ::group] = 0
+    q[:, 1::group] = 3                                  # each group spans the full grid
+    w = ((q - 1) * 0.25).astype(np.float32)            # s = 0.25, z = 1 exactly
+    x = rng.standard_normal((5, m)).astype(np.float32)
+    theta = np.zeros((4, m // 2), np.float32)
+    loss, dth = oc.reconstruction_loss(theta, w, x, 2, group)
+    assert loss == 0.0 and np.all(dth == 0.0)
