@@ -197,6 +197,28 @@ bq_status bq_uniformity_loss(const float* y, int64_t rows, int32_t n, int32_t bi
  * afterwards). */
 bq_status bq_angle_sgd(float* theta, const float* dtheta, int64_t count, float lr, void* stream);
 
+/* Bytes of workspace bq_reconstruction_loss needs (0 for unsupported sizes). */
+size_t bq_reconstruction_workspace_size(int32_t n, int64_t out_features, int64_t tokens, int32_t bits,
+                                        int32_t group);
+
+/* Reconstruction loss of one linear layer under weight quantization, with a
+ * straight-through estimator, and its gradient in the angles: the quantized
+ * layer's output should match the original one (explainer article, section
+ * "training & results"), through the invariance y = W x = (W Q^T)(Q x)
+ * (abstract).  With V = W Q^T, W_hat = the dequantized bq_weight_rotate_pack
+ * codes of W ((q - z) s), x~_t = Q x_t and r[t][o] = (W_hat x~_t)_o - (W x_t)_o:
+ *   loss = (1/T) sum_t ||r_t||^2;
+ *   dtheta = backward(x, (2/T) r W_hat) + backward(W, (2/T) r^T x~), taking
+ *            dW_hat / dV as the identity (straight-through).
+ * layer: r == 1 (n = m, a power of two).  w: [out_features][n] float32; x:
+ * [tokens][n] float32 (device, 16-byte aligned).  dtheta: log2(n) * n/2 floats
+ * (written); loss: one float (written).  workspace: device, 256-byte aligned,
+ * >= bq_reconstruction_workspace_size(...).  bits / group: as for
+ * bq_weight_rotate_pack.  Deterministic (fixed summation orders). */
+bq_status bq_reconstruction_loss(const bq_layer* layer, const float* w, int64_t out_features, const float* x,
+                                 int64_t tokens, int32_t bits, int32_t group, float* dtheta, float* loss,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* bq_status_string(bq_status status);
 

@@ -18,6 +18,8 @@ from ._lib import (  # noqa: F401
     bq_weight_rotate_pack,
     bq_uniformity_loss,
     bq_angle_sgd,
+    bq_reconstruction_loss,
+    bq_reconstruction_workspace_size,
     load,
     quant_outputs,
     status_string,

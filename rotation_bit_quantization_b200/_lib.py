@@ -30,6 +30,8 @@ EXPORTED = (
     "bq_weight_rotate_pack",
     "bq_uniformity_loss",
     "bq_angle_sgd",
+    "bq_reconstruction_workspace_size",
+    "bq_reconstruction_loss",
     "bq_status_string",
 )
 
@@ -72,6 +74,8 @@ def load(path: str | None = None):
         "bq_weight_rotate_pack": (i32, [lp, vp, i32, i64, i32, i32, vp, vp, vp, vp]),
         "bq_uniformity_loss": (i32, [vp, i64, i32, i32, i32, ctypes.c_float, vp, vp, vp, vp]),
         "bq_angle_sgd": (i32, [vp, vp, i64, ctypes.c_float, vp]),
+        "bq_reconstruction_workspace_size": (sz, [i32, i64, i64, i32, i32]),
+        "bq_reconstruction_loss": (i32, [lp, vp, i64, vp, i64, i32, i32, vp, vp, vp, sz, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -248,3 +252,19 @@ def bq_angle_sgd(theta, dtheta, lr: float, stream=None):
     _dev(theta, "theta"); _dev(dtheta, "dtheta")
     _check("bq_angle_sgd", load().bq_angle_sgd(_ptr(theta), _ptr(dtheta), theta.numel(), float(lr), _stream(stream)))
     return theta
+
+
+def bq_reconstruction_workspace_size(n: int, out_features: int, tokens: int, bits: int, group: int) -> int:
+    return int(load().bq_reconstruction_workspace_size(n, out_features, tokens, bits, group))
+
+
+def bq_reconstruction_loss(layer: Layer, w, x, bits: int, group: int, dtheta, loss, workspace, stream=None):
+    """w: float32 (out_features, n); x: float32 (tokens, n); dtheta: float32 with log2(n)*n/2
+    elements; loss: float32 tensor of one element; workspace: uint8 CUDA tensor."""
+    for t, nm in ((w, "w"), (x, "x"), (dtheta, "dtheta"), (loss, "loss"), (workspace, "workspace")):
+        _dev(t, nm)
+    _check("bq_reconstruction_loss",
+           load().bq_reconstruction_loss(ctypes.byref(layer.c), _ptr(w), w.shape[0], _ptr(x), x.shape[0], bits, group,
+                                         _ptr(dtheta), _ptr(loss), _ptr(workspace),
+                                         workspace.numel() * workspace.element_size(), _stream(stream)))
+    return dtheta, loss

@@ -163,3 +163,17 @@ def test_angle_sgd_rejects_bad_arguments(lib):
     assert lib.bq_angle_sgd(FAKE, FAKE, -1, 0.1, None) == _lib.BQ_ERR_INVALID_ARG
     assert lib.bq_angle_sgd(FAKE, FAKE, 8, float("nan"), None) == _lib.BQ_ERR_INVALID_ARG
     assert lib.bq_angle_sgd(FAKE, FAKE, 0, 0.1, None) == _lib.BQ_OK
+
+
+def test_reconstruction_rejects_bad_arguments(lib):
+    assert lib.bq_reconstruction_workspace_size(256, 16, 8, 2, 64) > 0
+    assert lib.bq_reconstruction_workspace_size(250, 16, 8, 2, 64) == 0      # not a power of two
+    assert lib.bq_reconstruction_workspace_size(256, 0, 8, 2, 64) == 0
+    assert lib.bq_reconstruction_workspace_size(256, 16, 8, 3, 64) == 0
+    assert lib.bq_reconstruction_workspace_size(256, 16, 8, 2, 48) == 0
+    good = _lib.BQLayer(256, 256, 1, FAKE, None)
+    kron = _lib.BQLayer(256 * 3, 256, 3, FAKE, FAKE)
+    args = (FAKE, 16, FAKE, 8, 2, 64, FAKE, FAKE, FAKE)
+    assert lib.bq_reconstruction_loss(ctypes.byref(good), *args, 16, None) == _lib.BQ_ERR_WORKSPACE
+    assert lib.bq_reconstruction_loss(ctypes.byref(kron), *args, 1 << 30, None) == _lib.BQ_ERR_UNSUPPORTED
+    assert lib.bq_reconstruction_loss(None, *args, 1 << 30, None) == _lib.BQ_ERR_INVALID_ARG

@@ -107,3 +107,68 @@ def test_calibration_steps_lower_the_regulariser(bq):
         bq.bq_angle_sgd(theta, dth.view(theta.shape), lr)
     assert losses[-1] < 0.9 * losses[0], losses
     assert all(np.isfinite(losses))
+
+
+# --------------------------------------------------------------------------- reconstruction loss
+
+def _recon_gpu(bq, theta, w, x, bits, group):
+    torch = H.torch()
+    n = w.shape[1]
+    layer = bq.Layer(H.dev_f32(theta))
+    ws = torch.empty(bq.bq_reconstruction_workspace_size(n, w.shape[0], x.shape[0], bits, group),
+                     dtype=torch.uint8, device="cuda")
+    dth = torch.empty(theta.size, dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    bq.bq_reconstruction_loss(layer, H.dev_f32(w), H.dev_f32(x), bits, group, dth, loss, ws)
+    torch.cuda.synchronize()
+    return float(H.host(loss)[0]), H.host(dth).reshape(theta.shape), layer
+
+
+@pytest.mark.parametrize("m,out,T,bits,group", [(256, 48, 40, 2, 64), (1024, 40, 33, 4, 128), (4096, 96, 64, 2, 128)])
+def test_reconstruction_matches_oracle(bq, m, out, T, bits, group):
+    torch = H.torch()
+    rng = np.random.default_rng(m + out + T)
+    theta = wl.uniform_angles(rng, m)
+    w = (rng.standard_normal((out, m)) * 0.02).astype(np.float32)
+    w[:, rng.choice(m, max(1, m // 100), replace=False)] *= 10.0
+    x = _acts(m + 1, T, m)
+    loss, dth, layer = _recon_gpu(bq, theta, w, x, bits, group)
+    # the codes the GPU quantized (bitwise the quantizer on its float32 forward) equal the
+    # oracle's own codes here, so the two losses see the same W_hat
+    from oracle import butterfly as ob
+    from oracle import quant as oq
+    codes, _, _ = bq.quant_outputs(out, m, bits, group, "cuda")
+    c_gpu = torch.empty_like(codes); sc = torch.empty((out, m // group), dtype=torch.int16, device="cuda")
+    zc = torch.empty_like(sc)
+    bq.bq_weight_rotate_pack(layer, H.dev_f32(w), bits, group, c_gpu, sc, zc)
+    torch.cuda.synchronize()
+    c_ref, _, _ = oq.quantize_pack(ob.forward(theta, w.astype(np.float64)).astype(np.float32), bits, group)
+    assert np.array_equal(H.host(c_gpu), c_ref)
+    ref_loss, ref_dth = oc.reconstruction_loss(theta, w, x, bits, group)
+    assert abs(loss - ref_loss) <= 2e-4 * ref_loss
+    assert np.abs(dth - ref_dth).max() <= 2e-3 * np.abs(ref_dth).max()
+    loss2, dth2, _ = _recon_gpu(bq, theta, w, x, bits, group)
+    assert loss2 == loss and np.array_equal(dth2, dth)
+
+
+def test_calibration_steps_lower_the_reconstruction_loss(bq):
+    """Angle steps on the straight-through gradient lower the W2A16 reconstruction
+    loss of a layer whose activations carry outlier channels."""
+    torch = H.torch()
+    m, out, T, bits, group = 256, 64, 96, 2, 64
+    rng = np.random.default_rng(8)
+    theta = torch.from_numpy(wl.uniform_angles(rng, m)).cuda()
+    w = H.dev_f32((rng.standard_normal((out, m)) * 0.02).astype(np.float32))
+    x = H.dev_f32(_acts(9, T, m))
+    ws = torch.empty(bq.bq_reconstruction_workspace_size(m, out, T, bits, group), dtype=torch.uint8, device="cuda")
+    dth = torch.empty(theta.numel(), dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    losses = []
+    for step in range(15):
+        layer = bq.Layer(theta)
+        bq.bq_reconstruction_loss(layer, w, x, bits, group, dth, loss, ws)
+        torch.cuda.synchronize()
+        losses.append(float(loss.item()))
+        lr = 0.02 / float(dth.abs().max().item())
+        bq.bq_angle_sgd(theta, dth.view(theta.shape), lr)
+    assert min(losses[-3:]) < 0.9 * losses[0], losses
