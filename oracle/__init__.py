@@ -14,21 +14,23 @@ What it computes, and where the method is stated:
   explainer article, section "butterfly"), its inverse Q^T, the Kronecker
   composite B_m (x) O_r for widths that are not a power of two (explainer
   article, section "butterfly", last paragraph), and the backward pass
-  (dX, dtheta) that gradient-based calibration needs (abstract: "enables smooth
-  optimization").
+  (dX, dtheta) that gradient-based calibration needs (abstract: the continuous angles
+  are learned by gradient descent).
 * ``quant``      - per-group asymmetric round-to-nearest quantization with fp16
   scale and zero point and little-endian INT2/INT4 packing (2-bit weights:
   explainer article, section "training & results"; RTN block quantizer: WUSH
   technical summary, section 2 "method").  The pages give no formula; the
   readings taken are listed in the module docstring and in the design notes.
 
-* ``calib``      - the uniformity regulariser of calibration (abstract:
-  "uniformity regularization on post-transformation activations"; explainer
-  article, section "training & results": KL divergence between the rotated
-  activations' distribution and the uniform distribution over the quantization
-  intervals): a soft histogram over each group's RTN levels, its KL divergence
-  to uniform, and the gradient with respect to the activations.  The estimator
-  and smoothing are readings listed in the module docstring.
+* ``calib``      - the calibration losses: the uniformity regulariser (the
+  abstract names a uniformity regularisation of the transformed activations;
+  explainer article, section "training & results": the KL divergence between the
+  rotated activations' distribution and the uniform distribution over the
+  quantization intervals) as a soft histogram over each group's RTN levels, its
+  KL divergence to uniform and the gradient with respect to the activations;
+  and the reconstruction loss of a quantized layer with a straight-through
+  estimator.  The estimators and smoothing are readings listed in the module
+  docstring.
 
 Parity status: every function here is pinned by an independent check in
 ``tests/test_oracle_pins.py`` (closed forms, the Hadamard special case against

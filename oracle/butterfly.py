@@ -47,7 +47,7 @@ def num_stages(m: int) -> int:
 
 
 def num_angles(m: int) -> int:
-    """Learnable parameter count n*log2(n)/2 (abstract: "only n log n / 2 learnable parameters")."""
+    """Learnable parameter count n*log2(n)/2 (abstract: half of n log n angles are learned)."""
     return m * num_stages(m) // 2
 
 

@@ -28,7 +28,7 @@ def rand_theta(m, seed):
 
 @pytest.mark.parametrize("m", [2, 4, 8, 16, 64, 256])
 def test_orthogonal_by_construction(m):
-    # abstract: "guaranteeing orthogonality by construction"
+    # abstract: the parameterisation is orthogonal by construction
     Q = bf.dense_q(rand_theta(m, m), m)
     assert np.abs(Q @ Q.T - np.eye(m)).max() < 1e-12
     assert np.abs(Q.T @ Q - np.eye(m)).max() < 1e-12
