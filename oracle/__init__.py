@@ -31,6 +31,10 @@ What it computes, and where the method is stated:
   and the reconstruction loss of a quantized layer with a straight-through
   estimator.  The estimators and smoothing are readings listed in the module
   docstring.
+* ``w2a16``      - the W2A16 consumer GEMM (explainer article, section "training
+  & results": 2-bit weights, 16-bit activations; abstract: y = (W Q^T)(Q x)):
+  bfloat16 activations times the bfloat16-rounded dequantized codes, summed
+  exactly in float64.
 
 Parity status: every function here is pinned by an independent check in
 ``tests/test_oracle_pins.py`` (closed forms, the Hadamard special case against
