@@ -219,6 +219,41 @@ bq_status bq_reconstruction_loss(const bq_layer* layer, const float* w, int64_t 
                                  int64_t tokens, int32_t bits, int32_t group, float* dtheta, float* loss,
                                  void* workspace, size_t workspace_bytes, void* stream);
 
+/* W2A16 consumer GEMM on the tensor cores (tcgen05): the quantized layer of the
+ * invariance y = W x = (W Q^T)(Q x) (abstract) with 2-bit weights and 16-bit
+ * activations (explainer article, section "training & results": W2A16):
+ *   out[t][o] = sum_k x[t][k] * bf16((q[o][k] - z[o][k / group]) * s[o][k / group])
+ * where (q - z) s is formed exactly in float32 and rounded to nearest-even
+ * bfloat16, products are exact and sums are float32.
+ * x: [tokens][n] bfloat16, the rotated activations (e.g. bq_butterfly_fwd with
+ *   yt = BQ_BF16); device, 16-byte aligned.
+ * codes, scale_f16, zero_f16: the packed weights of bq_weight_rotate_pack for
+ *   [out_features][n] (codes [out][n*bits/8] bytes, 16-byte aligned; scale and
+ *   zero [out][n/group] fp16 bit patterns).  bits: 2, or 4 for W4A16.
+ * group: 64, 128 or 256 dividing n; n: a multiple of 64.
+ * out: [tokens][out_features] float32 (out_t = BQ_F32) or bfloat16 (BQ_BF16,
+ *   rounded to nearest-even); device.
+ * status: NULL, or a device int32 the caller zeroes; the kernel ORs a nonzero
+ *   code into it if one of its internal waits gave up after one second (the
+ *   output is then incomplete).  Nothing is launched on invalid arguments;
+ *   BQ_ERR_UNSUPPORTED if the driver's tensor-map encoder is unavailable. */
+bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, const uint8_t* codes,
+                        const uint16_t* scale_f16, const uint16_t* zero_f16, int64_t out_features,
+                        int32_t bits, int32_t group, void* out, bq_dtype out_t, int32_t* status,
+                        void* stream);
+
+/* Bytes of workspace bq_w2a16_linear needs: the bfloat16 rotated activations. */
+size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens);
+
+/* The whole quantized layer from raw activations: x~ = Q x (bq_butterfly_fwd to
+ * bfloat16 into the workspace), then bq_w2a16_gemm(x~, ...).  x: [tokens][n] of
+ * dtype xt; workspace: device, 256-byte aligned, >= bq_w2a16_linear_workspace_size;
+ * other arguments as for bq_w2a16_gemm. */
+bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int64_t tokens,
+                          const uint8_t* codes, const uint16_t* scale_f16, const uint16_t* zero_f16,
+                          int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,
+                          void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* bq_status_string(bq_status status);
 

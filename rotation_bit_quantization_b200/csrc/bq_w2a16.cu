@@ -1,0 +1,589 @@
+// W2A16 consumer GEMM on the fifth-generation tensor cores.
+//
+// The transform leaves a layer's output unchanged because y = W x = (W Q^T)(Q x)
+// (ButterflyQuant abstract), and the pages deploy it with 2-bit weights and
+// 16-bit activations (explainer article, section "training & results": W2A16).
+// The quantized layer is therefore a GEMM of the rotated bfloat16 activations
+// x~ = Q x with the dequantized codes of W Q^T:
+//   out[t][o] = sum_k x~[t][k] * bf16((q[o][k] - z[o][g]) * s[o][g]),  g = k / group,
+// with codes, scales and zero points in the layout bq_weight_rotate_pack writes
+// (4-bit codes, W4A16, use the same kernel).
+//
+// Design (one CTA per SM, persistent over 256 x 128 output tiles, K in stages of 64):
+//  * warp 8 (one thread) loads each stage's activation tile (256 tokens x 64,
+//    128-byte swizzled, the layout the tensor core reads) and the matching packed
+//    codes of 128 output features with the tensor memory accelerator, both
+//    completing on the stage's "full_a" barrier;
+//  * warps 4-7 (one output feature per thread) expand the codes to bfloat16
+//    (q - z) * s in registers and write them into the stage's weight tile in the
+//    same swizzled layout, then arrive on "full_b";
+//  * warp 9 (one thread) issues tcgen05.mma (bf16 x bf16 -> fp32, M = N = 128,
+//    K = 16): two MMAs per K step, one per 128-token half, sharing the weight
+//    tile, so each dequantized weight feeds 256 tokens; a commit per stage frees
+//    the stage, a commit per tile hands the accumulator to the epilogue;
+//  * warps 0-3 read the accumulators from tensor memory (two buffers of 256
+//    columns, so the epilogue of one tile overlaps the main loop of the next),
+//    convert and store them.
+// Dequantization is exact up to the final bfloat16 rounding: a code is placed in
+// the mantissa of 2^23 (one LOP3), (v - (2^23 + z 2^(b j))) is the exact integer
+// (q - z) 2^(b j), and the product with s 2^-(b j) is the exact (q - z) s, which
+// one cvt.rn.bf16x2 rounds; the packed f32x2 forms do two elements per
+// instruction.
+//
+// Every wait on a barrier is bounded (one second): a wait that runs out sets the
+// CTA's abort flag and a bit in the caller's status word, the other roles leave
+// their loops when they see the flag, the copies and MMAs already issued are
+// waited for (again bounded), and the tensor memory is freed before the kernel
+// returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "bq_internal.cuh"
+
+namespace bq {
+namespace {
+
+constexpr int kBM = 256;                                    // tokens per tile (two M = 128 halves)
+constexpr int kBN = 128;                                    // output features per tile
+constexpr int kBK = 64;                                     // K per stage: one 128-byte row of bf16
+constexpr int kStages = 4;
+constexpr int kABytes = kBM * kBK * 2;                      // 32 KiB activation tile
+constexpr int kBBytes = kBN * kBK * 2;                      // 16 KiB dequantized weight tile
+constexpr int kCodeBytes = kBN * 32;                        // packed codes of a stage (4-bit size)
+constexpr int kStageBytes = kABytes + kBBytes + kCodeBytes;  // 52 KiB, a multiple of 1024
+constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kSmemBytes = kBarOff + 256 + 1024;            // barriers, then slack for 1024-byte alignment
+constexpr int kEpiWarps = 4, kDeqWarps = 4, kTmaWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+// barrier block (byte offsets from kBarOff)
+constexpr int kFullA = 0, kFullB = 32, kEmpty = 64, kAccFull = 96, kAccEmpty = 112, kDrain = 128;
+constexpr int kTmemSlot = 136, kAbort = 140;
+
+// status bits: which wait ran out
+constexpr int kStTma = 1, kStDeq = 2, kStMmaOperands = 4, kStMmaAcc = 8, kStEpi = 16, kStDrain = 32;
+
+// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, N = 128, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait for the phase of `parity` to complete.  Returns false when the CTA's abort
+// flag is raised or the wait runs out (then it raises the flag and records `code`).
+__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+                                      int code) {
+  if (mbar_try(bar, parity)) return true;
+  const unsigned long long t0 = gtimer();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try(bar, parity)) return true;
+    if ((i & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (gtimer() - t0 > kWaitLimitNs) {
+        *abort_flag = 1;
+        if (status) atomicOr(status, code);
+        return false;
+      }
+    }
+  }
+}
+
+// A wait that ignores the abort flag (for work already issued), still bounded.
+__device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, int32_t* status) {
+  const unsigned long long t0 = gtimer();
+  while (!mbar_try(bar, parity)) {
+    if (gtimer() - t0 > kWaitLimitNs) {
+      if (status) atomicOr(status, kStDrain);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups 1024 bytes apart
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
+  return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
+      ::"r"(d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t addr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(addr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                 "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                 "+r"(r[29]), "+r"(r[30]), "+r"(r[31])::"memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
+               : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// ------------------------------------------------------------------ dequantization
+
+// Per-group constants of one output feature: for the code at position j of a
+// 16-bit half (bit offset BITS j), nc[j] = -(2^23 + z 2^(BITS j)) and
+// sf[j] = s 2^-(BITS j), held as pairs (j, j + 1) for the f32x2 forms.
+template <int BITS>
+struct Dequant {
+  static constexpr int J = 16 / BITS;  // codes per 16-bit half
+  float2 nc[J / 2], sf[J / 2];
+
+  __device__ __forceinline__ void set(float s, float z) {
+#pragma unroll
+    for (int p = 0; p < J / 2; ++p) {
+      const float w0 = static_cast<float>(1u << (BITS * 2 * p)), w1 = static_cast<float>(1u << (BITS * (2 * p + 1)));
+      nc[p] = make_float2(-(8388608.f + z * w0), -(8388608.f + z * w1));
+      sf[p] = make_float2(s * (1.f / w0), s * (1.f / w1));
+    }
+  }
+
+  // J codes at the bottom 16 bits of x -> J / 2 words of two bfloat16 each
+  __device__ __forceinline__ void half(uint32_t x, uint32_t* out) const {
+#pragma unroll
+    for (int p = 0; p < J / 2; ++p) {
+      constexpr uint32_t kMask = (1u << BITS) - 1u;
+      const uint32_t m0 = kMask << (BITS * 2 * p), m1 = kMask << (BITS * (2 * p + 1));
+      const float2 v = make_float2(__uint_as_float((x & m0) | 0x4B000000u), __uint_as_float((x & m1) | 0x4B000000u));
+      const float2 f = __fmul2_rn(__fadd2_rn(v, nc[p]), sf[p]);
+      out[p] = bf16x2(f.x, f.y);
+    }
+  }
+};
+
+// One output feature's 64 codes of a stage (shared memory at `codes`) -> its row
+// of the weight tile at `row` (128 bytes, 16-byte chunk c stored at c ^ (row & 7)).
+template <int BITS>
+__device__ __forceinline__ void dequant_stage(uint32_t codes, uint32_t row, int sw, const Dequant<BITS>& dq) {
+  uint32_t w[2 * BITS];
+  const uint4 a = ld_shared_v4(codes);
+  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+  if (BITS == 4) {
+    const uint4 b = ld_shared_v4(codes + 16);
+    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    uint32_t o[4];
+    if (BITS == 2) {
+      dq.half(w[c >> 1] >> (16 * (c & 1)), o);
+    } else {
+      dq.half(w[c], o);
+      dq.half(w[c] >> 16, o + 2);
+    }
+    st_shared_v4(row + ((c ^ sw) << 4), o);
+  }
+}
+
+// ------------------------------------------------------------------ epilogue store
+
+template <bool BF16>
+__device__ __forceinline__ void store_row32(void* out, long long t, int out_features, int c0, bool vec,
+                                            const uint32_t (&r)[32]) {
+  if (BF16) {
+    __nv_bfloat16* row = static_cast<__nv_bfloat16*>(out) + t * out_features;
+    if (vec && c0 + 32 <= out_features) {
+      uint4* dst = reinterpret_cast<uint4*>(row + c0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int e = 8 * i;
+        dst[i] = make_uint4(bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])),
+                            bf16x2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])),
+                            bf16x2(__uint_as_float(r[e + 4]), __uint_as_float(r[e + 5])),
+                            bf16x2(__uint_as_float(r[e + 6]), __uint_as_float(r[e + 7])));
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (c0 + e < out_features) row[c0 + e] = __float2bfloat16_rn(__uint_as_float(r[e]));
+    }
+  } else {
+    float* row = static_cast<float*>(out) + t * out_features;
+    if (vec && c0 + 32 <= out_features) {
+      uint4* dst = reinterpret_cast<uint4*>(row + c0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (c0 + e < out_features) row[c0 + e] = __uint_as_float(r[e]);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct GemmArgs {
+  const uint16_t* scale;  // [out_features][n / group] fp16 bits
+  const uint16_t* zero;
+  void* out;              // [tokens][out_features]
+  int tokens, out_features, n, group;
+  int m_tiles, tiles;
+  int vec;                // epilogue may use 16-byte stores
+  int32_t* status;
+};
+
+template <int BITS, bool BF16>
+__global__ void __launch_bounds__(kThreads, 1)
+    k_w2a16(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_codes,
+            const GemmArgs args) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw);
+  const uint32_t bars = base + kBarOff;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kBarOff + kAbort);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kBarOff + kTmemSlot);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kblocks = args.n / kBK;
+  constexpr uint32_t kCodeStage = kBN * kBK * BITS / 8;  // packed bytes of a stage
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(bars + kFullA + 8 * s, 1);
+      mbar_init(bars + kFullB + 8 * s, 32 * kDeqWarps);
+      mbar_init(bars + kEmpty + 8 * s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars + kAccFull + 8 * b, 1);
+      mbar_init(bars + kAccEmpty + 8 * b, 32 * kEpiWarps);
+    }
+    mbar_init(bars + kDrain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == kMmaWarp) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == kTmaWarp && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_x)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_codes)) : "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ---------------------------------------------------------------- loads
+    if (lane == 0) {
+      uint32_t it = 0, issued = 0, last_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
+        const int m0 = (tile % args.m_tiles) * kBM, n0 = (tile / args.m_tiles) * kBN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % kStages, par = (it / kStages) & 1u;
+          if (!wait_bar(bars + kEmpty + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
+            ok = false;
+            break;
+          }
+          const uint32_t st = base + s * kStageBytes;
+          mbar_expect_tx(bars + kFullA + 8 * s, kABytes + kCodeStage);
+          tma_2d(st, &map_x, kb * kBK, m0, bars + kFullA + 8 * s);
+          tma_2d(st + kABytes + kBBytes, &map_codes, kb * (kBK * BITS / 8), n0, bars + kFullA + 8 * s);
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | (par << s);
+        }
+      }
+      // copies still in flight land before the CTA exits
+      for (int s = 0; s < kStages; ++s)
+        if ((issued >> s) & 1u) wait_bar_drain(bars + kFullA + 8 * s, (last_parity >> s) & 1u, args.status);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      uint32_t it = 0;
+      bool ok = true;
+      int i = 0;
+      for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x, ++i) {
+        const uint32_t b = i & 1, use = (i >> 1) & 1;
+        if (!wait_bar(bars + kAccEmpty + 8 * b, use ^ 1u, abort_flag, args.status, kStMmaAcc)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem + 256u * b;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const uint32_t s = it % kStages, par = (it / kStages) & 1u;
+          if (!wait_bar(bars + kFullA + 8 * s, par, abort_flag, args.status, kStMmaOperands) ||
+              !wait_bar(bars + kFullB + 8 * s, par, abort_flag, args.status, kStMmaOperands)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a = base + s * kStageBytes, w = a + kABytes;
+#pragma unroll
+          for (int j = 0; j < kBK / 16; ++j) {
+            const uint64_t bd = sw128_desc(w + 32 * j);
+            const uint32_t acc = (kb | j) != 0;
+            umma_bf16(d0, sw128_desc(a + 32 * j), bd, acc);
+            umma_bf16(d0 + 128, sw128_desc(a + 128 * 128 + 32 * j), bd, acc);
+          }
+          umma_commit(bars + kEmpty + 8 * s);
+        }
+        if (ok) umma_commit(bars + kAccFull + 8 * b);
+      }
+      // every MMA issued has completed before the tensor memory is freed
+      umma_commit(bars + kDrain);
+      wait_bar_drain(bars + kDrain, 0, args.status);
+    }
+    __syncwarp();
+  } else if (warp >= kEpiWarps) {
+    // ---------------------------------------------------------------- dequantization
+    const int d = threadIdx.x - 32 * kEpiWarps;  // output feature of the tile
+    const int sw = d & 7;
+    const int gpr = args.n / args.group, kb_per_group = args.group / kBK;
+    Dequant<BITS> dq;
+    float s_next = 0.f, z_next = 0.f;
+    auto load_sz = [&](int tile, int g) {
+      s_next = 0.f;
+      z_next = 0.f;
+      if (tile < args.tiles) {
+        const long long o = static_cast<long long>(tile / args.m_tiles) * kBN + d;
+        if (o < args.out_features) {
+          s_next = __half2float(__ushort_as_half(__ldg(args.scale + o * gpr + g)));
+          z_next = __half2float(__ushort_as_half(__ldg(args.zero + o * gpr + g)));
+        }
+      }
+    };
+    load_sz(blockIdx.x, 0);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
+      for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        if (kb % kb_per_group == 0) {
+          dq.set(s_next, z_next);
+          const int g = kb / kb_per_group;
+          if (g + 1 < gpr) load_sz(tile, g + 1);
+          else load_sz(tile + gridDim.x, 0);
+        }
+        const uint32_t s = it % kStages, par = (it / kStages) & 1u;
+        if (!wait_bar(bars + kFullA + 8 * s, par, abort_flag, args.status, kStDeq)) {
+          ok = false;
+          break;
+        }
+        const uint32_t st = base + s * kStageBytes;
+        dequant_stage<BITS>(st + kABytes + kBBytes + d * (kBK * BITS / 8), st + kABytes + d * (kBK * 2), sw, dq);
+        fence_proxy_async();
+        mbar_arrive(bars + kFullB + 8 * s);
+      }
+    }
+  } else {
+    // ---------------------------------------------------------------- epilogue
+    int i = 0;
+    for (int tile = blockIdx.x; tile < args.tiles; tile += gridDim.x, ++i) {
+      const uint32_t b = i & 1, use = (i >> 1) & 1;
+      if (!wait_bar(bars + kAccFull + 8 * b, use, abort_flag, args.status, kStEpi)) break;
+      tc_fence_after();
+      const int m0 = (tile % args.m_tiles) * kBM, n0 = (tile / args.m_tiles) * kBN;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        const long long t = m0 + 128 * h + 32 * warp + lane;
+        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + 256u * b + 128u * h;
+#pragma unroll 1
+        for (int q = 0; q < kBN / 32; ++q) {
+          uint32_t r[32];
+          tmem_ld32(taddr + 32u * q, r);
+          tmem_wait_ld(r);
+          if (t < args.tokens) store_row32<BF16>(args.out, t, args.out_features, n0 + 32 * q, args.vec != 0, r);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bars + kAccEmpty + 8 * b);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* ptr, uint64_t inner, uint64_t outer,
+               uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = tensor_map_encoder();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t elem[2] = {1, 1};
+  return fn(map, type, 2, const_cast<void*>(ptr), dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <int BITS, bool BF16>
+bq_status run_gemm(const CUtensorMap& mx, const CUtensorMap& mc, const GemmArgs& a, cudaStream_t st) {
+  auto kern = k_w2a16<BITS, BF16>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = a.tiles < sms ? a.tiles : sms;
+  kern<<<grid, kThreads, kSmemBytes, st>>>(mx, mc, a);
+  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace bq
+
+using namespace bq;
+
+extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, const uint8_t* codes,
+                                   const uint16_t* scale_f16, const uint16_t* zero_f16, int64_t out_features,
+                                   int32_t bits, int32_t group, void* out, bq_dtype out_t, int32_t* status,
+                                   void* stream) {
+  if (tokens < 0 || out_features < 0 || n <= 0 || n % kBK != 0 || (bits != 2 && bits != 4)) return BQ_ERR_INVALID_ARG;
+  if ((group != 64 && group != 128 && group != 256) || n % group != 0) return BQ_ERR_INVALID_ARG;
+  if (out_t != BQ_F32 && out_t != BQ_BF16) return BQ_ERR_INVALID_ARG;
+  if (tokens > 0x7fffffffLL || out_features > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
+  if (tokens == 0 || out_features == 0) return BQ_OK;
+  if (!x || !codes || !scale_f16 || !zero_f16 || !out) return BQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(codes)) return BQ_ERR_INVALID_ARG;
+  CUtensorMap mx, mc;
+  if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(n), static_cast<uint64_t>(tokens),
+                 static_cast<uint64_t>(n) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+    return BQ_ERR_UNSUPPORTED;
+  const uint64_t row_bytes = static_cast<uint64_t>(n) * bits / 8;
+  if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes, static_cast<uint64_t>(out_features), row_bytes,
+                 kBK * bits / 8, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+    return BQ_ERR_UNSUPPORTED;
+  GemmArgs a;
+  a.scale = scale_f16;
+  a.zero = zero_f16;
+  a.out = out;
+  a.tokens = static_cast<int>(tokens);
+  a.out_features = static_cast<int>(out_features);
+  a.n = n;
+  a.group = group;
+  a.m_tiles = static_cast<int>((tokens + kBM - 1) / kBM);
+  const long long tiles = static_cast<long long>(a.m_tiles) * ((out_features + kBN - 1) / kBN);
+  if (tiles > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
+  a.tiles = static_cast<int>(tiles);
+  a.vec = aligned16(out) && out_features % (out_t == BQ_BF16 ? 8 : 4) == 0;
+  a.status = status;
+  auto st = static_cast<cudaStream_t>(stream);
+  if (bits == 2)
+    return out_t == BQ_BF16 ? run_gemm<2, true>(mx, mc, a, st) : run_gemm<2, false>(mx, mc, a, st);
+  return out_t == BQ_BF16 ? run_gemm<4, true>(mx, mc, a, st) : run_gemm<4, false>(mx, mc, a, st);
+}
+
+extern "C" size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens) {
+  if (n <= 0 || tokens < 0) return 0;
+  return (static_cast<size_t>(tokens) * static_cast<size_t>(n) * 2 + 255) & ~static_cast<size_t>(255);
+}
+
+extern "C" bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int64_t tokens,
+                                     const uint8_t* codes, const uint16_t* scale_f16, const uint16_t* zero_f16,
+                                     int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,
+                                     void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!layer || tokens < 0) return BQ_ERR_INVALID_ARG;
+  if (tokens == 0) return BQ_OK;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
+  if (workspace_bytes < bq_w2a16_linear_workspace_size(layer->n, tokens)) return BQ_ERR_WORKSPACE;
+  const bq_status s = bq_butterfly_fwd(layer, x, xt, workspace, BQ_BF16, tokens, stream);
+  if (s != BQ_OK) return s;
+  return bq_w2a16_gemm(workspace, tokens, layer->n, codes, scale_f16, zero_f16, out_features, bits, group, out, out_t,
+                       status, stream);
+}

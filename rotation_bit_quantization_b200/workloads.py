@@ -204,3 +204,25 @@ def shard_rows(total_rows: int, world: int, rank: int):
     start = rank * base + min(rank, extra)
     stop = start + base + (1 if rank < extra else 0)
     return start, stop
+
+
+def packed_weights(rng, out_features: int, n: int, bits: int, group: int):
+    """Random packed low-bit weights in the layout the weight quantizer writes: uniformly random
+    code bytes (so every code is uniform over the 2^bits levels), fp16 scales log-uniform in
+    [2^-9, 2^-5] (the step sizes of N(0, 0.02) rows spread over 3 to 15 levels) and zero points
+    uniform over the levels.  Returns (codes uint8 [out][n*bits/8], scale16, zero16 uint16 bits)."""
+    codes = rng.integers(0, 256, size=(out_features, n * bits // 8), dtype=np.uint8)
+    g = n // group
+    scale16 = (2.0 ** rng.uniform(-9.0, -5.0, size=(out_features, g))).astype(np.float16).view(np.uint16)
+    zero16 = rng.integers(0, 2 ** bits, size=(out_features, g)).astype(np.float16).view(np.uint16)
+    return codes, scale16, zero16
+
+
+def w2a16_4096(tokens: int = 2048, out_features: int = 11008, seed: int = 6):
+    """W2A16 layer of the LLaMA-2-7B MLP shape: rotated activations tokens x 4096 bf16
+    (0.5 * t(nu=3), the act workload's distribution) and INT2 g128 weights of out_features rows.
+    Returns (x bf16 bits, codes, scale16, zero16, bits, group)."""
+    rng = np.random.default_rng([seed, 1])
+    x = bf16_bits_from_f32((0.5 * student_t(rng, 3.0, (tokens, 4096))).astype(np.float32))
+    codes, s16, z16 = packed_weights(np.random.default_rng([seed, 2]), out_features, 4096, 2, 128)
+    return x, codes, s16, z16, 2, 128

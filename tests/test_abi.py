@@ -177,3 +177,34 @@ def test_reconstruction_rejects_bad_arguments(lib):
     assert lib.bq_reconstruction_loss(ctypes.byref(good), *args, 16, None) == _lib.BQ_ERR_WORKSPACE
     assert lib.bq_reconstruction_loss(ctypes.byref(kron), *args, 1 << 30, None) == _lib.BQ_ERR_UNSUPPORTED
     assert lib.bq_reconstruction_loss(None, *args, 1 << 30, None) == _lib.BQ_ERR_INVALID_ARG
+
+
+def test_w2a16_rejects_bad_arguments(lib):
+    ok = (FAKE, 16, 256, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, _lib.BQ_F32, None, None)
+
+    def call(**kw):
+        names = ("x", "tokens", "n", "codes", "scale", "zero", "out_features", "bits", "group", "out", "out_t",
+                 "status", "stream")
+        args = dict(zip(names, ok))
+        args.update(kw)
+        return lib.bq_w2a16_gemm(*[args[k] for k in names])
+
+    bad = _lib.BQ_ERR_INVALID_ARG
+    assert call(n=200) == bad                  # not a multiple of 64
+    assert call(bits=3) == bad
+    assert call(group=32) == bad
+    assert call(n=320, group=128) == bad       # group does not divide n
+    assert call(out_t=7) == bad
+    assert call(x=None) == bad
+    assert call(x=FAKE + 8) == bad             # misaligned activations
+    assert call(codes=FAKE + 4) == bad
+    assert call(tokens=-1) == bad
+    assert call(tokens=0) == _lib.BQ_OK        # nothing to do, nothing launched
+    assert call(out_features=0) == _lib.BQ_OK
+    assert lib.bq_w2a16_linear_workspace_size(4096, 3) == 4096 * 3 * 2
+    assert lib.bq_w2a16_linear_workspace_size(256, 1) == 512
+    layer = _lib.BQLayer(256, 256, 1, FAKE, None)
+    assert lib.bq_w2a16_linear(ctypes.byref(layer), FAKE, 0, 4, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, 0, FAKE, 16,
+                               None, None) == _lib.BQ_ERR_WORKSPACE
+    assert lib.bq_w2a16_linear(ctypes.byref(layer), FAKE, 0, 4, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, 0, FAKE + 16,
+                               1 << 20, None, None) == bad
