@@ -9,26 +9,39 @@
 // with codes, scales and zero points in the layout bq_weight_rotate_pack writes
 // (4-bit codes, W4A16, use the same kernel).
 //
-// Design (one CTA per SM, persistent over 256 x 128 output tiles, K in stages of 64):
-//  * warp 8 (one thread) loads each stage's activation tile (256 tokens x 64,
-//    128-byte swizzled, the layout the tensor core reads) and the matching packed
-//    codes of 128 output features with the tensor memory accelerator, both
-//    completing on the stage's "full_a" barrier;
-//  * warps 4-7 (one output feature per thread) expand the codes to bfloat16
-//    (q - z) * s in registers and write them into the stage's weight tile in the
-//    same swizzled layout, then arrive on "full_b";
-//  * warp 9 (one thread) issues tcgen05.mma (bf16 x bf16 -> fp32, M = N = 128,
-//    K = 16): two MMAs per K step, one per 128-token half, sharing the weight
-//    tile, so each dequantized weight feeds 256 tokens; a commit per stage frees
-//    the stage, a commit per tile hands the accumulator to the epilogue;
-//  * warps 0-3 read the accumulators from tensor memory (two buffers of 256
-//    columns, so the epilogue of one tile overlaps the main loop of the next),
-//    convert and store them.
-// Dequantization is exact up to the final bfloat16 rounding: a code is placed in
-// the mantissa of 2^23 (one LOP3), (v - (2^23 + z 2^(b j))) is the exact integer
-// (q - z) 2^(b j), and the product with s 2^-(b j) is the exact (q - z) s, which
-// one cvt.rn.bf16x2 rounds; the packed f32x2 forms do two elements per
-// instruction.
+// The MMA computes D[o][t] (output features along M, tokens along N) with the
+// dequantized weights as its A operand in TENSOR memory, so they never pass
+// through shared memory: shared memory carries only the activation tiles (written
+// once by the tensor memory accelerator, read once by the MMAs) and the packed
+// codes, which halves its traffic per flop against staging both operands there
+// (shared-memory bandwidth, not the tensor cores, bounds the two-operand form).
+//
+// One CTA per SM, persistent over tiles of 128 output features x 256 tokens, K in
+// stages of 64:
+//  * warp 12 (one thread) loads each stage's activation tile (256 tokens x 64,
+//    128-byte swizzled, the layout the MMA reads) and the packed codes of the
+//    tile's 128 features with the tensor memory accelerator into a 5-deep ring,
+//    completing on "full_x";
+//  * warps 4-11 (two threads per feature, 32 of its 64 codes each) expand a
+//    stage's codes to bfloat16 (q - z) * s in registers and store them with
+//    tcgen05.st into an 8-deep ring of A operands in tensor memory (lane =
+//    feature, 32 columns of bf16 pairs), then arrive on "full_w";
+//  * warp 13 (one thread) issues tcgen05.mma (bf16 x bf16 -> fp32, M = 128,
+//    N = 256, K = 16), so each dequantized weight feeds 256 tokens; commits free
+//    the activation stage and the weight stage, and one per tile hands the
+//    accumulator (256 columns) to the epilogue;
+//  * warps 0-3 read the accumulator (lane = feature), transpose 32 x 32 blocks
+//    through shared memory so that each thread holds one token's 32 consecutive
+//    features, and store them.
+// Dequantization is exact up to the final bfloat16 rounding.  2-bit codes: a
+// group has four possible weights, bf16((q - z) s) for q = 0..3 (the product is
+// exact in float32, one cvt.rn rounds it); their low and high bytes form two
+// 4-byte tables, and each pair of codes becomes one bf16x2 word by a byte
+// permutation whose selector (q0, q0 + 4, q1, q1 + 4) one integer multiply-add
+// builds from the codes.  4-bit codes: a code is placed in the mantissa of 2^23
+// (one LOP3), (v - (2^23 + z 2^(b j))) is the exact integer (q - z) 2^(b j), the
+// product with s 2^-(b j) is the exact (q - z) s, and one cvt.rn.bf16x2 rounds
+// it; the packed f32x2 forms do two elements per instruction.
 //
 // Every wait on a barrier is bounded (one second): a wait that runs out sets the
 // CTA's abort flag and a bit in the caller's status word, the other roles leave
@@ -45,30 +58,32 @@
 namespace bq {
 namespace {
 
-constexpr int kBM = 256;                                    // tokens per tile (two M = 128 halves)
-constexpr int kBN = 128;                                    // output features per tile
-constexpr int kBK = 64;                                     // K per stage: one 128-byte row of bf16
-constexpr int kStages = 4;
-constexpr int kABytes = kBM * kBK * 2;                      // 32 KiB activation tile
-constexpr int kBBytes = kBN * kBK * 2;                      // 16 KiB dequantized weight tile
-constexpr int kCodeBytes = kBN * 32;                        // packed codes of a stage (4-bit size)
-constexpr int kStageBytes = kABytes + kBBytes + kCodeBytes;  // 52 KiB, a multiple of 1024
-constexpr int kBarOff = kStages * kStageBytes;
-constexpr int kSmemBytes = kBarOff + 256 + 1024;            // barriers, then slack for 1024-byte alignment
-constexpr int kEpiWarps = 4, kDeqWarps = 4, kTmaWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kBM = 128;                                 // output features per tile (the MMA's M)
+constexpr int kBN = 256;                                 // tokens per tile (the MMA's N)
+constexpr int kBK = 64;                                  // K per stage: one 128-byte row of bf16
+constexpr int kStages = 5;                               // activation + code ring (shared memory)
+constexpr int kWStages = 8;                              // weight ring (tensor memory)
+constexpr int kXBytes = kBN * kBK * 2;                   // 32 KiB activation tile
+constexpr int kCodeBytes = kBM * kBK / 2;                // packed codes of a stage (4-bit size), 4 KiB
+constexpr int kStageBytes = kXBytes + kCodeBytes;        // 36 KiB, a multiple of 1024
+constexpr int kEpiOff = kStages * kStageBytes;           // epilogue transposes: 4 warps x 32 x 33 floats
+constexpr int kBarOff = kEpiOff + 4 * 32 * 33 * 4;
+constexpr int kSmemBytes = kBarOff + 320 + 1024;         // barriers, then slack for 1024-byte alignment
+constexpr int kEpiWarps = 4, kDeqWarps = 8, kTmaWarp = 12, kMmaWarp = 13;
+constexpr int kThreads = 32 * 14;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColW = 256;                          // weight ring: stage w at columns 256 + 32 w
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // barrier block (byte offsets from kBarOff)
-constexpr int kFullA = 0, kFullB = 32, kEmpty = 64, kAccFull = 96, kAccEmpty = 112, kDrain = 128;
-constexpr int kTmemSlot = 136, kAbort = 140;
+constexpr int kFullX = 0, kEmptyX = 64, kFullW = 128, kEmptyW = 192, kAccFull = 256, kAccEmpty = 264,
+              kDrain = 272, kTmemSlot = 280, kAbort = 284;
 
 // status bits: which wait ran out
 constexpr int kStTma = 1, kStDeq = 2, kStMmaOperands = 4, kStMmaAcc = 8, kStEpi = 16, kStDrain = 32;
 
-// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, N = 128, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(128 >> 4) << 24);
+// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, N = 256, M = 128
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -106,7 +121,7 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 
 // Wait for the phase of `parity` to complete.  Returns false when the CTA's abort
 // flag is raised or the wait runs out (then it raises the flag and records `code`).
-__device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
                                       int code) {
   if (mbar_try(bar, parity)) return true;
   const unsigned long long t0 = gtimer();
@@ -124,7 +139,7 @@ __device__ __noinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile in
 }
 
 // A wait that ignores the abort flag (for work already issued), still bounded.
-__device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, int32_t* status) {
+__device__ __forceinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, int32_t* status) {
   const unsigned long long t0 = gtimer();
   while (!mbar_try(bar, parity)) {
     if (gtimer() - t0 > kWaitLimitNs) {
@@ -135,7 +150,6 @@ __device__ __noinline__ bool wait_bar_drain(uint32_t bar, uint32_t parity, int32
   return true;
 }
 
-__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -151,11 +165,12 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
   return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) | (1ull << 16) | (64ull << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d, uint64_t a, uint64_t b, uint32_t accumulate) {
+// D (tensor memory) (+)= A (tensor memory, 128 lanes x 16 bf16) x B (shared memory, descriptor)
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d, uint32_t a, uint64_t b, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}"
-      ::"r"(d), "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
+      ::"r"(d), "r"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
       : "memory");
 }
 
@@ -184,10 +199,16 @@ __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
                  "+r"(r[29]), "+r"(r[30]), "+r"(r[31])::"memory");
 }
 
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, const uint32_t (&v)[4]) {
-  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3])
-               : "memory");
+__device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      ::"r"(addr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
 }
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -233,62 +254,103 @@ struct Dequant {
   }
 };
 
-// One output feature's 64 codes of a stage (shared memory at `codes`) -> its row
-// of the weight tile at `row` (128 bytes, 16-byte chunk c stored at c ^ (row & 7)).
+// The four weights a 2-bit group can hold as byte tables: byte q of `lo` / `hi` is
+// the low / high byte of bf16((q - z) s).
+struct Lut2 {
+  uint32_t lo, hi;
+
+  __device__ __forceinline__ void set(float s, float z) {
+    const uint32_t p01 = bf16x2((0.f - z) * s, (1.f - z) * s);
+    const uint32_t p23 = bf16x2((2.f - z) * s, (3.f - z) * s);
+    lo = __byte_perm(p01, p23, 0x6420);
+    hi = __byte_perm(p01, p23, 0x7531);
+  }
+
+  // 16 codes of one word (code i at bits 2i) -> 8 words of bf16 pairs (codes 2j, 2j + 1)
+  __device__ __forceinline__ void word(uint32_t c, uint32_t* out) const {
+    const uint32_t m0 = c & 0x03030303u, m1 = (c >> 2) & 0x03030303u;  // byte b: codes 4b, 4b + 1
+    const uint32_t m2 = (c >> 4) & 0x03030303u, m3 = (c >> 6) & 0x03030303u;  // codes 4b + 2, 4b + 3
+    // bytes (qa, qb, qc, qd) -> selector nibbles (qa, qa + 4, qb, qb + 4, qc, qc + 4, qd, qd + 4)
+    const uint32_t g0 = __byte_perm(m0, m1, 0x5140) * 0x11u + 0x40404040u;  // codes 0, 1, 4, 5
+    const uint32_t g1 = __byte_perm(m2, m3, 0x5140) * 0x11u + 0x40404040u;  // codes 2, 3, 6, 7
+    const uint32_t g2 = __byte_perm(m0, m1, 0x7362) * 0x11u + 0x40404040u;  // codes 8, 9, 12, 13
+    const uint32_t g3 = __byte_perm(m2, m3, 0x7362) * 0x11u + 0x40404040u;  // codes 10, 11, 14, 15
+    out[0] = __byte_perm(lo, hi, g0);
+    out[1] = __byte_perm(lo, hi, g1);
+    out[2] = __byte_perm(lo, hi, g0 >> 16);
+    out[3] = __byte_perm(lo, hi, g1 >> 16);
+    out[4] = __byte_perm(lo, hi, g2);
+    out[5] = __byte_perm(lo, hi, g3);
+    out[6] = __byte_perm(lo, hi, g2 >> 16);
+    out[7] = __byte_perm(lo, hi, g3 >> 16);
+  }
+};
+
+// Per-group expansion state: the byte tables for 2-bit codes, the f32x2 constants
+// for 4-bit codes.
 template <int BITS>
-__device__ __forceinline__ void dequant_stage(uint32_t codes, uint32_t row, int sw, const Dequant<BITS>& dq) {
-  uint32_t w[2 * BITS];
-  const uint4 a = ld_shared_v4(codes);
-  w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-  if (BITS == 4) {
-    const uint4 b = ld_shared_v4(codes + 16);
-    w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+struct Expand;
+
+template <>
+struct Expand<2> {
+  Lut2 t;
+  __device__ __forceinline__ void set(float s, float z) { t.set(s, z); }
+  // 32 codes (8 bytes at `codes` in shared memory) -> 16 words
+  __device__ __forceinline__ void run(uint32_t codes, uint32_t (&v)[16]) const {
+    uint32_t a, b;
+    asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(a), "=r"(b) : "r"(codes) : "memory");
+    t.word(a, v);
+    t.word(b, v + 8);
   }
+};
+
+template <>
+struct Expand<4> {
+  Dequant<4> dq;
+  __device__ __forceinline__ void set(float s, float z) { dq.set(s, z); }
+  // 32 codes (16 bytes at `codes` in shared memory) -> 16 words
+  __device__ __forceinline__ void run(uint32_t codes, uint32_t (&v)[16]) const {
+    const uint4 a = ld_shared_v4(codes);
+    const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    uint32_t o[4];
-    if (BITS == 2) {
-      dq.half(w[c >> 1] >> (16 * (c & 1)), o);
-    } else {
-      dq.half(w[c], o);
-      dq.half(w[c] >> 16, o + 2);
+    for (int c = 0; c < 4; ++c) {
+      dq.half(w[c], v + 4 * c);
+      dq.half(w[c] >> 16, v + 4 * c + 2);
     }
-    st_shared_v4(row + ((c ^ sw) << 4), o);
   }
-}
+};
 
 // ------------------------------------------------------------------ epilogue store
 
+// 32 consecutive features o0 .. o0 + 31 of token t
 template <bool BF16>
-__device__ __forceinline__ void store_row32(void* out, long long t, int out_features, int c0, bool vec,
-                                            const uint32_t (&r)[32]) {
+__device__ __forceinline__ void store_row32(void* out, long long t, int out_features, int o0, bool vec,
+                                            const float (&r)[32]) {
   if (BF16) {
     __nv_bfloat16* row = static_cast<__nv_bfloat16*>(out) + t * out_features;
-    if (vec && c0 + 32 <= out_features) {
-      uint4* dst = reinterpret_cast<uint4*>(row + c0);
+    if (vec && o0 + 32 <= out_features) {
+      uint4* dst = reinterpret_cast<uint4*>(row + o0);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int e = 8 * i;
-        dst[i] = make_uint4(bf16x2(__uint_as_float(r[e]), __uint_as_float(r[e + 1])),
-                            bf16x2(__uint_as_float(r[e + 2]), __uint_as_float(r[e + 3])),
-                            bf16x2(__uint_as_float(r[e + 4]), __uint_as_float(r[e + 5])),
-                            bf16x2(__uint_as_float(r[e + 6]), __uint_as_float(r[e + 7])));
+        dst[i] = make_uint4(bf16x2(r[e], r[e + 1]), bf16x2(r[e + 2], r[e + 3]), bf16x2(r[e + 4], r[e + 5]),
+                            bf16x2(r[e + 6], r[e + 7]));
       }
     } else {
 #pragma unroll
       for (int e = 0; e < 32; ++e)
-        if (c0 + e < out_features) row[c0 + e] = __float2bfloat16_rn(__uint_as_float(r[e]));
+        if (o0 + e < out_features) row[o0 + e] = __float2bfloat16_rn(r[e]);
     }
   } else {
     float* row = static_cast<float*>(out) + t * out_features;
-    if (vec && c0 + 32 <= out_features) {
-      uint4* dst = reinterpret_cast<uint4*>(row + c0);
+    if (vec && o0 + 32 <= out_features) {
+      float4* dst = reinterpret_cast<float4*>(row + o0);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) dst[i] = make_uint4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+      for (int i = 0; i < 8; ++i) dst[i] = make_float4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
     } else {
 #pragma unroll
       for (int e = 0; e < 32; ++e)
-        if (c0 + e < out_features) row[c0 + e] = __uint_as_float(r[e]);
+        if (o0 + e < out_features) row[o0 + e] = r[e];
     }
   }
 }
@@ -300,7 +362,7 @@ struct GemmArgs {
   const uint16_t* zero;
   void* out;              // [tokens][out_features]
   int tokens, out_features, n, group;
-  int m_tiles, tiles;
+  int t_tiles, tiles;     // token tiles of 128, and all tiles (token tile fastest)
   int vec;                // epilogue may use 16-byte stores
   int32_t* status;
 };
@@ -318,18 +380,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kBarOff + kTmemSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kblocks = args.n / kBK;
-  constexpr uint32_t kCodeStage = kBN * kBK * BITS / 8;  // packed bytes of a stage
+  constexpr uint32_t kCodeRow = kBK * BITS / 8;             // packed bytes of one feature per stage
+  constexpr uint32_t kTx = kXBytes + kBM * kCodeRow;        // bytes a stage's copies deliver
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(bars + kFullA + 8 * s, 1);
-      mbar_init(bars + kFullB + 8 * s, 32 * kDeqWarps);
-      mbar_init(bars + kEmpty + 8 * s, 1);
+      mbar_init(bars + kFullX + 8 * s, 1);
+      mbar_init(bars + kEmptyX + 8 * s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bars + kAccFull + 8 * b, 1);
-      mbar_init(bars + kAccEmpty + 8 * b, 32 * kEpiWarps);
+    for (int s = 0; s < kWStages; ++s) {
+      mbar_init(bars + kFullW + 8 * s, 32 * kDeqWarps);
+      mbar_init(bars + kEmptyW + 8 * s, 1);
     }
+    mbar_init(bars + kAccFull, 1);
+    mbar_init(bars + kAccEmpty, 32 * kEpiWarps);
     mbar_init(bars + kDrain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -355,24 +419,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, issued = 0, last_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
-        const int m0 = (tile % args.m_tiles) * kBM, n0 = (tile / args.m_tiles) * kBN;
+        const int t0 = (tile % args.t_tiles) * kBN, o0 = (tile / args.t_tiles) * kBM;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-          if (!wait_bar(bars + kEmpty + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
+          if (!wait_bar(bars + kEmptyX + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
             ok = false;
             break;
           }
           const uint32_t st = base + s * kStageBytes;
-          mbar_expect_tx(bars + kFullA + 8 * s, kABytes + kCodeStage);
-          tma_2d(st, &map_x, kb * kBK, m0, bars + kFullA + 8 * s);
-          tma_2d(st + kABytes + kBBytes, &map_codes, kb * (kBK * BITS / 8), n0, bars + kFullA + 8 * s);
+          mbar_expect_tx(bars + kFullX + 8 * s, kTx);
+          tma_2d(st, &map_x, kb * kBK, t0, bars + kFullX + 8 * s);
+          tma_2d(st + kXBytes, &map_codes, kb * kCodeRow, o0, bars + kFullX + 8 * s);
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | (par << s);
         }
       }
       // copies still in flight land before the CTA exits
       for (int s = 0; s < kStages; ++s)
-        if ((issued >> s) & 1u) wait_bar_drain(bars + kFullA + 8 * s, (last_parity >> s) & 1u, args.status);
+        if ((issued >> s) & 1u) wait_bar_drain(bars + kFullX + 8 * s, (last_parity >> s) & 1u, args.status);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
@@ -382,29 +446,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       int i = 0;
       for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x, ++i) {
-        const uint32_t b = i & 1, use = (i >> 1) & 1;
-        if (!wait_bar(bars + kAccEmpty + 8 * b, use ^ 1u, abort_flag, args.status, kStMmaAcc)) break;
+        // one accumulator set: tile i starts once the epilogue has read tile i - 1
+        if (!wait_bar(bars + kAccEmpty, (i & 1) ^ 1, abort_flag, args.status, kStMmaAcc)) break;
         tc_fence_after();
-        const uint32_t d0 = tmem + 256u * b;
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
           const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-          if (!wait_bar(bars + kFullA + 8 * s, par, abort_flag, args.status, kStMmaOperands) ||
-              !wait_bar(bars + kFullB + 8 * s, par, abort_flag, args.status, kStMmaOperands)) {
+          const uint32_t w = it % kWStages, wpar = (it / kWStages) & 1u;
+          if (!wait_bar(bars + kFullX + 8 * s, par, abort_flag, args.status, kStMmaOperands) ||
+              !wait_bar(bars + kFullW + 8 * w, wpar, abort_flag, args.status, kStMmaOperands)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a = base + s * kStageBytes, w = a + kABytes;
+          const uint32_t x = base + s * kStageBytes;
+          const uint32_t a = tmem + kColW + 32u * w;
 #pragma unroll
-          for (int j = 0; j < kBK / 16; ++j) {
-            const uint64_t bd = sw128_desc(w + 32 * j);
-            const uint32_t acc = (kb | j) != 0;
-            umma_bf16(d0, sw128_desc(a + 32 * j), bd, acc);
-            umma_bf16(d0 + 128, sw128_desc(a + 128 * 128 + 32 * j), bd, acc);
-          }
-          umma_commit(bars + kEmpty + 8 * s);
+          for (int j = 0; j < kBK / 16; ++j) umma_bf16_ta(tmem, a + 8 * j, sw128_desc(x + 32 * j), (kb | j) != 0);
+          umma_commit(bars + kEmptyX + 8 * s);
+          umma_commit(bars + kEmptyW + 8 * w);
         }
-        if (ok) umma_commit(bars + kAccFull + 8 * b);
+        if (ok) umma_commit(bars + kAccFull);
       }
       // every MMA issued has completed before the tensor memory is freed
       umma_commit(bars + kDrain);
@@ -413,16 +474,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp >= kEpiWarps) {
     // ---------------------------------------------------------------- dequantization
-    const int d = threadIdx.x - 32 * kEpiWarps;  // output feature of the tile
-    const int sw = d & 7;
+    const int dw = warp - kEpiWarps;             // 0 .. 7
+    const int f = 32 * (dw & 3) + lane;          // feature of the tile = tensor-memory lane, 0 .. 127
+    const int kh = dw >> 2;                      // which 32 of the stage's 64 codes
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const uint32_t col = 16u * kh;
     const int gpr = args.n / args.group, kb_per_group = args.group / kBK;
-    Dequant<BITS> dq;
+    Expand<BITS> ex;
     float s_next = 0.f, z_next = 0.f;
     auto load_sz = [&](int tile, int g) {
       s_next = 0.f;
       z_next = 0.f;
       if (tile < args.tiles) {
-        const long long o = static_cast<long long>(tile / args.m_tiles) * kBN + d;
+        const long long o = static_cast<long long>(tile / args.t_tiles) * kBM + f;
         if (o < args.out_features) {
           s_next = __half2float(__ushort_as_half(__ldg(args.scale + o * gpr + g)));
           z_next = __half2float(__ushort_as_half(__ldg(args.zero + o * gpr + g)));
@@ -435,44 +499,59 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
       for (int kb = 0; kb < kblocks; ++kb, ++it) {
         if (kb % kb_per_group == 0) {
-          dq.set(s_next, z_next);
+          ex.set(s_next, z_next);
           const int g = kb / kb_per_group;
           if (g + 1 < gpr) load_sz(tile, g + 1);
           else load_sz(tile + gridDim.x, 0);
         }
         const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-        if (!wait_bar(bars + kFullA + 8 * s, par, abort_flag, args.status, kStDeq)) {
+        const uint32_t w = it % kWStages, wpar = (it / kWStages) & 1u;
+        if (!wait_bar(bars + kFullX + 8 * s, par, abort_flag, args.status, kStDeq)) {
           ok = false;
           break;
         }
-        const uint32_t st = base + s * kStageBytes;
-        dequant_stage<BITS>(st + kABytes + kBBytes + d * (kBK * BITS / 8), st + kABytes + d * (kBK * 2), sw, dq);
-        fence_proxy_async();
-        mbar_arrive(bars + kFullB + 8 * s);
+        uint32_t v[16];
+        ex.run(base + s * kStageBytes + kXBytes + f * kCodeRow + kh * (kCodeRow / 2), v);
+        if (!wait_bar(bars + kEmptyW + 8 * w, wpar ^ 1u, abort_flag, args.status, kStDeq)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        tmem_st16(tmem + lane_base + kColW + 32u * w + col, v);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bars + kFullW + 8 * w);
       }
     }
   } else {
     // ---------------------------------------------------------------- epilogue
+    float* buf = reinterpret_cast<float*>(gbase + kEpiOff) + warp * (32 * 33);
     int i = 0;
     for (int tile = blockIdx.x; tile < args.tiles; tile += gridDim.x, ++i) {
-      const uint32_t b = i & 1, use = (i >> 1) & 1;
-      if (!wait_bar(bars + kAccFull + 8 * b, use, abort_flag, args.status, kStEpi)) break;
+      if (!wait_bar(bars + kAccFull, i & 1, abort_flag, args.status, kStEpi)) break;
       tc_fence_after();
-      const int m0 = (tile % args.m_tiles) * kBM, n0 = (tile / args.m_tiles) * kBN;
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const long long t = m0 + 128 * h + 32 * warp + lane;
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(32 * warp) << 16) + 256u * b + 128u * h;
+      const int t0 = (tile % args.t_tiles) * kBN, o0 = (tile / args.t_tiles) * kBM;
+      {
 #pragma unroll 1
         for (int q = 0; q < kBN / 32; ++q) {
           uint32_t r[32];
-          tmem_ld32(taddr + 32u * q, r);
+          tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32u * q, r);
           tmem_wait_ld(r);
-          if (t < args.tokens) store_row32<BF16>(args.out, t, args.out_features, n0 + 32 * q, args.vec != 0, r);
+          // r[j] = D[feature 32 warp + lane][token 32 q + j]: transpose so that this
+          // thread holds token 32 q + lane's 32 features
+#pragma unroll
+          for (int j = 0; j < 32; ++j) buf[j * 33 + lane] = __uint_as_float(r[j]);
+          __syncwarp();
+          float c[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) c[j] = buf[lane * 33 + j];
+          __syncwarp();
+          const long long t = t0 + 32 * q + lane;
+          if (t < args.tokens) store_row32<BF16>(args.out, t, args.out_features, o0 + 32 * warp, args.vec != 0, c);
         }
       }
       tc_fence_before();
-      mbar_arrive(bars + kAccEmpty + 8 * b);
+      mbar_arrive(bars + kAccEmpty);
     }
   }
 
@@ -543,11 +622,11 @@ extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, con
   if (!aligned16(x) || !aligned16(codes)) return BQ_ERR_INVALID_ARG;
   CUtensorMap mx, mc;
   if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(n), static_cast<uint64_t>(tokens),
-                 static_cast<uint64_t>(n) * 2, kBK, kBM, CU_TENSOR_MAP_SWIZZLE_128B))
+                 static_cast<uint64_t>(n) * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
     return BQ_ERR_UNSUPPORTED;
   const uint64_t row_bytes = static_cast<uint64_t>(n) * bits / 8;
   if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes, static_cast<uint64_t>(out_features), row_bytes,
-                 kBK * bits / 8, kBN, CU_TENSOR_MAP_SWIZZLE_NONE))
+                 kBK * bits / 8, kBM, CU_TENSOR_MAP_SWIZZLE_NONE))
     return BQ_ERR_UNSUPPORTED;
   GemmArgs a;
   a.scale = scale_f16;
@@ -557,8 +636,8 @@ extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, con
   a.out_features = static_cast<int>(out_features);
   a.n = n;
   a.group = group;
-  a.m_tiles = static_cast<int>((tokens + kBM - 1) / kBM);
-  const long long tiles = static_cast<long long>(a.m_tiles) * ((out_features + kBN - 1) / kBN);
+  a.t_tiles = static_cast<int>((tokens + kBN - 1) / kBN);
+  const long long tiles = static_cast<long long>(a.t_tiles) * ((out_features + kBM - 1) / kBM);
   if (tiles > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
   a.tiles = static_cast<int>(tiles);
   a.vec = aligned16(out) && out_features % (out_t == BQ_BF16 ? 8 : 4) == 0;
