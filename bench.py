@@ -57,6 +57,10 @@ def workload_spec(name: str):
         return dict(make=None, kind="uniformity", rows=65536, n=4096, bits=4, group=128, layers=1,
                     label="uniformity regulariser: 65536 tokens x n=4096 float32 rotated activations -> "
                           "per-group KL to uniform over the INT4 g128 levels + dL/dY (one calibration batch of one layer)")
+    if name == "w2a16":
+        return dict(make=None, kind="gemm", rows=2048, n=4096, bits=2, group=128, out_features=11008,
+                    label="W2A16 linear: rotated activations 2048 x 4096 bf16 times INT2 g128 weights 11008 x 4096 "
+                          "-> 2048 x 11008 bf16 (LLaMA-2-7B MLP up-projection shape)")
     if name == "act5120":
         return dict(make=lambda rank: wl.act_5120(8192), kind="quant", rows=8192, n=5120, bits=4, group=128,
                     label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> INT4 RTN g128 (LLaMA-2-13B shape)")
@@ -492,6 +496,133 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
     }
 
 
+def oracle_gemm_rate(x_bits, codes, s16, z16, bits, group, tokens_sample):
+    """Output elements/s of the float64 oracle GEMM on a bounded sample of tokens (all features),
+    counting the dequantization of the whole weight matrix."""
+    from oracle import w2a16 as ow
+    from rotation_bit_quantization_b200 import workloads as wl
+    xs = wl.f32_from_bf16_bits(x_bits[:tokens_sample])
+    t0 = time.perf_counter()
+    ow.w2a16_gemm(xs, codes, s16, z16, bits, group)
+    el = time.perf_counter() - t0
+    flops = 2.0 * tokens_sample * x_bits.shape[1] * codes.shape[0]
+    return flops / el, el
+
+
+def run_gemm_bench(args, spec, rank, world, local_rank):
+    """The W2A16 consumer GEMM (bq_w2a16_gemm) on the LLaMA-2-7B MLP shape."""
+    import torch
+    import torch.distributed as dist
+
+    import rotation_bit_quantization_b200 as bq
+    from rotation_bit_quantization_b200 import build as bq_build
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    bq_build.build()
+    bq.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    tokens = spec["rows"]
+    xb, codes_h, s16, z16, bits, group = wl.w2a16_4096(tokens, spec["out_features"], seed=6 + rank)
+    n, out_f = xb.shape[1], codes_h.shape[0]
+    x_host = torch.from_numpy(xb.view(np.int16)).view(torch.bfloat16)
+    x = x_host.to(dev)
+    codes = torch.from_numpy(codes_h).to(dev)
+    scale = torch.from_numpy(s16.view(np.int16)).to(dev)
+    zero = torch.from_numpy(z16.view(np.int16)).to(dev)
+    out = torch.empty((tokens, out_f), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bq.bq_w2a16_gemm(x, codes, scale, zero, bits, group, out, status)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id_for(dev))
+    t_busy = time.perf_counter()
+    while time.perf_counter() - t_busy < 0.5:
+        for _ in range(10):
+            flush.zero_()
+            step()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for s_, e_ in evs:
+        flush.zero_()
+        s_.record(stream)
+        step()
+        e_.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise SystemExit(f"w2a16 kernel reported a wait timeout (status {int(status.item())})")
+    total_ms = float(sum(s_.elapsed_time(e_) for s_, e_ in evs))
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / args.steps
+    flops = 2.0 * tokens * n * out_f
+    tflops = flops * world / (ms * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_host.pin_memory()
+        o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        x_dev = torch.empty_like(x)
+
+        def e2e_step():
+            x_dev.copy_(x_pin, non_blocking=True)
+            bq.bq_w2a16_gemm(x_dev, codes, scale, zero, bits, group, out, status)
+            o_pin.copy_(out, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": flops * world / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, el = oracle_gemm_rate(xb, codes_h, s16, z16, bits, group, tokens_sample=256)
+        cpu = {"value": rate / 1e12, "unit": "TFLOP/s", "cores": len(os.sched_getaffinity(0)), "kind": "oracle",
+               "sample": f"256 of {tokens} tokens x all {out_f} features, dequantization of the whole weight "
+                         f"matrix included, {el:.1f} s (numpy float64 matmul on the host's BLAS threads)"}
+    peaks, peak_src = load_peaks()
+    traffic, traffic_kernel = recorded_traffic("w2a16")
+    return {
+        "metric": "W2A16 GEMM TFLOP/s (bf16 x INT2 g128 on tcgen05), 2048 x 4096 x 11008", "value": tflops,
+        "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded)", "config": {"workload": spec["label"], "tokens": tokens, "n": n,
+                                                 "out_features": out_f, "bits": bits, "group": group,
+                                                 "l2": "1 GiB written between timed steps (L2 flushed)"},
+        "roofline": {"bound": "tensor", "achieved": tflops / world, "peak": peaks.get("bf16_tflops", 1590.0),
+                     "unit": "TFLOP/s", "frac": tflops / world / peaks.get("bf16_tflops", 1590.0),
+                     "traffic": traffic, "peak_source": peak_src + " (bf16 burst)",
+                     "algorithmic_flops_per_launch": flops, "kernel": traffic_kernel or "k_w2a16"},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args, spec):
@@ -536,7 +667,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="act4096",
-                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity"])
+                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity", "w2a16"])
     ap.add_argument("--rows", type=int, default=0, help="override the workload's rows (tokens per layer for bwd)")
     ap.add_argument("--layers", type=int, default=0, help="override the backward workload's layer count")
     ap.add_argument("--no-e2e", action="store_true")
@@ -553,8 +684,8 @@ def main():
         # that has to fit the profiling size rules; never the bench line's size
         from rotation_bit_quantization_b200 import workloads as wl
         rows = args.rows or spec["rows"]
-        if spec["kind"] in ("bwd", "uniformity"):
-            spec = dict(spec, rows=rows, layers=args.layers or spec["layers"])
+        if spec["kind"] in ("bwd", "uniformity", "gemm"):
+            spec = dict(spec, rows=rows, layers=args.layers or spec.get("layers", 1))
         else:
             base = {"act4096": lambda r, k: wl.act_4096(r, seed_offset=k), "fwd4096": lambda r, k: wl.act_4096(r, seed_offset=k),
                     "weight4096": lambda r, k: wl.weight_4096(r), "act5120": lambda r, k: wl.act_5120(r)}[args.workload]
@@ -563,7 +694,7 @@ def main():
             f", layers={spec['layers']}]" if spec["kind"] == "bwd" else "]")
 
     if args.impl == "reference":
-        if spec["kind"] in ("bwd", "uniformity"):
+        if spec["kind"] in ("bwd", "uniformity", "gemm"):
             raise SystemExit("--impl reference covers the transform + quantize workloads only")
         if rank != 0:
             return 0
@@ -583,6 +714,8 @@ def main():
             res = run_bwd_bench(args, spec, rank, world, local_rank)
         elif spec["kind"] == "uniformity":
             res = run_uniformity_bench(args, spec, rank, world, local_rank)
+        elif spec["kind"] == "gemm":
+            res = run_gemm_bench(args, spec, rank, world, local_rank)
         else:
             res = run_ours(args, spec, rank, world, local_rank)
     finally:
