@@ -102,6 +102,29 @@ def forward(theta, x):
     return x
 
 
+def hadamard_preset_forward(quadrant, x):
+    """y = Q x for the Hadamard preset: rotation (s, p) at the angle pi/4 + k pi/2,
+    k = quadrant[s][p] & 3 (quadrant None: k = 0 everywhere), with its cos and sin
+    taken as exactly +-1/sqrt(2).  H_n is the butterfly at particular angles
+    (explainer article, section "butterfly"); every entry of the result is
+    +-1/sqrt(n)."""
+    x = np.asarray(x, dtype=np.float64)
+    m = x.shape[-1]
+    r = 1.0 / np.sqrt(2.0)
+    for s in range(num_stages(m)):
+        i, j, p = pair_indices(m, s)
+        k = np.zeros(len(p), dtype=np.int64) if quadrant is None else (np.asarray(quadrant)[s][p].astype(np.int64) & 3)
+        c = np.where((k == 0) | (k == 3), r, -r)
+        sn = np.where(k <= 1, r, -r)
+        xi = x[..., i]
+        xj = x[..., j]
+        y = np.empty_like(x)
+        y[..., i] = c * xi - sn * xj
+        y[..., j] = sn * xi + c * xj
+        x = y
+    return x
+
+
 def inverse(theta, y):
     """x = Q^T y: stages L-1, ..., 0 with every angle negated (Q is orthogonal)."""
     y = np.asarray(y, dtype=np.float64)
