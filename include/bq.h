@@ -79,6 +79,21 @@ size_t bq_table_floats(int32_t m);
  * The table must be rebuilt whenever theta changes. */
 bq_status bq_precompute_cs(const float* theta, int32_t m, float* table, void* stream);
 
+/* Hadamard presets: the table of the butterfly at the angles that make it a
+ * Hadamard matrix (explainer article, section "butterfly": H_n is a butterfly
+ * with particular angles; QuaRot's fixed and UniSVQ's randomized Hadamard
+ * rotations are the baselines the pages compare with).  Angle (s, p) is
+ * pi/4 + k pi/2 with k = quadrant[s*(m/2) + p] & 3 (quadrant: device bytes
+ * [log2(m)*(m/2)], or NULL for k = 0 everywhere, which gives
+ * Q = H_m diag(d) / sqrt(m) with d the Kronecker power of (1, -1)).  Every
+ * entry of Q is +-1/sqrt(m).  cos and sin are taken as +-1/sqrt(2) exactly,
+ * so the scaled-form coefficients are exactly +-1 and the output scale is
+ * +-2^(-log2(m)/2) (a power of two for even log2 m).
+ * theta: NULL, or device float32 [log2(m)*(m/2)] that receives the angles (a
+ * starting point for calibration; bq_precompute_cs of them reproduces the
+ * table up to float32 rounding of the angles). */
+bq_status bq_precompute_hadamard(int32_t m, const uint8_t* quadrant, float* table, float* theta, void* stream);
+
 /* y = Q x for every row (abstract: the activation side Q x).
  * x: rows*n elements of type xt; y: rows*n elements of type yt.  x == y is
  * allowed when xt == yt (each row is read completely before it is written). */

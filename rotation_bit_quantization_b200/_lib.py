@@ -21,6 +21,7 @@ BQ_F32, BQ_BF16 = 0, 1
 EXPORTED = (
     "bq_table_floats",
     "bq_precompute_cs",
+    "bq_precompute_hadamard",
     "bq_butterfly_fwd",
     "bq_butterfly_inv",
     "bq_butterfly_bwd_workspace_size",
@@ -68,6 +69,7 @@ def load(path: str | None = None):
     sig = {
         "bq_table_floats": (sz, [i32]),
         "bq_precompute_cs": (i32, [vp, i32, vp, vp]),
+        "bq_precompute_hadamard": (i32, [i32, vp, vp, vp, vp]),
         "bq_butterfly_fwd": (i32, [lp, vp, i32, vp, i32, i64, vp]),
         "bq_butterfly_inv": (i32, [lp, vp, i32, vp, i32, i64, vp]),
         "bq_butterfly_bwd_workspace_size": (sz, [i32, i32, i64]),
@@ -160,6 +162,31 @@ class Layer:
         bq_precompute_cs(theta, self.m, self.table, stream)
         self.c = BQLayer(self.n, self.m, self.r, self.table.data_ptr(),
                          None if self.O is None else self.O.data_ptr())
+
+    @classmethod
+    def hadamard(cls, m: int, quadrant=None, O=None, device="cuda", stream=None):
+        """The Hadamard preset of width m (bq_precompute_hadamard): every angle pi/4, or
+        pi/4 + k pi/2 with k from `quadrant` (uint8 CUDA tensor of shape (log2 m, m/2))."""
+        torch = _torch()
+        lib = load()
+        L = m.bit_length() - 1
+        if m < 2 or (1 << L) != m or lib.bq_table_floats(m) == 0:
+            raise ValueError(f"unsupported butterfly width m={m}")
+        if quadrant is not None:
+            _dev(quadrant, "quadrant")
+            if quadrant.dtype != torch.uint8 or quadrant.numel() != L * (m // 2):
+                raise ValueError("quadrant must be uint8 with log2(m) * m/2 elements")
+        self = cls.__new__(cls)
+        self.m, self.r = m, 1 if O is None else int(O.shape[0])
+        self.n = self.m * self.r
+        self.theta = torch.empty((L, m // 2), dtype=torch.float32, device=device)
+        self.table = torch.empty(lib.bq_table_floats(m), dtype=torch.float32, device=device)
+        self.O = None if O is None else _dev(O, "O")
+        _check("bq_precompute_hadamard", lib.bq_precompute_hadamard(m, _ptr(quadrant), _ptr(self.table),
+                                                                    _ptr(self.theta), _stream(stream)))
+        self.c = BQLayer(self.n, self.m, self.r, self.table.data_ptr(),
+                         None if self.O is None else self.O.data_ptr())
+        return self
 
     @property
     def fast_form(self) -> bool:

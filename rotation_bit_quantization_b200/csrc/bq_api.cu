@@ -85,6 +85,11 @@ bq_status bq_precompute_cs(const float* theta, int32_t m, float* table, void* st
   return launch_prepare(theta, m, table, static_cast<cudaStream_t>(stream));
 }
 
+bq_status bq_precompute_hadamard(int32_t m, const uint8_t* quadrant, float* table, float* theta, void* stream) {
+  if (!valid_m(m) || !table || !aligned16(table) || (reinterpret_cast<uintptr_t>(theta) & 3u)) return BQ_ERR_INVALID_ARG;
+  return launch_prepare_hadamard(quadrant, theta, m, table, static_cast<cudaStream_t>(stream));
+}
+
 bq_status bq_butterfly_fwd(const bq_layer* layer, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                            void* stream) {
   return transform(layer, x, xt, y, yt, rows, stream, false);

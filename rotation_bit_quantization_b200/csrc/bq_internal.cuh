@@ -94,6 +94,7 @@ struct QuantArgs {
 
 // Launchers (defined in the .cu files).  Each returns BQ_OK or BQ_ERR_CUDA.
 bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t st);
+bq_status launch_prepare_hadamard(const uint8_t* quadrant, float* theta_out, int m, float* table, cudaStream_t st);
 bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool fast4096_supports(const KLayer& L, const QuantArgs* q);

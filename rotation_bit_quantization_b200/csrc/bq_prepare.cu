@@ -76,6 +76,50 @@ __global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ t
   }
 }
 
+// Hadamard presets.  H_n is the butterfly at particular angles (explainer
+// article, section "butterfly"): at theta = pi/4 every rotation is
+// [[1, -1], [1, 1]] / sqrt(2).  theta = pi/4 + k pi/2 (k = 0..3) gives the four
+// rotations with entries +-1/sqrt(2), so a product of such stages has every entry
+// +-1/sqrt(n): k = 0 everywhere is the fixed Hadamard transform, random k per
+// rotation a randomized one.  The angles' cos and sin are +-1/sqrt(2) exactly in
+// float64 here (not float32 angles through sincos), so t = s / c is +-1, every
+// coefficient of the scaled form is exactly +-1 (all positions carry the same
+// |scale| at each stage) and the output scale is +-(1/sqrt(2))^L: the forward
+// kernels then compute the butterfly with exact coefficient products.
+__global__ void k_prepare_hadamard(const uint8_t* __restrict__ quadrant, float* __restrict__ table,
+                                   float* __restrict__ theta_out, TableLayout tl) {
+  extern __shared__ double d[];
+  const int m = tl.m, L = tl.L, half = m / 2;
+  const int tid = threadIdx.x, T = blockDim.x;
+  float2* cs = reinterpret_cast<float2*>(table + tl.off_cs);
+  float* fast = table + tl.off_fast;
+  float* sigma = table + tl.off_sigma;
+  const double r = 0.70710678118654752440;  // 1 / sqrt(2)
+  const double kPi = 3.14159265358979323846;
+  for (int i = tid; i < m; i += T) d[i] = 1.0;
+  __syncthreads();
+  for (int s = 0; s < L; ++s) {
+    for (int p = tid; p < half; p += T) {
+      const int k = quadrant ? (quadrant[s * half + p] & 3) : 0;
+      const double c = (k == 0 || k == 3) ? r : -r;   // cos(pi/4 + k pi/2)
+      const double sn = (k <= 1) ? r : -r;            // sin(pi/4 + k pi/2)
+      cs[s * half + p] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+      if (theta_out) theta_out[s * half + p] = static_cast<float>(kPi / 4 + (k < 2 ? k : k - 4) * (kPi / 2));
+      const int i = ((p >> s) << (s + 1)) | (p & ((1 << s) - 1));
+      const int j = i + (1 << s);
+      const double di = d[i], dj = d[j], t = sn / c;
+      fast[size_t(s) * m + i] = static_cast<float>(-t * dj / di);
+      fast[size_t(s) * m + j] = static_cast<float>(t * di / dj);
+      d[i] = di * c;
+      d[j] = dj * c;
+    }
+    __syncthreads();
+  }
+  for (int i = tid; i < m; i += T) sigma[i] = static_cast<float>(d[i]);
+  __syncthreads();
+  if (tid < 16) table[tid] = tid == 0 ? 1.f : tid == 1 ? static_cast<float>(m) : tid == 2 ? static_cast<float>(L) : 0.f;
+}
+
 // Position held in register slot e by thread t of a 128-thread row group, for
 // the three passes of the specialised n = 4096 kernel (see bq_fast4096.cu).
 __device__ __forceinline__ int pos_pass(int pass, int t, int e) {
@@ -132,14 +176,31 @@ __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
 
 }  // namespace
 
+bq_status launch_prepare_any(const float* theta, const uint8_t* quadrant, float* theta_out, bool hadamard, int m,
+                             float* table, cudaStream_t st);
+
 bq_status launch_prepare(const float* theta, int m, float* table, cudaStream_t st) {
+  return launch_prepare_any(theta, nullptr, nullptr, false, m, table, st);
+}
+
+bq_status launch_prepare_hadamard(const uint8_t* quadrant, float* theta_out, int m, float* table, cudaStream_t st) {
+  return launch_prepare_any(nullptr, quadrant, theta_out, true, m, table, st);
+}
+
+bq_status launch_prepare_any(const float* theta, const uint8_t* quadrant, float* theta_out, bool hadamard, int m,
+                             float* table, cudaStream_t st) {
   TableLayout tl = table_layout(m);
   const size_t smem = sizeof(double) * size_t(m);
   if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(k_prepare, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-      return BQ_ERR_CUDA;
+    const cudaError_t e =
+        hadamard ? cudaFuncSetAttribute(k_prepare_hadamard, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem))
+                 : cudaFuncSetAttribute(k_prepare, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+    if (e != cudaSuccess) return BQ_ERR_CUDA;
   }
-  k_prepare<<<1, 1024, smem, st>>>(theta, table, tl);
+  if (hadamard)
+    k_prepare_hadamard<<<1, 1024, smem, st>>>(quadrant, table, theta_out, tl);
+  else
+    k_prepare<<<1, 1024, smem, st>>>(theta, table, tl);
   if (m == 4096) {
     const int total = kImageLanes * (kImageCols + kImageInvCols);
     k_image4096<<<(total + 255) / 256, 256, 0, st>>>(table, tl);

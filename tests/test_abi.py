@@ -208,3 +208,11 @@ def test_w2a16_rejects_bad_arguments(lib):
                                None, None) == _lib.BQ_ERR_WORKSPACE
     assert lib.bq_w2a16_linear(ctypes.byref(layer), FAKE, 0, 4, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, 0, FAKE + 16,
                                1 << 20, None, None) == bad
+
+
+def test_hadamard_preset_rejects_bad_arguments(lib):
+    assert lib.bq_precompute_hadamard(4095, None, FAKE, None, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_hadamard(8192, None, FAKE, None, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_hadamard(4096, None, None, None, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_hadamard(4096, None, FAKE + 4, None, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_precompute_hadamard(4096, None, FAKE, FAKE + 2, None) == _lib.BQ_ERR_INVALID_ARG
