@@ -535,8 +535,11 @@ def run_gemm_bench(args, spec, rank, world, local_rank):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    ws_bytes = bq.bq_w2a16_gemm_workspace_size(tokens, n, out_f)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
     def step():
-        bq.bq_w2a16_gemm(x, codes, scale, zero, bits, group, out, status)
+        bq.bq_w2a16_gemm(x, codes, scale, zero, bits, group, out, workspace=ws, status=status)
 
     for _ in range(args.warmup):
         flush.zero_()
@@ -580,7 +583,7 @@ def run_gemm_bench(args, spec, rank, world, local_rank):
 
         def e2e_step():
             x_dev.copy_(x_pin, non_blocking=True)
-            bq.bq_w2a16_gemm(x_dev, codes, scale, zero, bits, group, out, status)
+            bq.bq_w2a16_gemm(x_dev, codes, scale, zero, bits, group, out, workspace=ws, status=status)
             o_pin.copy_(out, non_blocking=True)
 
         for _ in range(args.warmup):

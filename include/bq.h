@@ -248,22 +248,34 @@ bq_status bq_reconstruction_loss(const bq_layer* layer, const float* w, int64_t 
  * group: 64, 128 or 256 dividing n; n: a multiple of 64.
  * out: [tokens][out_features] float32 (out_t = BQ_F32) or bfloat16 (BQ_BF16,
  *   rounded to nearest-even); device.
+ * workspace: NULL, or device memory (256-byte aligned) of at least
+ *   bq_w2a16_gemm_workspace_size(tokens, n, out_features) bytes.  With few
+ *   output tiles (few tokens) the kernel splits K over more SMs and adds the
+ *   slices' float32 partial sums in a fixed order (bitwise reproducible); without
+ *   the workspace it does not split K (same results up to float32 summation
+ *   order, slower for decode-sized token counts).
  * status: NULL, or a device int32 the caller zeroes; the kernel ORs a nonzero
  *   code into it if one of its internal waits gave up after one second (the
  *   output is then incomplete).  Nothing is launched on invalid arguments;
  *   BQ_ERR_UNSUPPORTED if the driver's tensor-map encoder is unavailable. */
 bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, const uint8_t* codes,
                         const uint16_t* scale_f16, const uint16_t* zero_f16, int64_t out_features,
-                        int32_t bits, int32_t group, void* out, bq_dtype out_t, int32_t* status,
-                        void* stream);
+                        int32_t bits, int32_t group, void* out, bq_dtype out_t, void* workspace,
+                        size_t workspace_bytes, int32_t* status, void* stream);
 
-/* Bytes of workspace bq_w2a16_linear needs: the bfloat16 rotated activations. */
-size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens);
+/* Bytes of split-K workspace bq_w2a16_gemm uses for this shape on the current
+ * device (0 when K is not split). */
+size_t bq_w2a16_gemm_workspace_size(int64_t tokens, int32_t n, int64_t out_features);
+
+/* Bytes of workspace bq_w2a16_linear needs: the bfloat16 rotated activations
+ * plus the GEMM's split-K workspace. */
+size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens, int64_t out_features);
 
 /* The whole quantized layer from raw activations: x~ = Q x (bq_butterfly_fwd to
  * bfloat16 into the workspace), then bq_w2a16_gemm(x~, ...).  x: [tokens][n] of
- * dtype xt; workspace: device, 256-byte aligned, >= bq_w2a16_linear_workspace_size;
- * other arguments as for bq_w2a16_gemm. */
+ * dtype xt; workspace: device, 256-byte aligned, >= bq_w2a16_linear_workspace_size
+ * (at least the activations' bytes, else BQ_ERR_WORKSPACE); other arguments as
+ * for bq_w2a16_gemm. */
 bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int64_t tokens,
                           const uint8_t* codes, const uint16_t* scale_f16, const uint16_t* zero_f16,
                           int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,

@@ -21,6 +21,7 @@ from ._lib import (  # noqa: F401
     bq_reconstruction_loss,
     bq_reconstruction_workspace_size,
     bq_w2a16_gemm,
+    bq_w2a16_gemm_workspace_size,
     bq_w2a16_linear,
     bq_w2a16_linear_workspace_size,
     load,

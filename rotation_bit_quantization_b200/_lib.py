@@ -34,6 +34,7 @@ EXPORTED = (
     "bq_reconstruction_workspace_size",
     "bq_reconstruction_loss",
     "bq_w2a16_gemm",
+    "bq_w2a16_gemm_workspace_size",
     "bq_w2a16_linear_workspace_size",
     "bq_w2a16_linear",
     "bq_status_string",
@@ -81,8 +82,9 @@ def load(path: str | None = None):
         "bq_angle_sgd": (i32, [vp, vp, i64, ctypes.c_float, vp]),
         "bq_reconstruction_workspace_size": (sz, [i32, i64, i64, i32, i32]),
         "bq_reconstruction_loss": (i32, [lp, vp, i64, vp, i64, i32, i32, vp, vp, vp, sz, vp]),
-        "bq_w2a16_gemm": (i32, [vp, i64, i32, vp, vp, vp, i64, i32, i32, vp, i32, vp, vp]),
-        "bq_w2a16_linear_workspace_size": (sz, [i32, i64]),
+        "bq_w2a16_gemm": (i32, [vp, i64, i32, vp, vp, vp, i64, i32, i32, vp, i32, vp, sz, vp, vp]),
+        "bq_w2a16_gemm_workspace_size": (sz, [i64, i32, i64]),
+        "bq_w2a16_linear_workspace_size": (sz, [i32, i64, i64]),
         "bq_w2a16_linear": (i32, [lp, vp, i32, i64, vp, vp, vp, i64, i32, i32, vp, i32, vp, sz, vp, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
     }
@@ -303,23 +305,31 @@ def bq_reconstruction_loss(layer: Layer, w, x, bits: int, group: int, dtheta, lo
     return dtheta, loss
 
 
-def bq_w2a16_gemm(x, codes, scale, zero, bits: int, group: int, out, status=None, stream=None):
+def bq_w2a16_gemm_workspace_size(tokens: int, n: int, out_features: int) -> int:
+    return int(load().bq_w2a16_gemm_workspace_size(tokens, n, out_features))
+
+
+def bq_w2a16_gemm(x, codes, scale, zero, bits: int, group: int, out, workspace=None, status=None, stream=None):
     """x: bfloat16 (tokens, n) rotated activations; codes/scale/zero: the packed weights of
     bq_weight_rotate_pack for (out_features, n); out: float32 or bfloat16 (tokens, out_features);
+    workspace: None or a uint8 CUDA tensor of bq_w2a16_gemm_workspace_size bytes (split K);
     status: None or an int32 CUDA tensor of one element (zeroed by the caller)."""
     for t, nm in ((x, "x"), (codes, "codes"), (scale, "scale"), (zero, "zero"), (out, "out")):
         _dev(t, nm)
-    if status is not None:
-        _dev(status, "status")
+    for t, nm in ((workspace, "workspace"), (status, "status")):
+        if t is not None:
+            _dev(t, nm)
     tokens, n = x.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("bq_w2a16_gemm",
            load().bq_w2a16_gemm(_ptr(x), tokens, n, _ptr(codes), _ptr(scale), _ptr(zero), codes.shape[0], bits,
-                                group, _ptr(out), _dtype_code(out), _ptr(status), _stream(stream)))
+                                group, _ptr(out), _dtype_code(out), _ptr(workspace), ws_bytes, _ptr(status),
+                                _stream(stream)))
     return out
 
 
-def bq_w2a16_linear_workspace_size(n: int, tokens: int) -> int:
-    return int(load().bq_w2a16_linear_workspace_size(n, tokens))
+def bq_w2a16_linear_workspace_size(n: int, tokens: int, out_features: int) -> int:
+    return int(load().bq_w2a16_linear_workspace_size(n, tokens, out_features))
 
 
 def bq_w2a16_linear(layer: Layer, x, codes, scale, zero, bits: int, group: int, out, workspace, status=None,

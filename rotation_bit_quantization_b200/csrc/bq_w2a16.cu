@@ -18,18 +18,24 @@
 //
 // One CTA per SM, persistent over tiles of 128 output features x 256 tokens, K in
 // stages of 64:
-//  * warp 12 (one thread) loads each stage's activation tile (256 tokens x 64,
-//    128-byte swizzled, the layout the MMA reads) and the packed codes of the
-//    tile's 128 features with the tensor memory accelerator into a 5-deep ring,
-//    completing on "full_x";
-//  * warps 4-11 (two threads per feature, 32 of its 64 codes each) expand a
-//    stage's codes to bfloat16 (q - z) * s in registers and store them with
-//    tcgen05.st into an 8-deep ring of A operands in tensor memory (lane =
-//    feature, 32 columns of bf16 pairs), then arrive on "full_w";
-//  * warp 13 (one thread) issues tcgen05.mma (bf16 x bf16 -> fp32, M = 128,
-//    N = 256, K = 16), so each dequantized weight feeds 256 tokens; commits free
-//    the activation stage and the weight stage, and one per tile hands the
-//    accumulator (256 columns) to the epilogue;
+//  * a 5-deep ring of stages, each an activation tile (up to 256 tokens x 64,
+//    128-byte swizzled, the layout the MMA reads) with the packed codes of the
+//    tile's 128 features in shared memory, and the A operand they become in
+//    tensor memory (lane = feature, 32 columns of bf16 pairs); one "empty"
+//    barrier per stage, committed by the MMAs, frees both halves;
+//  * warp 12 (one thread) waits for a stage to be empty and loads it with the
+//    tensor memory accelerator, completing on "full_x";
+//  * warps 4-11 (two threads per feature, 32 of its 64 codes each) wait for
+//    full_x, expand the codes to bfloat16 (q - z) * s in registers, store them
+//    with tcgen05.st into the stage's A slot and arrive on "full_w".  full_x of
+//    a round completes only after the copy was issued, which was after the
+//    stage's previous MMAs had committed, so the A slot is free by then;
+//  * warp 13 (one thread) waits for full_w alone (every dequantizing thread
+//    acquired full_x before arriving, so the activation tile is ordered before
+//    the MMAs too) and issues tcgen05.mma (bf16 x bf16 -> fp32, M = 128,
+//    N = up to 256, K = 16), so each dequantized weight feeds up to 256 tokens;
+//    one commit per stage frees it, one per work unit hands the accumulator
+//    (256 columns) to the epilogue;
 //  * warps 0-3 read the accumulator (lane = feature), transpose 32 x 32 blocks
 //    through shared memory so that each thread holds one token's 32 consecutive
 //    features, and store them.
@@ -59,10 +65,10 @@ namespace bq {
 namespace {
 
 constexpr int kBM = 128;                                 // output features per tile (the MMA's M)
-constexpr int kBN = 256;                                 // tokens per tile (the MMA's N)
+constexpr int kBN = 256;                                 // largest token tile (the MMA's N; smaller for few tokens)
 constexpr int kBK = 64;                                  // K per stage: one 128-byte row of bf16
-constexpr int kStages = 5;                               // activation + code ring (shared memory)
-constexpr int kWStages = 8;                              // weight ring (tensor memory)
+constexpr int kStages = 5;                               // ring depth: activations + codes (shared memory)
+                                                         // and the weights they pair with (tensor memory)
 constexpr int kXBytes = kBN * kBK * 2;                   // 32 KiB activation tile
 constexpr int kCodeBytes = kBM * kBK / 2;                // packed codes of a stage (4-bit size), 4 KiB
 constexpr int kStageBytes = kXBytes + kCodeBytes;        // 36 KiB, a multiple of 1024
@@ -72,18 +78,20 @@ constexpr int kSmemBytes = kBarOff + 320 + 1024;         // barriers, then slack
 constexpr int kEpiWarps = 4, kDeqWarps = 8, kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * 14;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColW = 256;                          // weight ring: stage w at columns 256 + 32 w
+constexpr uint32_t kColW = 256;                          // weight ring: stage s at columns 256 + 32 s
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // barrier block (byte offsets from kBarOff)
-constexpr int kFullX = 0, kEmptyX = 64, kFullW = 128, kEmptyW = 192, kAccFull = 256, kAccEmpty = 264,
-              kDrain = 272, kTmemSlot = 280, kAbort = 284;
+constexpr int kFullX = 0, kFullW = 64, kEmpty = 128, kAccFull = 192, kAccEmpty = 200, kDrain = 208,
+              kTmemSlot = 216, kAbort = 220;
 
 // status bits: which wait ran out
 constexpr int kStTma = 1, kStDeq = 2, kStMmaOperands = 4, kStMmaAcc = 8, kStEpi = 16, kStDrain = 32;
 
-// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, N = 256, M = 128
-constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(kBN >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+// instruction descriptor: fp32 accumulate, bf16 A and B, both K-major, M = 128, N = ntok
+__host__ __device__ constexpr uint32_t make_idesc(int ntok) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (uint32_t(ntok >> 3) << 17) | (uint32_t(kBM >> 4) << 24);
+}
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -166,11 +174,11 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t addr) {
 }
 
 // D (tensor memory) (+)= A (tensor memory, 128 lanes x 16 bf16) x B (shared memory, descriptor)
-__device__ __forceinline__ void umma_bf16_ta(uint32_t d, uint32_t a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d, uint32_t a, uint64_t b, uint32_t idesc, uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}"
-      ::"r"(d), "r"(a), "l"(b), "r"(kIdesc), "r"(accumulate)
+      ::"r"(d), "r"(a), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
@@ -361,11 +369,33 @@ struct GemmArgs {
   const uint16_t* scale;  // [out_features][n / group] fp16 bits
   const uint16_t* zero;
   void* out;              // [tokens][out_features]
+  float* part;            // split-K partial sums [f_tile][t_tile][ksplit][ntok][128] (ksplit > 1)
   int tokens, out_features, n, group;
-  int t_tiles, tiles;     // token tiles of 128, and all tiles (token tile fastest)
+  int ntok, npad;         // tokens per tile (the MMA's N, a multiple of 16) and its 32-rounded width
+  uint32_t idesc;
+  int kblocks, ksplit;    // K stages of 64, and the slices K is cut into
+  int t_tiles, units;     // token tiles; work units = t_tiles x ksplit x feature tiles
   int vec;                // epilogue may use 16-byte stores
   int32_t* status;
 };
+
+// Work unit u: token tile fastest, then K slice, then feature tile.
+struct Unit {
+  int t_tile, ks, f_tile, t0, o0, kb0, kb1;
+};
+
+__device__ __forceinline__ Unit unit_of(const GemmArgs& a, int u) {
+  Unit r;
+  r.t_tile = u % a.t_tiles;
+  const int rest = u / a.t_tiles;
+  r.ks = rest % a.ksplit;
+  r.f_tile = rest / a.ksplit;
+  r.t0 = r.t_tile * a.ntok;
+  r.o0 = r.f_tile * kBM;
+  r.kb0 = r.ks * a.kblocks / a.ksplit;
+  r.kb1 = (r.ks + 1) * a.kblocks / a.ksplit;
+  return r;
+}
 
 template <int BITS, bool BF16>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -379,18 +409,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kBarOff + kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kBarOff + kTmemSlot);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kblocks = args.n / kBK;
   constexpr uint32_t kCodeRow = kBK * BITS / 8;             // packed bytes of one feature per stage
-  constexpr uint32_t kTx = kXBytes + kBM * kCodeRow;        // bytes a stage's copies deliver
+  const uint32_t tx = static_cast<uint32_t>(args.ntok) * (kBK * 2) + kBM * kCodeRow;  // bytes of a stage's copies
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(bars + kFullX + 8 * s, 1);
-      mbar_init(bars + kEmptyX + 8 * s, 1);
-    }
-    for (int s = 0; s < kWStages; ++s) {
       mbar_init(bars + kFullW + 8 * s, 32 * kDeqWarps);
-      mbar_init(bars + kEmptyW + 8 * s, 1);
+      mbar_init(bars + kEmpty + 8 * s, 1);
     }
     mbar_init(bars + kAccFull, 1);
     mbar_init(bars + kAccEmpty, 32 * kEpiWarps);
@@ -416,22 +442,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kTmaWarp) {
     // ---------------------------------------------------------------- loads
     if (lane == 0) {
-      uint32_t it = 0, issued = 0, last_parity = 0;
+      uint32_t s = 0, par = 0, issued = 0, last_parity = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
-        const int t0 = (tile % args.t_tiles) * kBN, o0 = (tile / args.t_tiles) * kBM;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-          if (!wait_bar(bars + kEmptyX + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
+      for (int u = blockIdx.x; ok && u < args.units; u += gridDim.x) {
+        const Unit U = unit_of(args, u);
+        for (int kb = U.kb0; kb < U.kb1; ++kb) {
+          if (!wait_bar(bars + kEmpty + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
             ok = false;
             break;
           }
           const uint32_t st = base + s * kStageBytes;
-          mbar_expect_tx(bars + kFullX + 8 * s, kTx);
-          tma_2d(st, &map_x, kb * kBK, t0, bars + kFullX + 8 * s);
-          tma_2d(st + kXBytes, &map_codes, kb * kCodeRow, o0, bars + kFullX + 8 * s);
+          mbar_expect_tx(bars + kFullX + 8 * s, tx);
+          tma_2d(st, &map_x, kb * kBK, U.t0, bars + kFullX + 8 * s);
+          tma_2d(st + kXBytes, &map_codes, kb * kCodeRow, U.o0, bars + kFullX + 8 * s);
           issued |= 1u << s;
           last_parity = (last_parity & ~(1u << s)) | (par << s);
+          if (++s == kStages) {
+            s = 0;
+            par ^= 1u;
+          }
         }
       }
       // copies still in flight land before the CTA exits
@@ -442,28 +471,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kMmaWarp) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      uint32_t it = 0;
+      uint32_t s = 0, par = 0;
+      const uint32_t idesc = args.idesc;
       bool ok = true;
       int i = 0;
-      for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x, ++i) {
-        // one accumulator set: tile i starts once the epilogue has read tile i - 1
+      for (int u = blockIdx.x; ok && u < args.units; u += gridDim.x, ++i) {
+        const Unit U = unit_of(args, u);
+        // one accumulator: unit i starts once the epilogue has read unit i - 1
         if (!wait_bar(bars + kAccEmpty, (i & 1) ^ 1, abort_flag, args.status, kStMmaAcc)) break;
         tc_fence_after();
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
-          const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-          const uint32_t w = it % kWStages, wpar = (it / kWStages) & 1u;
-          if (!wait_bar(bars + kFullX + 8 * s, par, abort_flag, args.status, kStMmaOperands) ||
-              !wait_bar(bars + kFullW + 8 * w, wpar, abort_flag, args.status, kStMmaOperands)) {
+        uint32_t acc = 0;
+        for (int kb = U.kb0; kb < U.kb1; ++kb) {
+          if (!wait_bar(bars + kFullW + 8 * s, par, abort_flag, args.status, kStMmaOperands)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t x = base + s * kStageBytes;
-          const uint32_t a = tmem + kColW + 32u * w;
+          const uint64_t xd = sw128_desc(base + s * kStageBytes);
+          const uint32_t a = tmem + kColW + 32u * s;
 #pragma unroll
-          for (int j = 0; j < kBK / 16; ++j) umma_bf16_ta(tmem, a + 8 * j, sw128_desc(x + 32 * j), (kb | j) != 0);
-          umma_commit(bars + kEmptyX + 8 * s);
-          umma_commit(bars + kEmptyW + 8 * w);
+          for (int j = 0; j < kBK / 16; ++j) {
+            umma_bf16_ta(tmem, a + 8 * j, xd + 2 * j, idesc, acc);  // +32 bytes of K per step
+            acc = 1;
+          }
+          umma_commit(bars + kEmpty + 8 * s);
+          if (++s == kStages) {
+            s = 0;
+            par ^= 1u;
+          }
         }
         if (ok) umma_commit(bars + kAccFull);
       }
@@ -481,77 +516,110 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t col = 16u * kh;
     const int gpr = args.n / args.group, kb_per_group = args.group / kBK;
     Expand<BITS> ex;
-    float s_next = 0.f, z_next = 0.f;
-    auto load_sz = [&](int tile, int g) {
-      s_next = 0.f;
-      z_next = 0.f;
-      if (tile < args.tiles) {
-        const long long o = static_cast<long long>(tile / args.t_tiles) * kBM + f;
-        if (o < args.out_features) {
-          s_next = __half2float(__ushort_as_half(__ldg(args.scale + o * gpr + g)));
-          z_next = __half2float(__ushort_as_half(__ldg(args.zero + o * gpr + g)));
-        }
+    // (s, z) of the next group this thread expands: units in CTA order, each from
+    // the group of its first stage to the group of its last; the unit's geometry
+    // is computed once per unit
+    int pu = blockIdx.x, pg = 0, pg_last = -1;
+    long long po = 0;
+    auto enter = [&]() {
+      if (pu < args.units) {
+        const Unit P = unit_of(args, pu);
+        pg = P.kb0 / kb_per_group;
+        pg_last = (P.kb1 - 1) / kb_per_group;
+        po = static_cast<long long>(P.o0) + f;
       }
     };
-    load_sz(blockIdx.x, 0);
-    uint32_t it = 0;
+    float s_next = 0.f, z_next = 0.f;
+    auto load_sz = [&]() {
+      s_next = 0.f;
+      z_next = 0.f;
+      if (pu < args.units && po < args.out_features) {
+        s_next = __half2float(__ushort_as_half(__ldg(args.scale + po * gpr + pg)));
+        z_next = __half2float(__ushort_as_half(__ldg(args.zero + po * gpr + pg)));
+      }
+    };
+    auto advance = [&]() {
+      if (pg < pg_last) {
+        ++pg;
+      } else {
+        pu += gridDim.x;
+        enter();
+      }
+    };
+    enter();
+    load_sz();
+    uint32_t s = 0, par = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < args.tiles; tile += gridDim.x) {
-      for (int kb = 0; kb < kblocks; ++kb, ++it) {
-        if (kb % kb_per_group == 0) {
+    for (int u = blockIdx.x; ok && u < args.units; u += gridDim.x) {
+      const Unit U = unit_of(args, u);
+      for (int kb = U.kb0; kb < U.kb1; ++kb) {
+        if (kb == U.kb0 || (kb & (kb_per_group - 1)) == 0) {  // kb_per_group is 1, 2 or 4
           ex.set(s_next, z_next);
-          const int g = kb / kb_per_group;
-          if (g + 1 < gpr) load_sz(tile, g + 1);
-          else load_sz(tile + gridDim.x, 0);
+          advance();
+          load_sz();
         }
-        const uint32_t s = it % kStages, par = (it / kStages) & 1u;
-        const uint32_t w = it % kWStages, wpar = (it / kWStages) & 1u;
+        // full_x: the stage's copies landed, so its previous MMAs (which read the A
+        // slot too) have committed
         if (!wait_bar(bars + kFullX + 8 * s, par, abort_flag, args.status, kStDeq)) {
           ok = false;
           break;
         }
+        tc_fence_after();
         uint32_t v[16];
         ex.run(base + s * kStageBytes + kXBytes + f * kCodeRow + kh * (kCodeRow / 2), v);
-        if (!wait_bar(bars + kEmptyW + 8 * w, wpar ^ 1u, abort_flag, args.status, kStDeq)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        tmem_st16(tmem + lane_base + kColW + 32u * w + col, v);
+        tmem_st16(tmem + lane_base + kColW + 32u * s + col, v);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bars + kFullW + 8 * w);
+        mbar_arrive(bars + kFullW + 8 * s);
+        if (++s == kStages) {
+          s = 0;
+          par ^= 1u;
+        }
       }
     }
   } else {
     // ---------------------------------------------------------------- epilogue
     float* buf = reinterpret_cast<float*>(gbase + kEpiOff) + warp * (32 * 33);
+    const int nchunks = args.npad / 32;
     int i = 0;
-    for (int tile = blockIdx.x; tile < args.tiles; tile += gridDim.x, ++i) {
+    for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++i) {
       if (!wait_bar(bars + kAccFull, i & 1, abort_flag, args.status, kStEpi)) break;
       tc_fence_after();
-      const int t0 = (tile % args.t_tiles) * kBN, o0 = (tile / args.t_tiles) * kBM;
-      {
+      const Unit U = unit_of(args, u);
+      // split K: this slice's partial sums, rows of 128 features per token of the tile
+      float* slice = args.ksplit > 1 ? args.part + ((static_cast<size_t>(U.f_tile) * args.t_tiles + U.t_tile) *
+                                                        args.ksplit + U.ks) * args.ntok * kBM
+                                     : nullptr;
 #pragma unroll 1
-        for (int q = 0; q < kBN / 32; ++q) {
-          uint32_t r[32];
-          tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32u * q, r);
-          tmem_wait_ld(r);
-          // r[j] = D[feature 32 warp + lane][token 32 q + j]: transpose so that this
-          // thread holds token 32 q + lane's 32 features
+      for (int q = 0; q < nchunks; ++q) {
+        uint32_t r[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32u * q, r);
+        tmem_wait_ld(r);
+        if (q == nchunks - 1) {  // the accumulator is free once its last columns are read
+          tc_fence_before();
+          mbar_arrive(bars + kAccEmpty);
+        }
+        // r[j] = D[feature 32 warp + lane][token 32 q + j]: transpose so that this
+        // thread holds token 32 q + lane's 32 features
 #pragma unroll
-          for (int j = 0; j < 32; ++j) buf[j * 33 + lane] = __uint_as_float(r[j]);
-          __syncwarp();
-          float c[32];
+        for (int j = 0; j < 32; ++j) buf[j * 33 + lane] = __uint_as_float(r[j]);
+        __syncwarp();
+        float c[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) c[j] = buf[lane * 33 + j];
-          __syncwarp();
-          const long long t = t0 + 32 * q + lane;
-          if (t < args.tokens) store_row32<BF16>(args.out, t, args.out_features, o0 + 32 * warp, args.vec != 0, c);
+        for (int j = 0; j < 32; ++j) c[j] = buf[lane * 33 + j];
+        __syncwarp();
+        const int tt = 32 * q + lane;  // token within the tile
+        if (tt < args.ntok && U.t0 + tt < args.tokens) {
+          if (slice) {
+            float4* d4 = reinterpret_cast<float4*>(slice + static_cast<size_t>(tt) * kBM + 32 * warp);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) d4[k] = make_float4(c[4 * k], c[4 * k + 1], c[4 * k + 2], c[4 * k + 3]);
+          } else {
+            store_row32<BF16>(args.out, static_cast<long long>(U.t0) + tt, args.out_features, U.o0 + 32 * warp,
+                              args.vec != 0, c);
+          }
         }
       }
-      tc_fence_before();
-      mbar_arrive(bars + kAccEmpty);
     }
   }
 
@@ -560,6 +628,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kMmaWarp) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// Split K: out[t][o] = sum over the slices, in slice order, of the partial sums.
+// One thread per output element, features fastest (coalesced reads and writes).
+template <bool BF16>
+__global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__ part, void* __restrict__ out,
+                                                       int tokens, int out_features, int ntok, int t_tiles,
+                                                       int ksplit) {
+  const long long total = static_cast<long long>(tokens) * out_features;
+  for (long long e = blockIdx.x * 256LL + threadIdx.x; e < total; e += static_cast<long long>(gridDim.x) * 256) {
+    const int t = static_cast<int>(e / out_features), o = static_cast<int>(e % out_features);
+    const int t_tile = t / ntok, f_tile = o / kBM;
+    const float* p = part + ((static_cast<size_t>(f_tile) * t_tiles + t_tile) * ksplit * ntok + (t % ntok)) * kBM +
+                     (o % kBM);
+    float v = 0.f;
+    for (int k = 0; k < ksplit; ++k) v += __ldg(p + static_cast<size_t>(k) * ntok * kBM);
+    if (BF16)
+      static_cast<__nv_bfloat16*>(out)[e] = __float2bfloat16_rn(v);
+    else
+      static_cast<float*>(out)[e] = v;
   }
 }
 
@@ -593,15 +682,51 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* ptr, uint
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int BITS, bool BF16>
-bq_status run_gemm(const CUtensorMap& mx, const CUtensorMap& mc, const GemmArgs& a, cudaStream_t st) {
+bq_status run_gemm(const CUtensorMap& mx, const CUtensorMap& mc, const GemmArgs& a, int grid, cudaStream_t st) {
   auto kern = k_w2a16<BITS, BF16>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) != cudaSuccess)
     return BQ_ERR_CUDA;
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int grid = a.tiles < sms ? a.tiles : sms;
   kern<<<grid, kThreads, kSmemBytes, st>>>(mx, mc, a);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms > 0 ? sms : 148;
+}
+
+// The launch shape: token tile (the MMA's N), tiles, and the K split that gives at
+// least two work units per SM when there are few tiles (at least 4 K stages each).
+struct Plan {
+  int ntok, npad, t_tiles, f_tiles, kblocks, ksplit;
+  size_t part_bytes;
+};
+
+Plan plan_of(long long tokens, int n, long long out_features, int sms) {
+  Plan p;
+  p.ntok = tokens >= kBN ? kBN : static_cast<int>((tokens + 15) / 16 * 16);
+  if (p.ntok < 16) p.ntok = 16;
+  p.npad = (p.ntok + 31) / 32 * 32;
+  p.t_tiles = static_cast<int>((tokens + p.ntok - 1) / p.ntok);
+  p.f_tiles = static_cast<int>((out_features + kBM - 1) / kBM);
+  p.kblocks = n / kBK;
+  const long long tiles = static_cast<long long>(p.t_tiles) * p.f_tiles;
+  long long k = 1;
+  if (tiles < sms) {
+    k = (2LL * sms + tiles - 1) / tiles;
+    const long long kmax = p.kblocks / 4 > 0 ? p.kblocks / 4 : 1;
+    if (k > kmax) k = kmax;
+  }
+  p.ksplit = static_cast<int>(k);
+  p.part_bytes = p.ksplit > 1 ? static_cast<size_t>(tiles) * p.ksplit * kBM * p.ntok * sizeof(float) : 0;
+  return p;
+}
+
+bool valid_gemm_shape(long long tokens, int n, long long out_features, int bits, int group) {
+  if (tokens < 0 || out_features < 0 || n <= 0 || n % kBK != 0 || (bits != 2 && bits != 4)) return false;
+  if ((group != 64 && group != 128 && group != 256) || n % group != 0) return false;
+  return true;
 }
 
 }  // namespace
@@ -609,20 +734,35 @@ bq_status run_gemm(const CUtensorMap& mx, const CUtensorMap& mc, const GemmArgs&
 
 using namespace bq;
 
+extern "C" size_t bq_w2a16_gemm_workspace_size(int64_t tokens, int32_t n, int64_t out_features) {
+  if (tokens <= 0 || out_features <= 0 || n <= 0 || n % kBK != 0) return 0;
+  const Plan p = plan_of(tokens, n, out_features, sm_count());
+  return p.part_bytes;
+}
+
 extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, const uint8_t* codes,
                                    const uint16_t* scale_f16, const uint16_t* zero_f16, int64_t out_features,
-                                   int32_t bits, int32_t group, void* out, bq_dtype out_t, int32_t* status,
-                                   void* stream) {
-  if (tokens < 0 || out_features < 0 || n <= 0 || n % kBK != 0 || (bits != 2 && bits != 4)) return BQ_ERR_INVALID_ARG;
-  if ((group != 64 && group != 128 && group != 256) || n % group != 0) return BQ_ERR_INVALID_ARG;
+                                   int32_t bits, int32_t group, void* out, bq_dtype out_t, void* workspace,
+                                   size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!valid_gemm_shape(tokens, n, out_features, bits, group)) return BQ_ERR_INVALID_ARG;
   if (out_t != BQ_F32 && out_t != BQ_BF16) return BQ_ERR_INVALID_ARG;
   if (tokens > 0x7fffffffLL || out_features > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
   if (tokens == 0 || out_features == 0) return BQ_OK;
   if (!x || !codes || !scale_f16 || !zero_f16 || !out) return BQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes)) return BQ_ERR_INVALID_ARG;
+  if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  Plan p = plan_of(tokens, n, out_features, sms);
+  // without a workspace big enough for the split-K partial sums, K is not split
+  if (p.ksplit > 1 && (!workspace || workspace_bytes < p.part_bytes)) {
+    p.ksplit = 1;
+    p.part_bytes = 0;
+  }
+  const long long units = static_cast<long long>(p.t_tiles) * p.f_tiles * p.ksplit;
+  if (units > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
   CUtensorMap mx, mc;
   if (!encode_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, static_cast<uint64_t>(n), static_cast<uint64_t>(tokens),
-                 static_cast<uint64_t>(n) * 2, kBK, kBN, CU_TENSOR_MAP_SWIZZLE_128B))
+                 static_cast<uint64_t>(n) * 2, kBK, static_cast<uint32_t>(p.ntok), CU_TENSOR_MAP_SWIZZLE_128B))
     return BQ_ERR_UNSUPPORTED;
   const uint64_t row_bytes = static_cast<uint64_t>(n) * bits / 8;
   if (!encode_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes, row_bytes, static_cast<uint64_t>(out_features), row_bytes,
@@ -632,25 +772,49 @@ extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, con
   a.scale = scale_f16;
   a.zero = zero_f16;
   a.out = out;
+  a.part = p.ksplit > 1 ? static_cast<float*>(workspace) : nullptr;
   a.tokens = static_cast<int>(tokens);
   a.out_features = static_cast<int>(out_features);
   a.n = n;
   a.group = group;
-  a.t_tiles = static_cast<int>((tokens + kBN - 1) / kBN);
-  const long long tiles = static_cast<long long>(a.t_tiles) * ((out_features + kBM - 1) / kBM);
-  if (tiles > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
-  a.tiles = static_cast<int>(tiles);
+  a.ntok = p.ntok;
+  a.npad = p.npad;
+  a.idesc = make_idesc(p.ntok);
+  a.kblocks = p.kblocks;
+  a.ksplit = p.ksplit;
+  a.t_tiles = p.t_tiles;
+  a.units = static_cast<int>(units);
   a.vec = aligned16(out) && out_features % (out_t == BQ_BF16 ? 8 : 4) == 0;
   a.status = status;
   auto st = static_cast<cudaStream_t>(stream);
+  const int grid = units < sms ? static_cast<int>(units) : sms;
+  bq_status s;
   if (bits == 2)
-    return out_t == BQ_BF16 ? run_gemm<2, true>(mx, mc, a, st) : run_gemm<2, false>(mx, mc, a, st);
-  return out_t == BQ_BF16 ? run_gemm<4, true>(mx, mc, a, st) : run_gemm<4, false>(mx, mc, a, st);
+    s = out_t == BQ_BF16 ? run_gemm<2, true>(mx, mc, a, grid, st) : run_gemm<2, false>(mx, mc, a, grid, st);
+  else
+    s = out_t == BQ_BF16 ? run_gemm<4, true>(mx, mc, a, grid, st) : run_gemm<4, false>(mx, mc, a, grid, st);
+  if (s != BQ_OK || p.ksplit == 1) return s;
+  const long long total = tokens * out_features;
+  long long rgrid = (total + 255) / 256;
+  if (rgrid > 8LL * sms) rgrid = 8LL * sms;
+  if (out_t == BQ_BF16)
+    k_splitk_reduce<true><<<static_cast<unsigned>(rgrid), 256, 0, st>>>(a.part, out, a.tokens, a.out_features, a.ntok,
+                                                                        a.t_tiles, a.ksplit);
+  else
+    k_splitk_reduce<false><<<static_cast<unsigned>(rgrid), 256, 0, st>>>(a.part, out, a.tokens, a.out_features,
+                                                                         a.ntok, a.t_tiles, a.ksplit);
+  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-extern "C" size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens) {
-  if (n <= 0 || tokens < 0) return 0;
+namespace {
+size_t act_bytes(int32_t n, int64_t tokens) {
   return (static_cast<size_t>(tokens) * static_cast<size_t>(n) * 2 + 255) & ~static_cast<size_t>(255);
+}
+}  // namespace
+
+extern "C" size_t bq_w2a16_linear_workspace_size(int32_t n, int64_t tokens, int64_t out_features) {
+  if (n <= 0 || tokens < 0 || out_features < 0) return 0;
+  return act_bytes(n, tokens) + bq_w2a16_gemm_workspace_size(tokens, n, out_features);
 }
 
 extern "C" bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int64_t tokens,
@@ -660,9 +824,10 @@ extern "C" bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dt
   if (!layer || tokens < 0) return BQ_ERR_INVALID_ARG;
   if (tokens == 0) return BQ_OK;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
-  if (workspace_bytes < bq_w2a16_linear_workspace_size(layer->n, tokens)) return BQ_ERR_WORKSPACE;
+  const size_t xb = act_bytes(layer->n, tokens);
+  if (workspace_bytes < xb) return BQ_ERR_WORKSPACE;
   const bq_status s = bq_butterfly_fwd(layer, x, xt, workspace, BQ_BF16, tokens, stream);
   if (s != BQ_OK) return s;
   return bq_w2a16_gemm(workspace, tokens, layer->n, codes, scale_f16, zero_f16, out_features, bits, group, out, out_t,
-                       status, stream);
+                       static_cast<uint8_t*>(workspace) + xb, workspace_bytes - xb, status, stream);
 }

@@ -180,11 +180,11 @@ def test_reconstruction_rejects_bad_arguments(lib):
 
 
 def test_w2a16_rejects_bad_arguments(lib):
-    ok = (FAKE, 16, 256, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, _lib.BQ_F32, None, None)
+    ok = (FAKE, 16, 256, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, _lib.BQ_F32, None, 0, None, None)
 
     def call(**kw):
         names = ("x", "tokens", "n", "codes", "scale", "zero", "out_features", "bits", "group", "out", "out_t",
-                 "status", "stream")
+                 "ws", "ws_bytes", "status", "stream")
         args = dict(zip(names, ok))
         args.update(kw)
         return lib.bq_w2a16_gemm(*[args[k] for k in names])
@@ -201,8 +201,11 @@ def test_w2a16_rejects_bad_arguments(lib):
     assert call(tokens=-1) == bad
     assert call(tokens=0) == _lib.BQ_OK        # nothing to do, nothing launched
     assert call(out_features=0) == _lib.BQ_OK
-    assert lib.bq_w2a16_linear_workspace_size(4096, 3) == 4096 * 3 * 2
-    assert lib.bq_w2a16_linear_workspace_size(256, 1) == 512
+    assert call(ws=FAKE + 16, ws_bytes=1 << 20) == bad      # workspace not 256-byte aligned
+    assert lib.bq_w2a16_gemm_workspace_size(0, 4096, 128) == 0
+    assert lib.bq_w2a16_gemm_workspace_size(16, 4000, 128) == 0
+    assert lib.bq_w2a16_linear_workspace_size(4096, 3, 0) == 4096 * 3 * 2
+    assert lib.bq_w2a16_linear_workspace_size(256, 1, 0) == 512
     layer = _lib.BQLayer(256, 256, 1, FAKE, None)
     assert lib.bq_w2a16_linear(ctypes.byref(layer), FAKE, 0, 4, FAKE, FAKE, FAKE, 128, 2, 64, FAKE, 0, FAKE, 16,
                                None, None) == _lib.BQ_ERR_WORKSPACE

@@ -38,14 +38,18 @@ def _dev_weights(codes, s16, z16):
             torch.from_numpy(np.ascontiguousarray(z16).view(np.int16)).cuda())
 
 
-def _gemm(bq, xb, codes, s16, z16, bits, group, bf16_out):
+def _gemm(bq, xb, codes, s16, z16, bits, group, bf16_out, split=True):
     torch = H.torch()
     x = H.dev_bf16_bits(xb)
     c, s, z = _dev_weights(codes, s16, z16)
     out = torch.empty((xb.shape[0], codes.shape[0]), dtype=torch.bfloat16 if bf16_out else torch.float32,
                       device="cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    bq.bq_w2a16_gemm(x, c, s, z, bits, group, out, status)
+    ws = None
+    if split:
+        nbytes = bq.bq_w2a16_gemm_workspace_size(xb.shape[0], xb.shape[1], codes.shape[0])
+        ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device="cuda")
+    bq.bq_w2a16_gemm(x, c, s, z, bits, group, out, workspace=ws, status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     return H.host(out)
@@ -90,6 +94,28 @@ def test_gemm_matches_oracle(bq, tokens, n, out, bits, group, bf16_out):
         assert rel < 2.0 ** -16            # the typical float32 error is far inside the bound
 
 
+@pytest.mark.parametrize("tokens,out,bits,group", [(1, 11008, 2, 128), (16, 11008, 2, 128), (7, 4096, 4, 128),
+                                                  (40, 1000, 2, 64), (100, 2048, 4, 256)])
+def test_gemm_decode_sizes_split_k(bq, tokens, out, bits, group):
+    """Few tokens: K is split over the SMs and the slices are added in a fixed order;
+    the result matches the oracle, repeats bitwise, and equals the unsplit kernel to
+    float32 summation order."""
+    n = 4096
+    xb, codes, s16, z16 = _inputs(tokens + out + 3 * bits, tokens, n, out, bits, group)
+    torch = H.torch()
+    assert bq.bq_w2a16_gemm_workspace_size(tokens, n, out) > 0
+    got = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, False), False)
+    again = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, False), False)
+    assert np.array_equal(got, again)
+    ref, sum_abs = ow.w2a16_gemm(wl.f32_from_bf16_bits(xb), codes, s16, z16, bits, group)
+    rel = _assert_close(got, ref, sum_abs, n, False)
+    assert rel < 2.0 ** -16
+    unsplit = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, False, split=False), False)
+    _assert_close(unsplit, ref, sum_abs, n, False)
+    bf = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, True), True)
+    _assert_close(bf, ref, sum_abs, n, True)
+
+
 def test_gemm_full_layer_sampled_tokens_and_determinism(bq):
     """The LLaMA-2-7B MLP shape (2048 x 4096 activations, 11008 x 4096 INT2 g128
     weights, 688 tiles, several per CTA): sampled tokens against the oracle, and two
@@ -123,14 +149,15 @@ def test_linear_is_forward_then_gemm_and_matches_oracle(bq):
     layer = bq.Layer(H.dev_f32(theta))
     xd = H.dev_f32(x)
     c, s, z = _dev_weights(codes, s16, z16)
-    ws = torch.empty(bq.bq_w2a16_linear_workspace_size(m, tokens), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(bq.bq_w2a16_linear_workspace_size(m, tokens, out), dtype=torch.uint8, device="cuda")
     y = torch.empty((tokens, out), dtype=torch.float32, device="cuda")
     bq.bq_w2a16_linear(layer, xd, c, s, z, bits, group, y, ws)
     # the same two steps called separately
     xt = torch.empty((tokens, m), dtype=torch.bfloat16, device="cuda")
     bq.bq_butterfly_fwd(layer, xd, xt)
     y2 = torch.empty_like(y)
-    bq.bq_w2a16_gemm(xt, c, s, z, bits, group, y2)
+    gws = torch.empty(max(bq.bq_w2a16_gemm_workspace_size(tokens, m, out), 256), dtype=torch.uint8, device="cuda")
+    bq.bq_w2a16_gemm(xt, c, s, z, bits, group, y2, workspace=gws)
     torch.cuda.synchronize()
     assert torch.equal(y, y2)
     # oracle: Q x in float64 rounded to bf16; the GPU's bf16 rotated activations may sit
