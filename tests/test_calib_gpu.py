@@ -172,3 +172,35 @@ def test_calibration_steps_lower_the_reconstruction_loss(bq):
         lr = 0.02 / float(dth.abs().max().item())
         bq.bq_angle_sgd(theta, dth.view(theta.shape), lr)
     assert min(losses[-3:]) < 0.9 * losses[0], losses
+
+
+def test_calibration_from_the_hadamard_preset_beats_it(bq):
+    """The method's claim on a synthetic layer: starting from the fixed Hadamard
+    rotation (QuaRot's transform, the butterfly at pi/4), gradient steps on the W2A16
+    reconstruction loss find angles with a lower loss than the Hadamard's own.  The
+    layer's weights carry a few outlier input channels that the fixed rotation spreads
+    but cannot adapt to."""
+    torch = H.torch()
+    m, out, T, bits, group = 256, 64, 128, 2, 64
+    rng = np.random.default_rng(17)
+    w = (rng.standard_normal((out, m)) * 0.02).astype(np.float32)
+    w[:, rng.choice(m, 4, replace=False)] *= 12.0
+    x = _acts(18, T, m)
+    had = bq.Layer.hadamard(m)
+    theta = had.theta.clone()
+    wd, xd = H.dev_f32(w), H.dev_f32(x)
+    ws = torch.empty(bq.bq_reconstruction_workspace_size(m, out, T, bits, group), dtype=torch.uint8, device="cuda")
+    dth = torch.empty(theta.numel(), dtype=torch.float32, device="cuda")
+    loss = torch.empty(1, dtype=torch.float32, device="cuda")
+    losses = []
+    for step in range(40):
+        layer = bq.Layer(theta)
+        bq.bq_reconstruction_loss(layer, wd, xd, bits, group, dth, loss, ws)
+        torch.cuda.synchronize()
+        losses.append(float(loss.item()))
+        lr = 0.01 / float(dth.abs().max().item())
+        bq.bq_angle_sgd(theta, dth.view(theta.shape), lr)
+    # the first loss is the Hadamard preset's (its angles are pi/4 in float32)
+    ref_loss, _ = oc.reconstruction_loss(H.host(had.theta), w, x, bits, group)
+    assert abs(losses[0] - ref_loss) <= 2e-4 * ref_loss
+    assert min(losses[-5:]) < 0.9 * losses[0], losses

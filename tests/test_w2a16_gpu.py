@@ -168,3 +168,33 @@ def test_linear_is_forward_then_gemm_and_matches_oracle(bq):
     tol = (m / 16 + 1) * 2.0 ** -23 * sum_abs + 2.0 ** -7 * sum_abs \
         + H.F32_TOL * np.linalg.norm(x, axis=1)[:, None] * w_abs[None, :]
     assert np.all(np.abs(H.host(y).astype(np.float64) - ref) <= tol)
+
+
+def test_quantized_layer_end_to_end_reproduces_the_float_layer(bq):
+    """y = W x = (W Q^T)(Q x): rotate-pack W on the GPU, then bq_w2a16_linear on the raw
+    activations.  The result equals the oracle's exact product of the same bf16 operands
+    (the bound above), and differs from the float layer W x only by the weight
+    quantization: |y - W x| <= sum_k |x~_k| s_k / 2 (each weight within half a step of
+    its code), plus the bf16 rounding of the operands."""
+    torch = H.torch()
+    m, tokens, out, bits, group = 4096, 64, 512, 4, 128
+    rng = np.random.default_rng(31)
+    theta = wl.uniform_angles(rng, m)
+    w = (rng.standard_normal((out, m)) * 0.02).astype(np.float32)
+    x = (rng.standard_normal((tokens, m)) * 0.5).astype(np.float32)
+    layer = bq.Layer(H.dev_f32(theta))
+    codes, scale, zero = bq.quant_outputs(out, m, bits, group, "cuda")
+    bq.bq_weight_rotate_pack(layer, H.dev_f32(w), bits, group, codes, scale, zero)
+    y = torch.empty((tokens, out), dtype=torch.float32, device="cuda")
+    ws = torch.empty(bq.bq_w2a16_linear_workspace_size(m, tokens, out), dtype=torch.uint8, device="cuda")
+    bq.bq_w2a16_linear(layer, H.dev_f32(x), codes, scale, zero, bits, group, y, ws)
+    torch.cuda.synchronize()
+    got = H.host(y).astype(np.float64)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    xt = ob.forward(theta, x.astype(np.float64))
+    s = H.host(scale).view(np.uint16).view(np.float16).astype(np.float64)       # (out, m/group)
+    step = np.repeat(s, group, axis=1)                                          # per weight
+    qerr = np.abs(xt) @ (step / 2).T + 2.0 ** -7 * (np.abs(xt) @ np.abs(ob.forward(theta, w.astype(np.float64))).T)
+    assert np.all(np.abs(got - exact) <= qerr * 1.05 + 1e-4)
+    # and the quantized layer is much closer to W x than a zero output would be
+    assert np.linalg.norm(got - exact) < 0.2 * np.linalg.norm(exact)
