@@ -203,6 +203,44 @@ def cpu_oracle_rate(w, rows_target_s: float, max_rows: int):
     return done / el, cores, f"{done} rows of the workload ({nchunks} chunks of {chunk}), {el:.1f} s on {cores} threads"
 
 
+def cpu_dense_rate(w, rows_sample: int):
+    """Rows/s of the materialised-Q path on the host: Q built once (the stage-wise float64
+    oracle applied to the identity, not timed), then y = X Q^T as one float64 matmul and the
+    float32-step quantizer, on a sample of rows."""
+    from oracle import butterfly as ob
+    from oracle import quant as oq
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    src = w.x if w.x is not None else w.w
+    dt = w.x_dtype if w.x is not None else w.w_dtype
+    n = w.m * w.r
+    eye = np.eye(n)
+    qt = ob.forward(w.theta, eye) if w.r == 1 else ob.kron_forward(w.theta, w.O, eye, w.m)   # row j = Q e_j
+    xs = src[:rows_sample]
+    xf = (wl.f32_from_bf16_bits(xs) if dt == "bf16" else xs).astype(np.float64)
+    t0 = time.perf_counter()
+    y = xf @ qt
+    oq.quantize_pack(y.astype(np.float32), w.bits, w.group)
+    el = time.perf_counter() - t0
+    return xs.shape[0] / el, len(os.sched_getaffinity(0)), (
+        f"{xs.shape[0]} rows, dense {n} x {n} float64 Q (built once, not timed) times the rows on the host's "
+        f"BLAS threads plus the quantizer, {el:.2f} s")
+
+
+def cpu_bwd_rate(layer: int, tokens_sample: int, m: int = 4096):
+    """Tokens/s of the float64 oracle backward (Y, dX, dtheta) on a sample of one layer's tokens."""
+    from oracle import butterfly as ob
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    w = wl.backward_layer_host(layer, tokens_sample, m)
+    x = wl.f32_from_bf16_bits(w.x).astype(np.float64)
+    t0 = time.perf_counter()
+    ob.backward(w.theta, x, w.dy.astype(np.float64))
+    el = time.perf_counter() - t0
+    return tokens_sample / el, (f"{tokens_sample} tokens of layer {layer} (stage-wise float64 numpy), {el:.1f} s; "
+                                f"the per-token rate applies to all 32 layers (an extrapolation)")
+
+
 # ----------------------------------------------------------------------------- our arm
 
 def run_ours(args, spec, rank, world, local_rank):
@@ -360,6 +398,9 @@ def run_ours(args, spec, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, cores, sample = cpu_oracle_rate(w, rows_target_s=10.0, max_rows=rows * 8)
         result["cpu_baseline"] = {"value": rate, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample}
+        rate, cores, sample = cpu_dense_rate(w, rows_sample=min(rows, 512))
+        result["cpu_baseline_dense"] = {"value": rate, "unit": "rows/s", "cores": cores, "kind": "oracle (dense Q)",
+                                        "sample": sample}
     return result
 
 
@@ -415,6 +456,52 @@ def run_bwd_bench(args, spec, rank, world, local_rank):
     traffic, traffic_kernel = recorded_traffic("bwd") if not (args.rows or args.layers) else (None, None)
     peaks, peak_src = load_peaks()
     achieved = tokens * by_tok / (ms * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers, on one layer of the workload
+    # (the whole 103 GB batch does not fit a host round trip per step): H2D of X and dY,
+    # the launch, D2H of Y, dX and dtheta
+    e2e = None
+    if not args.no_e2e:
+        x1 = x[0].cpu().pin_memory()
+        dy1 = dy[0].cpu().pin_memory()
+        y1h = torch.empty(y[0].shape, dtype=y.dtype).pin_memory()
+        dx1h = torch.empty(dx[0].shape, dtype=dx.dtype).pin_memory()
+        dth1h = torch.empty(dth[0:1].shape, dtype=dth.dtype).pin_memory()
+        x1d, dy1d = torch.empty_like(x[0:1]), torch.empty_like(dy[0:1])
+        y1d, dx1d, dth1d = torch.empty_like(y[0:1]), torch.empty_like(dx[0:1]), torch.empty_like(dth[0:1])
+        ws1 = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, 1, T), dtype=torch.uint8, device=dev)
+
+        def e2e_step():
+            x1d[0].copy_(x1, non_blocking=True)
+            dy1d[0].copy_(dy1, non_blocking=True)
+            bq.bq_butterfly_bwd(layers[:1], x1d, y1d, dy1d, dx1d, dth1d, ws1)
+            y1h.copy_(y1d[0], non_blocking=True)
+            dx1h.copy_(dx1d[0], non_blocking=True)
+            dth1h.copy_(dth1d, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_e2e = min(args.steps, 3)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": T * world / (float(te.item()) * 1e-3), "unit": "tokens/s",
+               "h2d_bytes_per_step": x1.numel() * 2 + dy1.numel() * 4,
+               "d2h_bytes_per_step": y1h.numel() * 2 + dx1h.numel() * 4 + dth1h.numel() * 4,
+               "scope": f"one layer of the workload ({T} tokens), host buffers pinned"}
+        del x1, dy1, y1h, dx1h, x1d, dy1d, y1d, dx1d
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, sample = cpu_bwd_rate(0, 256, m)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample}
     return {
         "metric": "butterfly backward tokens/s (Y, dX, dtheta), n=4096", "value": tokens * world / (ms * 1e-3),
         "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -425,7 +512,7 @@ def run_bwd_bench(args, spec, rank, world, local_rank):
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
                      "algorithmic_bytes_per_token": by_tok, "algorithmic_flops_per_token": 368640,
                      "kernel": traffic_kernel},
-        "gpu_launches": args.steps, "clocks": clocks,
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": args.steps, "clocks": clocks,
     }
 
 
@@ -483,6 +570,49 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
     by_row = 4 * n + 4 * n + 4 * (n // group)
     peaks, peak_src = load_peaks()
     achieved = rows * by_row / (ms * 1e-3) / 1e9
+    # end to end through the public API with host buffers: H2D of y, the launch, D2H of
+    # dL/dY, the per-group KL and the loss
+    e2e = None
+    if not args.no_e2e:
+        y_pin = y.cpu().pin_memory()
+        dy_pin = torch.empty(dy.shape, dtype=dy.dtype).pin_memory()
+        kl_pin = torch.empty(kl.shape, dtype=kl.dtype).pin_memory()
+        loss_pin = torch.empty(1, dtype=torch.float32).pin_memory()
+        y_dev = torch.empty_like(y)
+
+        def e2e_step():
+            y_dev.copy_(y_pin, non_blocking=True)
+            bq.bq_uniformity_loss(y_dev, bits, group, 1e-4, kl, dy, loss)
+            dy_pin.copy_(dy, non_blocking=True)
+            kl_pin.copy_(kl, non_blocking=True)
+            loss_pin.copy_(loss, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        n_e2e = min(args.steps, 5)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s",
+               "h2d_bytes_per_step": y.numel() * 4, "d2h_bytes_per_step": dy.numel() * 4 + kl.numel() * 4 + 4}
+        del y_pin, dy_pin, y_dev
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import calib as oc
+        sample = y[:512].cpu().numpy()
+        t0 = time.perf_counter()
+        oc.uniformity_loss(sample, bits, group, 1e-4)
+        el = time.perf_counter() - t0
+        cpu = {"value": sample.shape[0] / el, "unit": "rows/s", "cores": 1, "kind": "oracle",
+               "sample": f"{sample.shape[0]} rows of the batch (float64 numpy), {el:.1f} s"}
     return {
         "metric": "uniformity regulariser rows/s (per-group KL + dL/dY), n=4096 INT4 g128", "value": rows * world / (ms * 1e-3),
         "unit": "rows/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -492,7 +622,7 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
                      "algorithmic_bytes_per_row": by_row},
-        "gpu_launches": 2 * args.steps, "clocks": clocks,
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps, "clocks": clocks,
     }
 
 
