@@ -55,8 +55,13 @@ def test_fwd_inv_f32_small(bq, m, rows):
     xb = torch.empty_like(y)
     bq.bq_butterfly_inv(layer, y, xb)
     torch.cuda.synchronize()
-    H.assert_f32_close(H.host(xb), ob.inverse(theta, H.host(y).astype(np.float64)), x.astype(np.float64))
-    H.assert_f32_close(H.host(xb), x.astype(np.float64), x.astype(np.float64))
+    H.assert_f32_close(H.host(xb), x.astype(np.float64), x.astype(np.float64))   # Q^T (Q x) = x
+    # the inverse on its own seeded input against the oracle
+    ys = rng.standard_normal((rows, m)).astype(np.float32)
+    xi = torch.empty((rows, m), dtype=torch.float32, device="cuda")
+    bq.bq_butterfly_inv(layer, H.dev_f32(ys), xi)
+    torch.cuda.synchronize()
+    H.assert_f32_close(H.host(xi), ob.inverse(theta, ys.astype(np.float64)), ys.astype(np.float64))
 
 
 @pytest.mark.parametrize("m,r", [(4, 3), (16, 5), (64, 2), (256, 7), (1024, 5), (512, 8)])
@@ -93,11 +98,13 @@ def test_bf16_io(bq):
     bq.bq_butterfly_fwd(layer, xi, xi)
     torch.cuda.synchronize()
     assert torch.equal(xi.view(torch.int16), y16.view(torch.int16))
-    # inverse from bf16 back to fp32
+    # inverse from bf16 (a seeded bf16 input) to fp32
+    yb = wl.bf16_bits_from_f32(np.random.default_rng(77).standard_normal((24, 4096)).astype(np.float32))
     back = torch.empty((24, 4096), dtype=torch.float32, device="cuda")
-    bq.bq_butterfly_inv(layer, y16, back)
+    bq.bq_butterfly_inv(layer, H.dev_bf16_bits(yb), back)
     torch.cuda.synchronize()
-    H.assert_f32_close(H.host(back), ob.inverse(w.theta, H.input_f64(H.host(y16), "bf16")), xf)
+    yf = H.input_f64(yb, "bf16")
+    H.assert_f32_close(H.host(back), ob.inverse(w.theta, yf), yf)
 
 
 def test_zero_angles_is_exact_identity(bq):
@@ -140,9 +147,21 @@ def test_tiny_workload(bq):
 
 # --------------------------------------------------------------------------- quantization
 
+def identity_layer(bq, n, O_shape=None):
+    """theta = 0 (and O = I): Q = I exactly, so quantizing through it applies the
+    library's quantizer to the given float32 values themselves."""
+    m = n if O_shape is None else n // O_shape
+    L = m.bit_length() - 1
+    O = None if O_shape is None else np.eye(O_shape, dtype=np.float32)
+    return make_layer(bq, np.zeros((L, m // 2), np.float32), O)
+
+
 def check_quant(bq, layer, x_dev, x_f64, theta, bits, group, weight=False, O=None, m=None, sample=None):
-    """Bit-exact against the oracle quantizer on the GPU's float32 output; end to end
-    against the float64 oracle within one level on at most 1e-4 of the entries."""
+    """The fused codes are bitwise the library's quantizer applied to the kernel's own
+    float32 output (quantized again through the identity layer: GPU against GPU, no
+    oracle input from the device); end to end against the float64 oracle within one
+    level on at most 1e-4 of the entries.  The quantizer itself is pinned against the
+    oracle bit for bit on seeded inputs (test_quantizer_matches_oracle_bitwise)."""
     torch = H.torch()
     rows = x_dev.shape[0]
     n = x_dev.shape[1]
@@ -154,10 +173,13 @@ def check_quant(bq, layer, x_dev, x_f64, theta, bits, group, weight=False, O=Non
     idx = np.arange(rows) if sample is None else sample
     y_gpu = H.host(y32)[idx]
     c_gpu, s_gpu, z_gpu = H.host(codes)[idx], H.host(scale)[idx].view(np.uint16), H.host(zero)[idx].view(np.uint16)
-    c_ref, s_ref, z_ref = oq.quantize_pack(y_gpu, bits, group)
-    assert np.array_equal(s_gpu, s_ref), "scales differ from the oracle quantizer on identical input"
-    assert np.array_equal(z_gpu, z_ref), "zero points differ from the oracle quantizer on identical input"
-    assert np.array_equal(c_gpu, c_ref), "codes differ from the oracle quantizer on identical input"
+    ident = identity_layer(bq, n, None if O is None else O.shape[0])
+    c2, s2, z2 = bq.quant_outputs(rows, n, bits, group, "cuda")
+    bq.bq_transform_quantize(ident, y32, bits, group, c2, s2, z2)
+    torch.cuda.synchronize()
+    assert np.array_equal(s_gpu, H.host(s2)[idx].view(np.uint16)), "fused scales differ from the quantizer of the float32 output"
+    assert np.array_equal(z_gpu, H.host(z2)[idx].view(np.uint16)), "fused zero points differ from the quantizer of the float32 output"
+    assert np.array_equal(c_gpu, H.host(c2)[idx]), "fused codes differ from the quantizer of the float32 output"
     # end to end against the float64 transform
     xs = x_f64[idx]
     ref = ob.forward(theta, xs) if O is None else ob.kron_forward(theta, O, xs, m)
@@ -177,6 +199,31 @@ def test_quant_settings_small(bq, bits, group):
     x = (rng.standard_normal((19, m)) * 3).astype(np.float32)
     layer = make_layer(bq, theta)
     check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, bits, group)
+
+
+@pytest.mark.parametrize("n,r", [(4096, 1), (5120, 5), (1024, 1), (256, 1)])
+@pytest.mark.parametrize("bits,group", [(4, 128), (2, 128), (4, 64), (2, 32), (4, 256)])
+def test_quantizer_matches_oracle_bitwise(bq, n, r, bits, group):
+    """theta = 0 (and O = I) makes Q the identity exactly, so the fused kernels quantize
+    the seeded float32 input itself: codes, scales and zero points equal the oracle
+    quantizer's bit for bit (the n = 4096, n = 5120 and generic epilogues), including
+    exact ties (values on half steps) and outlier channels."""
+    torch = H.torch()
+    if n % group:
+        pytest.skip("group does not divide n")
+    rng = np.random.default_rng(n + bits * 7 + group)
+    x = (rng.standard_normal((33, n)) * 2.0).astype(np.float32)
+    x[:, rng.choice(n, 3, replace=False)] *= 40.0
+    # a few groups on an exact grid, so that many values sit on rounding ties
+    x[5, :group] = (np.arange(group) % 9 - 4).astype(np.float32) * np.float32(0.5)
+    layer = identity_layer(bq, n, None if r == 1 else r)
+    codes, scale, zero = bq.quant_outputs(33, n, bits, group, "cuda")
+    bq.bq_transform_quantize(layer, H.dev_f32(x), bits, group, codes, scale, zero)
+    torch.cuda.synchronize()
+    c_ref, s_ref, z_ref = oq.quantize_pack(x, bits, group)
+    assert np.array_equal(H.host(scale).view(np.uint16), s_ref)
+    assert np.array_equal(H.host(zero).view(np.uint16), z_ref)
+    assert np.array_equal(H.host(codes), c_ref)
 
 
 def test_quant_degenerate_groups(bq):
