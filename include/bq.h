@@ -256,8 +256,12 @@ bq_status bq_reconstruction_loss(const bq_layer* layer, const float* w, int64_t 
  *   order, slower for decode-sized token counts).
  * status: NULL, or a device int32 the caller zeroes; the kernel ORs a nonzero
  *   code into it if one of its internal waits gave up after one second (the
- *   output is then incomplete).  Nothing is launched on invalid arguments;
- *   BQ_ERR_UNSUPPORTED if the driver's tensor-map encoder is unavailable. */
+ *   output is then incomplete): 1 the copy issuer waited for a free stage,
+ *   2 a dequantizing thread for its copies, 4 the MMA issuer for its operands,
+ *   8 the MMA issuer for the accumulator, 16 the epilogue for the accumulator,
+ *   32 the final wait for copies or MMAs in flight.  Nothing is launched on
+ *   invalid arguments; BQ_ERR_UNSUPPORTED if the driver's tensor-map encoder is
+ *   unavailable. */
 bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, const uint8_t* codes,
                         const uint16_t* scale_f16, const uint16_t* zero_f16, int64_t out_features,
                         int32_t bits, int32_t group, void* out, bq_dtype out_t, void* workspace,
