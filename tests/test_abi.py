@@ -5,6 +5,8 @@ import ctypes
 import os
 import re
 
+import numpy as np
+
 import pytest
 
 from rotation_bit_quantization_b200 import _lib, build
@@ -219,3 +221,64 @@ def test_hadamard_preset_rejects_bad_arguments(lib):
     assert lib.bq_precompute_hadamard(4096, None, None, None, None) == _lib.BQ_ERR_INVALID_ARG
     assert lib.bq_precompute_hadamard(4096, None, FAKE + 4, None, None) == _lib.BQ_ERR_INVALID_ARG
     assert lib.bq_precompute_hadamard(4096, None, FAKE, FAKE + 2, None) == _lib.BQ_ERR_INVALID_ARG
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor in the host-side error-path tests (no device needed)."""
+
+    def __init__(self, shape, dtype):
+        self.shape, self.dtype = shape, dtype
+        self.is_cuda = True
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return FAKE
+
+    def numel(self):
+        return int(np.prod(self.shape))
+
+    def element_size(self):
+        return 1
+
+
+class _Stream:
+    cuda_stream = 0
+
+
+def test_binding_maps_a_failing_launch_to_an_exception(lib, monkeypatch):
+    """A launch error (a fake cudaErrorMemoryAllocation reported by the library as
+    BQ_ERR_CUDA) reaches the caller as BQError with that status and its name, and a
+    rejected argument as BQ_ERR_INVALID_ARG: the binding never swallows a status."""
+    import torch
+
+    class FakeLib:
+        def __getattr__(self, name):
+            return getattr(lib, name)
+
+        def bq_w2a16_gemm(self, *args):
+            return _lib.BQ_ERR_CUDA
+
+        def bq_uniformity_loss(self, *args):
+            return _lib.BQ_ERR_INVALID_ARG
+
+    monkeypatch.setattr(_lib, "_lib", FakeLib())
+    x = _FakeCudaTensor((16, 256), torch.bfloat16)
+    c = _FakeCudaTensor((128, 64), torch.uint8)
+    s = _FakeCudaTensor((128, 4), torch.int16)
+    out = _FakeCudaTensor((16, 128), torch.float32)
+    with pytest.raises(_lib.BQError) as e:
+        _lib.bq_w2a16_gemm(x, c, s, s, 2, 64, out, stream=_Stream())
+    assert e.value.status == _lib.BQ_ERR_CUDA and "cuda" in str(e.value).lower()
+    y = _FakeCudaTensor((4, 256), torch.float32)
+    kl = _FakeCudaTensor((4, 2), torch.float32)
+    with pytest.raises(_lib.BQError) as e:
+        _lib.bq_uniformity_loss(y, 4, 128, 1e-4, kl, stream=_Stream())
+    assert e.value.status == _lib.BQ_ERR_INVALID_ARG
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        _lib._dev(torch.zeros(4), "x")
