@@ -253,7 +253,9 @@ bq_status bq_reconstruction_loss(const bq_layer* layer, const float* w, int64_t 
  *   output tiles (few tokens) the kernel splits K over more SMs and adds the
  *   slices' float32 partial sums in a fixed order (bitwise reproducible); without
  *   the workspace it does not split K (same results up to float32 summation
- *   order, slower for decode-sized token counts).
+ *   order, slower for decode-sized token counts).  1-3 tokens (with n a multiple
+ *   of 512 and tokens * n <= 16384) run on a CUDA-core kernel instead, with the
+ *   same bf16 weights and float32 products; it needs no workspace.
  * status: NULL, or a device int32 the caller zeroes; the kernel ORs a nonzero
  *   code into it if one of its internal waits gave up after one second (the
  *   output is then incomplete): 1 the copy issuer waited for a free stage,

@@ -652,6 +652,162 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__
   }
 }
 
+// ------------------------------------------------------------------ decode path (1-3 tokens)
+//
+// With a handful of tokens each dequantized weight feeds only T products, and the
+// tensor-core kernel is bound by its MMA issue rate (four instructions per K stage of
+// 128 features whatever N is).  This kernel does the same arithmetic on the CUDA
+// cores: lane l of the block's 8 warps owns output feature 32 b + l, warp w a
+// contiguous eighth of K; the weights are the same bf16((q - z) s) values (2-bit
+// codes by the byte tables, 4-bit codes by the exact float form), each product of
+// two bf16 values is exact in float32 and is added into one of eight interleaved
+// accumulation chains per token (64 terms each for n = 4096), and the chains and the
+// eight warps' slices are added in a fixed order.  The activations are staged once
+// per block as float32 in shared memory and read by broadcast; each warp keeps the
+// codes and group parameters of four steps ahead in registers.  At about 5.7
+// instructions per weight for one token it is instruction bound (the expansion to
+// bf16 pairs and their unpacking cost 2.7 of them), ahead of the tensor-core kernel
+// up to 3 tokens.
+constexpr int kGemvMaxTokens = 3;                        // at 4 tokens both paths take the same time
+constexpr int kGemvWarps = 8;
+constexpr int kGemvSmemFloats = 16384;                   // T x n activations, at most 64 KiB
+
+template <int BITS, int T, bool BF16>
+__global__ void __launch_bounds__(32 * kGemvWarps, 2)
+    k_w2a16_gemv(const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ codes,
+                 const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, void* __restrict__ out,
+                 int n, int out_features, int group) {
+  extern __shared__ float xs[];                           // [T][n]
+  __shared__ float red[kGemvWarps][T][32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < T * n / 2; i += 32 * kGemvWarps) {
+    const uint32_t w = reinterpret_cast<const uint32_t*>(x)[i];
+    xs[2 * i] = __uint_as_float(w << 16);
+    xs[2 * i + 1] = __uint_as_float(w & 0xffff0000u);
+  }
+  __syncthreads();
+  const int o = blockIdx.x * 32 + lane;
+  const bool live = o < out_features;
+  const int kw = n / kGemvWarps, k0 = warp * kw;          // kw: a multiple of 64
+  const int steps = kw / 64;                              // 64 codes per step: inside one group (group >= 64)
+  const int gpr = n / group;
+  const uint8_t* row = codes + static_cast<size_t>(live ? o : 0) * (static_cast<size_t>(n) * BITS / 8);
+  // the codes and group parameters of step i + kPre are loaded while step i is expanded
+  constexpr int kPre = 4, kWords = BITS / 2;              // 16-byte words of codes per step
+  uint4 cr[kPre][kWords];
+  float sr[kPre], zr[kPre];
+  auto fetch = [&](int i, uint4 (&c)[kWords], float& sv, float& zv) {
+#pragma unroll
+    for (int q = 0; q < kWords; ++q) c[q] = make_uint4(0u, 0u, 0u, 0u);
+    sv = 0.f;
+    zv = 0.f;
+    if (live && i < steps) {
+      const int k = k0 + 64 * i;
+      const uint4* src = reinterpret_cast<const uint4*>(row + static_cast<size_t>(k) * BITS / 8);
+#pragma unroll
+      for (int q = 0; q < kWords; ++q) c[q] = __ldcs(src + q);
+      const size_t gi = static_cast<size_t>(o) * gpr + k / group;
+      sv = __half2float(__ushort_as_half(__ldg(scale + gi)));
+      zv = __half2float(__ushort_as_half(__ldg(zero + gi)));
+    }
+  };
+#pragma unroll
+  for (int p = 0; p < kPre; ++p) fetch(p, cr[p], sr[p], zr[p]);
+  float2 acc[T][4];
+#pragma unroll
+  for (int t = 0; t < T; ++t)
+#pragma unroll
+    for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.f, 0.f);
+  Expand<BITS> ex;
+#pragma unroll 1
+  for (int i = 0; i < steps; ++i) {
+    const int k = k0 + 64 * i;
+    ex.set(sr[0], zr[0]);
+    uint32_t wv[32];
+    if constexpr (BITS == 2) {
+      ex.t.word(cr[0][0].x, wv);
+      ex.t.word(cr[0][0].y, wv + 8);
+      ex.t.word(cr[0][0].z, wv + 16);
+      ex.t.word(cr[0][0].w, wv + 24);
+    } else {
+      const uint32_t cw[8] = {cr[0][0].x, cr[0][0].y, cr[0][0].z, cr[0][0].w,
+                              cr[0][1].x, cr[0][1].y, cr[0][1].z, cr[0][1].w};
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        ex.dq.half(cw[c], wv + 4 * c);
+        ex.dq.half(cw[c] >> 16, wv + 4 * c + 2);
+      }
+    }
+#pragma unroll
+    for (int p = 0; p + 1 < kPre; ++p) {
+#pragma unroll
+      for (int q = 0; q < kWords; ++q) cr[p][q] = cr[p + 1][q];
+      sr[p] = sr[p + 1];
+      zr[p] = zr[p + 1];
+    }
+    fetch(i + kPre, cr[kPre - 1], sr[kPre - 1], zr[kPre - 1]);
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {                      // words j, j + 1: weights of k + 2j .. k + 2j + 3
+      const float2 w0 = make_float2(__uint_as_float(wv[j] << 16), __uint_as_float(wv[j] & 0xffff0000u));
+      const float2 w1 = make_float2(__uint_as_float(wv[j + 1] << 16), __uint_as_float(wv[j + 1] & 0xffff0000u));
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        const float4 xv = *reinterpret_cast<const float4*>(xs + t * n + k + 2 * j);
+        acc[t][j & 3] = __ffma2_rn(w0, make_float2(xv.x, xv.y), acc[t][j & 3]);
+        acc[t][(j + 1) & 3] = __ffma2_rn(w1, make_float2(xv.z, xv.w), acc[t][(j + 1) & 3]);
+      }
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const float a = ((acc[t][0].x + acc[t][0].y) + (acc[t][1].x + acc[t][1].y)) +
+                    ((acc[t][2].x + acc[t][2].y) + (acc[t][3].x + acc[t][3].y));
+    red[warp][t][lane] = a;
+  }
+  __syncthreads();
+  if (warp == 0 && live) {
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      float v = red[0][t][lane];
+#pragma unroll
+      for (int w = 1; w < kGemvWarps; ++w) v += red[w][t][lane];
+      if (BF16)
+        static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(t) * out_features + o] = __float2bfloat16_rn(v);
+      else
+        static_cast<float*>(out)[static_cast<size_t>(t) * out_features + o] = v;
+    }
+  }
+}
+
+template <int BITS, bool BF16>
+bq_status run_gemv_t(const void* x, int tokens, int n, const uint8_t* codes, const uint16_t* scale,
+                     const uint16_t* zero, void* out, int out_features, int group, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((out_features + 31) / 32);
+  const size_t smem = static_cast<size_t>(tokens) * n * sizeof(float);
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+#define BQ_GEMV_CASE(T)                                                                                      \
+  case T: {                                                                                                  \
+    auto kern = k_w2a16_gemv<BITS, T, BF16>;                                                                 \
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=   \
+        cudaSuccess)                                                                                         \
+      return BQ_ERR_CUDA;                                                                                    \
+    kern<<<grid, 32 * kGemvWarps, smem, st>>>(xb, codes, scale, zero, out, n, out_features, group);          \
+    break;                                                                                                   \
+  }
+  switch (tokens) {
+    BQ_GEMV_CASE(1)
+    BQ_GEMV_CASE(2)
+    BQ_GEMV_CASE(3)
+    default: return BQ_ERR_INVALID_ARG;
+  }
+#undef BQ_GEMV_CASE
+  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
+bool gemv_applies(long long tokens, int n) {
+  return tokens >= 1 && tokens <= kGemvMaxTokens && n % (64 * kGemvWarps) == 0 && tokens * n <= kGemvSmemFloats;
+}
+
 // ------------------------------------------------------------------ host side
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -736,6 +892,7 @@ using namespace bq;
 
 extern "C" size_t bq_w2a16_gemm_workspace_size(int64_t tokens, int32_t n, int64_t out_features) {
   if (tokens <= 0 || out_features <= 0 || n <= 0 || n % kBK != 0) return 0;
+  if (gemv_applies(tokens, n)) return 0;
   const Plan p = plan_of(tokens, n, out_features, sm_count());
   return p.part_bytes;
 }
@@ -751,6 +908,15 @@ extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, con
   if (!x || !codes || !scale_f16 || !zero_f16 || !out) return BQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes)) return BQ_ERR_INVALID_ARG;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
+  if (gemv_applies(tokens, n)) {  // decode-sized: the CUDA-core kernel
+    auto st = static_cast<cudaStream_t>(stream);
+    const int t = static_cast<int>(tokens), of = static_cast<int>(out_features);
+    if (bits == 2)
+      return out_t == BQ_BF16 ? run_gemv_t<2, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
+                              : run_gemv_t<2, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
+    return out_t == BQ_BF16 ? run_gemv_t<4, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
+                            : run_gemv_t<4, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
+  }
   const int sms = sm_count();
   Plan p = plan_of(tokens, n, out_features, sms);
   // without a workspace big enough for the split-K partial sums, K is not split
