@@ -473,24 +473,31 @@ __device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long l
 // Copies this thread's share of a tensor-memory image (NCHUNK chunks of 16
 // columns, dealt round-robin to the slots) into its lane: all loads in flight
 // first (each warp load is one contiguous 512-byte run of the [column/4][lane]
-// image), then the stores.
+// image), then the stores.  Every CTA reads the same image at the same moment,
+// so each starts at a different chunk (block index mod NCHUNK): the requests in
+// flight then spread over the L2 slices instead of queueing on the same few.
+// (Sharing one L2 read per CTA pair through distributed shared memory was
+// slower: gathering 208 KB per SM that way costs more than the L2 reads saved.)
 template <int NCHUNK>
 __device__ __forceinline__ void fill_tmem(const float* image, uint32_t tb, int slot, int tau) {
   const float4* src = reinterpret_cast<const float4*>(image) + tau;  // block q of lane tau at [q * 128]
   constexpr int kMine = (NCHUNK + kSlots - 1) / kSlots;
   float4 f[kMine * 4];
+  const int rot = blockIdx.x % NCHUNK;
 #pragma unroll
   for (int i = 0; i < kMine; ++i) {
-    const int c = slot + i * kSlots;
-    if (c < NCHUNK) {
+    const int c0 = slot + i * kSlots;
+    if (c0 < NCHUNK) {
+      const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
 #pragma unroll
       for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
     }
   }
 #pragma unroll
   for (int i = 0; i < kMine; ++i) {
-    const int c = slot + i * kSlots;
-    if (c < NCHUNK) {
+    const int c0 = slot + i * kSlots;
+    if (c0 < NCHUNK) {
+      const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
       uint32_t v[16];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
