@@ -38,7 +38,8 @@
 //    (256 columns) to the epilogue;
 //  * warps 0-3 read the accumulator (lane = feature), transpose 32 x 32 blocks
 //    through shared memory so that each thread holds one token's 32 consecutive
-//    features, and store them.
+//    features, and store them; split-K partial rows ([token][128 features]) are
+//    stored straight from the accumulator's layout, one token row per warp store.
 // Dequantization is exact up to the final bfloat16 rounding.  2-bit codes: a
 // group has four possible weights, bf16((q - z) s) for q = 0..3 (the product is
 // exact in float32, one cvt.rn rounds it); their low and high bytes form two
@@ -590,34 +591,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       float* slice = args.ksplit > 1 ? args.part + ((static_cast<size_t>(U.f_tile) * args.t_tiles + U.t_tile) *
                                                         args.ksplit + U.ks) * args.ntok * kBM
                                      : nullptr;
+      // Chunk q: r[j] = D[feature 32 warp + lane][token 32 q + j].  The load of
+      // chunk q + 1 into the same registers starts as soon as r has been consumed,
+      // and the accumulator is handed back right after its last load.
+      const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+      const int tmax = min(args.ntok, args.tokens - U.t0);  // valid tokens of the tile
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base, r);
+      if (slice) {
+        // split-K partial rows [token][128 features]: each warp store writes one
+        // token's 32 features of this warp (128 contiguous bytes), no transpose
+        float* d = slice + 32 * warp + lane;
 #pragma unroll 1
-      for (int q = 0; q < nchunks; ++q) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 32u * q, r);
-        tmem_wait_ld(r);
-        if (q == nchunks - 1) {  // the accumulator is free once its last columns are read
-          tc_fence_before();
-          mbar_arrive(bars + kAccEmpty);
+        for (int q = 0; q < nchunks; ++q) {
+          tmem_wait_ld(r);
+          if (q + 1 == nchunks) {
+            tc_fence_before();
+            mbar_arrive(bars + kAccEmpty);
+          }
+          float c[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) c[j] = __uint_as_float(r[j]);
+          if (q + 1 < nchunks) tmem_ld32(tmem + lane_base + 32u * (q + 1), r);
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (32 * q + j < tmax) d[static_cast<size_t>(32 * q + j) * kBM] = c[j];
         }
-        // r[j] = D[feature 32 warp + lane][token 32 q + j]: transpose so that this
-        // thread holds token 32 q + lane's 32 features
+      } else {
+        // output rows: transposed through shared memory so that this thread holds
+        // token 32 q + lane's 32 consecutive features (16-byte stores)
+#pragma unroll 1
+        for (int q = 0; q < nchunks; ++q) {
+          tmem_wait_ld(r);
+          if (q + 1 == nchunks) {
+            tc_fence_before();
+            mbar_arrive(bars + kAccEmpty);
+          }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) buf[j * 33 + lane] = __uint_as_float(r[j]);
-        __syncwarp();
-        float c[32];
+          for (int j = 0; j < 32; ++j) buf[j * 33 + lane] = __uint_as_float(r[j]);
+          if (q + 1 < nchunks) tmem_ld32(tmem + lane_base + 32u * (q + 1), r);
+          __syncwarp();
+          float c[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) c[j] = buf[lane * 33 + j];
-        __syncwarp();
-        const int tt = 32 * q + lane;  // token within the tile
-        if (tt < args.ntok && U.t0 + tt < args.tokens) {
-          if (slice) {
-            float4* d4 = reinterpret_cast<float4*>(slice + static_cast<size_t>(tt) * kBM + 32 * warp);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) d4[k] = make_float4(c[4 * k], c[4 * k + 1], c[4 * k + 2], c[4 * k + 3]);
-          } else {
+          for (int j = 0; j < 32; ++j) c[j] = buf[lane * 33 + j];
+          __syncwarp();
+          const int tt = 32 * q + lane;  // token within the tile
+          if (tt < tmax)
             store_row32<BF16>(args.out, static_cast<long long>(U.t0) + tt, args.out_features, U.o0 + 32 * warp,
                               args.vec != 0, c);
-          }
         }
       }
     }
