@@ -40,6 +40,9 @@
 //    through shared memory so that each thread holds one token's 32 consecutive
 //    features, and store them; split-K partial rows ([token][128 features]) are
 //    stored straight from the accumulator's layout, one token row per warp store.
+//    For bfloat16 output the accumulator is first drained (rounded to bf16 pairs,
+//    six chunks parked in spare tensor-memory columns, two in registers) and
+//    handed back, so the next unit's MMAs do not wait for the transposes.
 // Dequantization is exact up to the final bfloat16 rounding.  2-bit codes: a
 // group has four possible weights, bf16((q - z) s) for q = 0..3 (the product is
 // exact in float32, one cvt.rn rounds it); their low and high bytes form two
@@ -80,6 +83,8 @@ constexpr int kEpiWarps = 4, kDeqWarps = 8, kTmaWarp = 12, kMmaWarp = 13;
 constexpr int kThreads = 32 * 14;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColW = 256;                          // weight ring: stage s at columns 256 + 32 s
+constexpr uint32_t kColSpare = kColW + 32 * kStages;    // 96 spare columns: six drained bf16 chunks
+static_assert(kColSpare + 6 * 16 <= kTmemCols, "spare tensor-memory columns");
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // barrier block (byte offsets from kBarOff)
@@ -218,6 +223,21 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]
 }
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t addr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(addr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld16(uint32_t (&r)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                 "+r"(r[15])::"memory");
+}
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -617,8 +637,72 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < 32; ++j)
             if (32 * q + j < tmax) d[static_cast<size_t>(32 * q + j) * kBM] = c[j];
         }
+      } else if (BF16) {
+        // bfloat16 rows: the accumulator is drained before anything is stored.  Each
+        // chunk is rounded to bf16 pairs at once (word k = tokens 2k, 2k + 1 of the
+        // chunk); chunks 0-5 go to the spare tensor-memory columns, chunks 6-7 stay
+        // in registers, and the accumulator is handed back to the MMAs; the
+        // transposes and stores then overlap the next unit's MMAs.
+        uint32_t keep[2][16];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < nchunks) {
+            tmem_wait_ld(r);
+            uint32_t p[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) p[k] = bf16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+            if (q + 1 < nchunks) tmem_ld32(tmem + lane_base + 32u * (q + 1), r);
+            if (q < 6) {
+              tmem_st16(tmem + lane_base + kColSpare + 16u * q, p);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) keep[q - 6][k] = p[k];
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bars + kAccEmpty);
+        tmem_wait_st();
+        // per warp [32 tokens][40 halves]: rows of 80 bytes, 16-byte aligned
+        uint16_t* b16 = reinterpret_cast<uint16_t*>(buf);
+        const int o = U.o0 + 32 * warp;  // first feature of this warp
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < nchunks) {
+            uint32_t w[16];
+            if (q < 6) {
+              tmem_ld16(tmem + lane_base + kColSpare + 16u * q, w);
+              tmem_wait_ld16(w);
+            } else {
+#pragma unroll
+              for (int k = 0; k < 16; ++k) w[k] = keep[q - 6][k];
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              b16[(2 * k) * 40 + lane] = static_cast<uint16_t>(w[k] & 0xffffu);
+              b16[(2 * k + 1) * 40 + lane] = static_cast<uint16_t>(w[k] >> 16);
+            }
+            __syncwarp();
+            const int tt = 32 * q + lane;  // token within the tile
+            if (tt < tmax) {
+              const uint16_t* src = b16 + lane * 40;
+              uint16_t* row = static_cast<uint16_t*>(args.out) +
+                              (static_cast<long long>(U.t0) + tt) * args.out_features;
+              if (args.vec != 0 && o + 32 <= args.out_features) {
+                uint4* dst = reinterpret_cast<uint4*>(row + o);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = reinterpret_cast<const uint4*>(src)[i];
+              } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                  if (o + e < args.out_features) row[o + e] = src[e];
+              }
+            }
+            __syncwarp();
+          }
+        }
       } else {
-        // output rows: transposed through shared memory so that this thread holds
+        // float32 rows: transposed through shared memory so that this thread holds
         // token 32 q + lane's 32 consecutive features (16-byte stores)
 #pragma unroll 1
         for (int q = 0; q < nchunks; ++q) {
