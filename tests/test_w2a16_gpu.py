@@ -94,6 +94,26 @@ def test_gemm_matches_oracle(bq, tokens, n, out, bits, group, bf16_out):
         assert rel < 2.0 ** -16            # the typical float32 error is far inside the bound
 
 
+@pytest.mark.parametrize("tokens,n,out,bits,group", [
+    (4, 256, 128, 2, 64),        # one 32-token chunk
+    (100, 1024, 200, 2, 128),    # 4 chunks of a 112-token tile, ragged features
+    (200, 512, 264, 4, 256),     # 7 chunks: six parked in tensor memory, one in registers
+    (257, 512, 136, 2, 64),      # a full tile (eight chunks) and a one-token tile
+    (300, 1024, 130, 4, 128),    # features not a multiple of 8: scalar stores
+])
+def test_gemm_bf16_unsplit_drained_epilogue(bq, tokens, n, out, bits, group):
+    """bfloat16 output without a K split: the epilogue drains the accumulator (bf16
+    pairs, chunks 0-5 in spare tensor-memory columns, 6-7 in registers) before the
+    transposed stores.  Each output is the float32 result rounded once, so it equals
+    the float32-output run rounded to bfloat16."""
+    xb, codes, s16, z16 = _inputs(tokens * 5 + out + bits, tokens, n, out, bits, group)
+    got = _gemm(bq, xb, codes, s16, z16, bits, group, True, split=False)
+    f32 = _gemm(bq, xb, codes, s16, z16, bits, group, False, split=False)
+    assert np.array_equal(got, wl.bf16_bits_from_f32(f32.astype(np.float32)))
+    ref, sum_abs = ow.w2a16_gemm(wl.f32_from_bf16_bits(xb), codes, s16, z16, bits, group)
+    _assert_close(_as_f64(got, True), ref, sum_abs, n, True)
+
+
 @pytest.mark.parametrize("tokens,out,bits,group", [(1, 11008, 2, 128), (16, 11008, 2, 128), (7, 4096, 4, 128),
                                                   (40, 1000, 2, 64), (100, 2048, 4, 256), (2, 1000, 4, 64),
                                                   (3, 130, 2, 256), (4, 4096, 4, 128), (1, 200, 4, 128)])
