@@ -19,7 +19,11 @@
 // [B][32] histogram in shared memory (each address has one writer, so the order
 // of the additions is fixed and results are reproducible), a group's columns are
 // added in a fixed order, and each level's logarithm is taken once and read back
-// by each lane from its own column for the gradient.
+// by each lane from its own column for the gradient.  (Two copies per lane, even
+// and odd values, measured slower: the chains of read-modify-writes are not the
+// limit.)  The loss (the mean over groups) is summed by a cluster of eight CTAs,
+// each over a fixed eighth, and added up in rank order by the first: one CTA alone
+// took about 100 us for the 2M per-group values of a 65536 x 4096 batch.
 #include <cfloat>
 
 #include "bq_rtn.cuh"
@@ -101,13 +105,14 @@ __global__ void __launch_bounds__(32 * kCalWarps) k_uniformity(const float* __re
 #pragma unroll
     for (int o = GL / 2; o > 0; o >>= 1) term += __shfl_xor_sync(0xffffffffu, term, o);
     if (live && q == 0) kl_group[g] = term;
-    // every lane gets its group's B logarithms into its own column of the histogram
+    // every lane gets its group's B logarithms, and puts their successive differences
+    // (the gradient's numerator for u in (k, k + 1)) into its own column
     float lgc[B];
 #pragma unroll
     for (int c = 0; c < B; ++c) lgc[c] = __shfl_sync(0xffffffffu, lgv[c % BPL], gi * GL + c / BPL);
     __syncwarp();
 #pragma unroll
-    for (int c = 0; c < B; ++c) hist[wl][c][lane] = lgc[c];
+    for (int c = 0; c < QMAX; ++c) hist[wl][c][lane] = lgc[c + 1] - lgc[c];
     __syncwarp();
     if (dy) {
       const float sc = gscale / p.s;
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(32 * kCalWarps) k_uniformity(const float* __re
           const float u = fmaf(v[4 * j + t], p.inv, z);
           const float uc = fminf(fmaxf(u, 0.f), qmax);
           const int k = min(static_cast<int>(uc), QMAX - 1);
-          d[t] = (u > 0.f && u < qmax) ? (hist[wl][k + 1][lane] - hist[wl][k][lane]) * sc : 0.f;
+          d[t] = (u > 0.f && u < qmax) ? hist[wl][k][lane] * sc : 0.f;
         }
         if (live) *reinterpret_cast<float4*>(dst + 4 * (GL * j + q)) = make_float4(d[0], d[1], d[2], d[3]);
       }
@@ -129,18 +134,49 @@ __global__ void __launch_bounds__(32 * kCalWarps) k_uniformity(const float* __re
   }
 }
 
-// loss = (sum of kl_group) / count, summed in a fixed order by one CTA
-__global__ void __launch_bounds__(1024) k_mean(const float* __restrict__ v, long long count, float* __restrict__ out) {
+// loss = (sum of kl_group) / count: a cluster of kMeanCtas CTAs, CTA r summing the
+// r-th of kMeanCtas equal slices (each thread a fixed strided subset in four fixed
+// partial sums, then a fixed tree), and CTA 0 adding the CTAs' totals in rank order
+// from their shared memory.  Fixed order throughout, and no memory outside the
+// cluster, so concurrent calls on other streams do not interfere.
+constexpr int kMeanCtas = 8;
+
+__global__ void __cluster_dims__(kMeanCtas, 1, 1) __launch_bounds__(1024)
+    k_mean(const float* __restrict__ v, long long count, float* __restrict__ out) {
   __shared__ double part[1024];
-  double acc = 0.0;
-  for (long long i = threadIdx.x; i < count; i += 1024) acc += static_cast<double>(v[i]);
-  part[threadIdx.x] = acc;
+  uint32_t rank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(rank));
+  const long long slice = (count + kMeanCtas - 1) / kMeanCtas;
+  const long long b0 = static_cast<long long>(rank) * slice;
+  const long long b1 = b0 + slice < count ? b0 + slice : count;
+  double acc[4] = {0.0, 0.0, 0.0, 0.0};
+  long long i = b0 + threadIdx.x;
+  for (; i + 3 * 1024 < b1; i += 4 * 1024) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) acc[k] += static_cast<double>(v[i + k * 1024]);
+  }
+  for (; i < b1; i += 1024) acc[0] += static_cast<double>(v[i]);  // the tail
+  part[threadIdx.x] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
   __syncthreads();
   for (int h = 512; h > 0; h >>= 1) {
     if (threadIdx.x < h) part[threadIdx.x] += part[threadIdx.x + h];
     __syncthreads();
   }
-  if (threadIdx.x == 0) *out = static_cast<float>(part[0] / static_cast<double>(count));
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (rank == 0 && threadIdx.x == 0) {
+    const uint32_t local = static_cast<uint32_t>(__cvta_generic_to_shared(&part[0]));
+    double total = 0.0;
+    for (uint32_t r = 0; r < kMeanCtas; ++r) {
+      uint32_t addr;
+      double t;
+      asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(addr) : "r"(local), "r"(r));
+      asm volatile("ld.shared::cluster.f64 %0, [%1];" : "=d"(t) : "r"(addr) : "memory");
+      total += t;
+    }
+    *out = static_cast<float>(total / static_cast<double>(count));
+  }
+  // the peers' totals stay in place until the first CTA has read them
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 __global__ void k_sgd(float* __restrict__ theta, const float* __restrict__ dtheta, long long count, float lr) {
@@ -194,7 +230,7 @@ extern "C" bq_status bq_uniformity_loss(const float* y, int64_t rows, int32_t n,
   bq_status s = bits == 4 ? uniformity_bits<4>(y, groups, group, eps, static_cast<float>(gscale), kl_group, dy, st)
                           : uniformity_bits<2>(y, groups, group, eps, static_cast<float>(gscale), kl_group, dy, st);
   if (s != BQ_OK || !loss) return s;
-  k_mean<<<1, 1024, 0, st>>>(kl_group, groups, loss);
+  k_mean<<<kMeanCtas, 1024, 0, st>>>(kl_group, groups, loss);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
