@@ -77,6 +77,23 @@ def test_uniformity_small_rows_and_degenerate_groups(bq):
     assert abs(loss - ref_loss) <= 2e-5 * abs(ref_loss)
 
 
+def test_uniformity_loss_mean_of_a_large_batch(bq):
+    """4097 rows x 4096 at INT4 g128 (131 104 groups, eight slices with ragged
+    tails): the loss is the mean of the returned per-group values (float64 sums
+    on both sides, so within one float32 step), repeats bitwise, and sampled rows'
+    per-group values match the oracle."""
+    rows, n, bits, group, eps = 4097, 4096, 4, 128, 1e-4
+    y = _acts(11, rows, n)
+    kl, _, loss = _run(bq, y, bits, group, eps)
+    mean = float(np.float32(kl.astype(np.float64).mean()))
+    assert abs(loss - mean) <= np.spacing(np.float32(abs(mean)))
+    kl2, _, loss2 = _run(bq, y, bits, group, eps)
+    assert loss2 == loss and np.array_equal(kl, kl2)
+    sample = np.array([0, 1, 2048, 4095, 4096])
+    _, ref_kl, _ = oc.uniformity_loss(y[sample], bits, group, eps)
+    assert np.abs(kl[sample] - ref_kl).max() <= 2e-5 * (1 + np.abs(ref_kl).max())
+
+
 def test_calibration_steps_lower_the_regulariser(bq):
     """Forward -> regulariser gradient -> backward (dtheta) -> angle step, repeated:
     the butterfly learns a rotation that spreads the outlier channels over the
