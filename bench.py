@@ -613,6 +613,7 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
         el = time.perf_counter() - t0
         cpu = {"value": sample.shape[0] / el, "unit": "rows/s", "cores": 1, "kind": "oracle",
                "sample": f"{sample.shape[0]} rows of the batch (float64 numpy), {el:.1f} s"}
+    traffic, traffic_kernel = recorded_traffic("uniformity") if not args.rows else (None, None)
     return {
         "metric": "uniformity regulariser rows/s (per-group KL + dL/dY), n=4096 INT4 g128", "value": rows * world / (ms * 1e-3),
         "unit": "rows/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
@@ -620,8 +621,8 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
         "data": "synthetic (seeded on device)", "config": {"workload": spec["label"], "rows": rows,
                                                            "l2": "input 1 GiB, larger than L2"},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
-                     "algorithmic_bytes_per_row": by_row},
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic, "peak_source": peak_src,
+                     "algorithmic_bytes_per_row": by_row, "kernel": traffic_kernel or "k_uniformity"},
         "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": 2 * args.steps, "clocks": clocks,
     }
 
