@@ -759,23 +759,12 @@ def run_gemm_bench(args, spec, rank, world, local_rank):
 
 # ----------------------------------------------------------------------------- reference arm
 
-def run_reference(args, spec):
-    w = spec["make"](0)
-    for _ in range(args.warmup):
-        cpu_oracle_rate(w, rows_target_s=1.0, max_rows=256)
-    rates = []
-    sample = cores = None
-    t0 = time.perf_counter()
-    for _ in range(args.steps):
-        rate, cores, sample = cpu_oracle_rate(w, rows_target_s=3.0, max_rows=spec["rows"])
-        rates.append(rate)
-    el = time.perf_counter() - t0
-    value = statistics.median(rates)
+def _reference_line(args, spec, metric, unit, value, el, cores, sample, config):
     return {
         "impl": "reference",
-        "metric": "butterfly fwd+quant rows/s and GB/s at n=4096 on 1 B200; % of FP32/HBM roofline",
+        "metric": metric,
         "value": value,
-        "unit": "rows/s",
+        "unit": unit,
         "n_gpus": 1,
         "steps": args.steps,
         "warmup": args.warmup,
@@ -785,11 +774,84 @@ def run_reference(args, spec):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded)",
-        "config": {"workload": spec["label"], "rows_per_gpu": spec["rows"], "n": spec["n"], "bits": spec["bits"],
-                   "group": spec["group"]},
-        "cpu_baseline": {"value": value, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "config": config,
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
+
+
+def run_reference(args, spec):
+    """The float64 oracle, as it stands, on the host cores: each step a bounded sample of
+    the workload, the metric and unit of our arm's line for that workload."""
+    kind = spec["kind"]
+    t0 = time.perf_counter()
+    if kind in ("quant", "fwd"):
+        w = spec["make"](0)
+        for _ in range(args.warmup):
+            cpu_oracle_rate(w, rows_target_s=1.0, max_rows=256)
+        rates = []
+        sample = cores = None
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            rate, cores, sample = cpu_oracle_rate(w, rows_target_s=3.0, max_rows=spec["rows"])
+            rates.append(rate)
+        el = time.perf_counter() - t0
+        return _reference_line(args, spec, "butterfly fwd+quant rows/s and GB/s at n=4096 on 1 B200; % of FP32/HBM roofline",
+                               "rows/s", statistics.median(rates), el, cores, sample,
+                               {"workload": spec["label"], "rows_per_gpu": spec["rows"], "n": spec["n"],
+                                "bits": spec["bits"], "group": spec["group"]})
+    if kind == "bwd":
+        for i in range(args.warmup):
+            cpu_bwd_rate(i, 16)
+        rates = []
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            rate, sample = cpu_bwd_rate(i % spec["layers"], 512)
+            rates.append(rate)
+        el = time.perf_counter() - t0
+        return _reference_line(args, spec, "butterfly backward tokens/s (Y, dX, dtheta), n=4096", "tokens/s",
+                               statistics.median(rates), el, 1, sample,
+                               {"workload": spec["label"], "layers": spec["layers"], "tokens_per_layer": spec["rows"]})
+    if kind == "uniformity":
+        from oracle import calib as oc
+        n, bits, group = spec["n"], spec["bits"], spec["group"]
+
+        def rows_sample(seed, rows):
+            # our arm's distribution: N(0, 0.5^2) with six outlier channels x40
+            rng = np.random.default_rng(seed)
+            y = (rng.standard_normal((rows, n)) * 0.5).astype(np.float32)
+            y[:, rng.choice(n, 6, replace=False)] *= 40.0
+            return y
+
+        for i in range(args.warmup):
+            oc.uniformity_loss(rows_sample(100 + i, 64), bits, group, 1e-4)
+        rates = []
+        t0 = time.perf_counter()
+        for i in range(args.steps):
+            y = rows_sample(i, 2048)
+            ts = time.perf_counter()
+            oc.uniformity_loss(y, bits, group, 1e-4)
+            rates.append(y.shape[0] / (time.perf_counter() - ts))
+        el = time.perf_counter() - t0
+        return _reference_line(args, spec, "uniformity regulariser rows/s (per-group KL + dL/dY), n=4096 INT4 g128",
+                               "rows/s", statistics.median(rates), el, 1,
+                               "2048 rows per step (float64 numpy), the batch's distribution",
+                               {"workload": spec["label"], "rows": spec["rows"]})
+    if kind == "gemm":
+        from rotation_bit_quantization_b200 import workloads as wl
+        xb, codes, s16, z16, bits, group = wl.w2a16_4096(256, spec["out_features"], seed=6)
+        oracle_gemm_rate(xb, codes, s16, z16, bits, group, 8)
+        rates = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            rate, _ = oracle_gemm_rate(xb, codes, s16, z16, bits, group, 256)
+            rates.append(rate / 1e12)
+        el = time.perf_counter() - t0
+        return _reference_line(args, spec, "W2A16 GEMM TFLOP/s (bf16 x INT2 g128 on tcgen05), 2048 x 4096 x 11008",
+                               "TFLOP/s", statistics.median(rates), el, 1,
+                               "256 tokens x 4096 x 11008 per step (float64 numpy, the whole weight matrix dequantized)",
+                               {"workload": spec["label"], "tokens": spec["rows"], "out_features": spec["out_features"]})
+    raise SystemExit(f"no reference arm for workload kind {kind}")
 
 
 # ----------------------------------------------------------------------------- main
@@ -828,8 +890,6 @@ def main():
             f", layers={spec['layers']}]" if spec["kind"] == "bwd" else "]")
 
     if args.impl == "reference":
-        if spec["kind"] in ("bwd", "uniformity", "gemm"):
-            raise SystemExit("--impl reference covers the transform + quantize workloads only")
         if rank != 0:
             return 0
         print(json.dumps(run_reference(args, spec)))
