@@ -30,11 +30,16 @@
  *    [2, 4096]; r in [1, 8]; n = m*r <= 16384.
  *  - Arithmetic is float32 (bf16 inputs are widened exactly; bf16 outputs are
  *    rounded to nearest even).
+ *  - Zero rows (tokens, out_features, count) launch nothing and return BQ_OK
+ *    once the other arguments are valid; the data pointers may then be NULL.
+ *    The exceptions need at least one token: bq_butterfly_bwd,
+ *    bq_butterfly_bwd_noalloc and bq_reconstruction_loss.
  *  - Errors: BQ_ERR_INVALID_ARG (bad sizes, null or misaligned pointers),
  *    BQ_ERR_UNSUPPORTED (valid request outside what this build implements),
- *    BQ_ERR_WORKSPACE (workspace too small), BQ_ERR_CUDA (a launch failed;
- *    the CUDA error is left for cudaGetLastError to report).  No entry point
- *    aborts, traps or asserts on the device.
+ *    BQ_ERR_WORKSPACE (workspace too small), BQ_ERR_CUDA (a CUDA call or a
+ *    launch failed).  The library carries its own CUDA runtime state, so its
+ *    CUDA error is read with bq_cuda_last_error, not the caller's
+ *    cudaGetLastError.  No entry point aborts, traps or asserts on the device.
  */
 #ifndef BQ_H_
 #define BQ_H_
@@ -120,9 +125,9 @@ size_t bq_butterfly_bwd_workspace_size(int32_t m, int32_t num_layers, int64_t ro
  *   and r == 1.
  * x: [num_layers][rows_per_layer][m] of type xt; y: same shape of type yt;
  * dy, dx: float32, same shape; dtheta: float32 [num_layers][log2(m)*(m/2)].
- * The token reduction is deterministic (fixed-order partial sums in
- * `workspace`, reduced by the last block of each layer); repeated calls give
- * bitwise identical dtheta.  workspace: device, >= the size queried above,
+ * rows_per_layer >= 1.  The token reduction is deterministic (fixed-order
+ * partial sums in `workspace`, reduced by the last block of each layer);
+ * repeated calls give bitwise identical dtheta.  workspace: device, >= the size queried above,
  * 16-byte aligned; its contents on entry are irrelevant. */
 bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers,
                            const void* x, bq_dtype xt, void* y, bq_dtype yt,
@@ -286,6 +291,14 @@ bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int
                           const uint8_t* codes, const uint16_t* scale_f16, const uint16_t* zero_f16,
                           int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,
                           void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
+
+/* The library's last CUDA runtime error (a cudaError_t value, 0 for none),
+ * cleared by the call: after BQ_ERR_CUDA it says which CUDA call or launch
+ * failed.  Host only; launches nothing. */
+int32_t bq_cuda_last_error(void);
+
+/* Static description of a cudaError_t value from bq_cuda_last_error. */
+const char* bq_cuda_error_string(int32_t code);
 
 /* Static, human-readable name of a status code. */
 const char* bq_status_string(bq_status status);

@@ -38,6 +38,8 @@ EXPORTED = (
     "bq_w2a16_linear_workspace_size",
     "bq_w2a16_linear",
     "bq_status_string",
+    "bq_cuda_last_error",
+    "bq_cuda_error_string",
 )
 
 
@@ -87,6 +89,8 @@ def load(path: str | None = None):
         "bq_w2a16_linear_workspace_size": (sz, [i32, i64, i64]),
         "bq_w2a16_linear": (i32, [lp, vp, i32, i64, vp, vp, vp, i64, i32, i32, vp, i32, vp, sz, vp, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
+        "bq_cuda_last_error": (i32, []),
+        "bq_cuda_error_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -102,7 +106,12 @@ def status_string(status: int) -> str:
 
 def _check(name: str, status: int):
     if status != BQ_OK:
-        raise BQError(name, status, status_string(status))
+        text = status_string(status)
+        if status == BQ_ERR_CUDA:  # which CUDA call failed, from the library's own runtime
+            code = int(load().bq_cuda_last_error())
+            if code:
+                text += f"; CUDA error {code}: {load().bq_cuda_error_string(code).decode()}"
+        raise BQError(name, status, text)
 
 
 # ----------------------------------------------------------------------------- marshalling helpers

@@ -74,6 +74,10 @@ using namespace bq;
 
 extern "C" {
 
+int32_t bq_cuda_last_error(void) { return static_cast<int32_t>(cudaGetLastError()); }
+
+const char* bq_cuda_error_string(int32_t code) { return cudaGetErrorString(static_cast<cudaError_t>(code)); }
+
 size_t bq_table_floats(int32_t m) {
   if (!valid_m(m)) return 0;
   return table_layout(m).total;

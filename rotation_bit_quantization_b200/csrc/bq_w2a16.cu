@@ -1093,6 +1093,8 @@ extern "C" bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dt
                                      int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,
                                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   if (!layer || tokens < 0) return BQ_ERR_INVALID_ARG;
+  if (!valid_gemm_shape(tokens, layer->n, out_features, bits, group) || (out_t != BQ_F32 && out_t != BQ_BF16))
+    return BQ_ERR_INVALID_ARG;
   if (tokens == 0) return BQ_OK;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
   const size_t xb = act_bytes(layer->n, tokens);

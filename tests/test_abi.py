@@ -282,3 +282,37 @@ def test_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError):
         _lib._dev(torch.zeros(4), "x")
+
+
+def test_zero_rows_launch_nothing(lib):
+    """Zero rows (tokens, features, count) return BQ_OK once the other arguments are
+    valid, with NULL data pointers: nothing is launched (this runs without a GPU).
+    The backward needs at least one token."""
+    layer = ctypes.byref(_layer(4096, 4096, 1, table=FAKE))
+    OK, BAD = _lib.BQ_OK, _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_butterfly_fwd(layer, None, _lib.BQ_BF16, None, _lib.BQ_F32, 0, None) == OK
+    assert lib.bq_butterfly_inv(layer, None, _lib.BQ_F32, None, _lib.BQ_BF16, 0, None) == OK
+    assert lib.bq_butterfly_fwd(layer, None, 7, None, _lib.BQ_F32, 0, None) == BAD        # bad dtype first
+    assert lib.bq_transform_quantize(layer, None, _lib.BQ_BF16, 0, 4, 128, None, None, None, None) == OK
+    assert lib.bq_transform_quantize(layer, None, _lib.BQ_BF16, 0, 3, 128, None, None, None, None) == BAD
+    assert lib.bq_weight_rotate_pack(layer, None, _lib.BQ_BF16, 0, 2, 128, None, None, None, None) == OK
+    assert lib.bq_uniformity_loss(None, 0, 4096, 4, 128, 1e-4, None, None, None, None) == OK
+    assert lib.bq_angle_sgd(None, None, 0, 0.1, None) == OK
+    assert lib.bq_w2a16_gemm(None, 0, 4096, None, None, None, 11008, 2, 128, None, _lib.BQ_BF16, None, 0, None,
+                             None) == OK
+    assert lib.bq_w2a16_gemm(None, 16, 4096, None, None, None, 0, 2, 128, None, _lib.BQ_BF16, None, 0, None,
+                             None) == OK
+    assert lib.bq_w2a16_linear(layer, None, _lib.BQ_BF16, 0, None, None, None, 11008, 2, 128, None, _lib.BQ_BF16,
+                               None, 0, None, None) == OK
+    assert lib.bq_w2a16_linear(layer, None, _lib.BQ_BF16, 0, None, None, None, 11008, 3, 128, None, _lib.BQ_BF16,
+                               None, 0, None, None) == BAD
+    bwd_layers = (_lib.BQLayer * 1)(_layer(4096, 4096, 1, table=FAKE))
+    assert lib.bq_butterfly_bwd(bwd_layers, 1, FAKE, _lib.BQ_BF16, FAKE, _lib.BQ_BF16, FAKE, FAKE, FAKE, 0, FAKE,
+                                1 << 20, None) == BAD
+
+
+def test_cuda_error_accessors(lib):
+    """The library's own CUDA runtime error is readable through the ABI (host only)."""
+    assert lib.bq_cuda_error_string(0) == b"no error"
+    assert isinstance(lib.bq_cuda_error_string(2), bytes) and lib.bq_cuda_error_string(2)
+    assert isinstance(int(lib.bq_cuda_last_error()), int)
