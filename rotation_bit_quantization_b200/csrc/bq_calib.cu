@@ -18,8 +18,9 @@
 // Each lane accumulates its values' weights into its own column of a per-warp
 // [B][32] histogram in shared memory (each address has one writer, so the order
 // of the additions is fixed and results are reproducible), a group's columns are
-// added in a fixed order, and each level's logarithm is taken once and read back
-// by each lane from its own column for the gradient.  (Two copies per lane, even
+// added in a fixed order, and each level's logarithm is taken once; the
+// differences of successive logarithms (the gradient's numerators) go back into
+// each lane's own column, one read per value for the gradient.  (Two copies per lane, even
 // and odd values, measured slower: the chains of read-modify-writes are not the
 // limit.)  The loss (the mean over groups) is summed by a cluster of eight CTAs,
 // each over a fixed eighth, and added up in rank order by the first: one CTA alone
