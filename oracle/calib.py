@@ -75,7 +75,7 @@ def uniformity_loss(y32, bits: int, group: int, eps: float):
     return loss, kl, dy
 
 
-def reconstruction_loss(theta, w, x, bits: int, group: int):
+def reconstruction_loss(theta, w, x, bits: int, group: int, abs_scale: bool = False):
     """Reconstruction loss of one linear layer under weight quantization, and its
     gradient with a straight-through estimator (readings of the explainer article,
     section "training & results": the quantized layer's output should match the
@@ -87,7 +87,10 @@ def reconstruction_loss(theta, w, x, bits: int, group: int):
     The straight-through estimator takes dW_hat / dV as the identity, so
         G_x = dloss/dx~ = (2/T) r W_hat,   G_v = dloss/dV = (2/T) r^T x~,
     and dtheta adds the backward of the activation side (rows x, gradient G_x)
-    and of the weight side (rows w, gradient G_v).  Returns (loss, dtheta)."""
+    and of the weight side (rows w, gradient G_v).  Returns (loss, dtheta), or with
+    abs_scale=True (loss, dtheta, A) where A = the sizes of the terms summed into
+    dtheta, both sides (``butterfly.backward_abs_scale``), which scales the tolerance
+    of a float32 dtheta per angle."""
     from . import butterfly as ob
     w = np.asarray(w, dtype=np.float64)
     x = np.asarray(x, dtype=np.float64)
@@ -102,4 +105,7 @@ def reconstruction_loss(theta, w, x, bits: int, group: int):
     g_v = (2.0 / T) * (r.T @ xt)
     _, _, dth_x = ob.backward(theta, x, g_x)
     _, _, dth_v = ob.backward(theta, w, g_v)
+    if abs_scale:
+        A = ob.backward_abs_scale(theta, x, g_x) + ob.backward_abs_scale(theta, w, g_v)
+        return loss, dth_x + dth_v, A
     return loss, dth_x + dth_v

@@ -262,6 +262,40 @@ def test_backward_abs_scale_bounds_dtheta():
     assert np.all(np.abs(dth) <= A * (1 + 1e-12))
 
 
+def test_backward_abs_scale_closed_form():
+    # theta = 0: v = x and g = dy at every stage, so A[s, p] is the plain sum over
+    # tokens of |dy_j x_i| + |dy_i x_j| for the pair (i, j) of stage s.  With dy
+    # non-zero only at positions 2 and 3 (m = 8), the pairs that touch them are
+    # (2, 3) at stage 0, (0, 2) and (1, 3) at stage 1, (2, 6) and (3, 7) at stage 2;
+    # every other entry is exactly 0.  A doubled, squared or dropped term fails.
+    m = 8
+    th = np.zeros((3, 4), dtype=np.float32)
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((5, m))
+    dy = np.zeros((5, m)); dy[:, 2] = rng.standard_normal(5); dy[:, 3] = rng.standard_normal(5)
+    A = bf.backward_abs_scale(th, x, dy)
+    want = np.zeros((3, 4))
+    want[0, 1] = (np.abs(dy[:, 3] * x[:, 2]) + np.abs(dy[:, 2] * x[:, 3])).sum()
+    want[1, 0] = np.abs(dy[:, 2] * x[:, 0]).sum()
+    want[1, 1] = np.abs(dy[:, 3] * x[:, 1]).sum()
+    want[2, 2] = np.abs(dy[:, 2] * x[:, 6]).sum()
+    want[2, 3] = np.abs(dy[:, 3] * x[:, 7]).sum()
+    assert np.allclose(A, want, rtol=1e-14, atol=0.0)
+
+
+def test_backward_abs_scale_single_rotation():
+    # m = 2, one stage at an arbitrary angle: v = y = R x, g = dy, so
+    # A = sum over tokens of |dy_1 y_0| + |dy_0 y_1|
+    th = np.array([[0.7]], dtype=np.float32)
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((7, 2)); dy = rng.standard_normal((7, 2))
+    c, sn = np.cos(np.float64(np.float32(0.7))), np.sin(np.float64(np.float32(0.7)))
+    y0 = c * x[:, 0] - sn * x[:, 1]
+    y1 = sn * x[:, 0] + c * x[:, 1]
+    A = bf.backward_abs_scale(th, x, dy)
+    assert np.isclose(A[0, 0], (np.abs(dy[:, 1] * y0) + np.abs(dy[:, 0] * y1)).sum(), rtol=1e-14, atol=0.0)
+
+
 # ---------------------------------------------------------------- quantizer
 
 def _golden_quant():
