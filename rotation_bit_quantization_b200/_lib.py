@@ -204,6 +204,11 @@ class Layer:
         """Whether the scaled two-FMA rotation form is in range for these angles (header flag)."""
         return bool(self.table[0].item() == 1.0)
 
+    @property
+    def fast_form_inverse(self) -> bool:
+        """Whether the scaled form of the inverse is in range for these angles (header flag)."""
+        return bool(self.table[3].item() == 1.0)
+
 
 # ----------------------------------------------------------------------------- entry points
 

@@ -6,20 +6,6 @@
 namespace bq {
 namespace {
 
-bool valid_m(int m) { return m >= 2 && m <= kMaxM && (m & (m - 1)) == 0; }
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-bool valid_dtype(bq_dtype t) { return t == BQ_F32 || t == BQ_BF16; }
-
-bq_status check_layer(const bq_layer* l) {
-  if (!l) return BQ_ERR_INVALID_ARG;
-  if (!valid_m(l->m) || l->r < 1 || l->r > kMaxR) return BQ_ERR_INVALID_ARG;
-  if (static_cast<long long>(l->m) * l->r != l->n || l->n > kMaxN) return BQ_ERR_INVALID_ARG;
-  if (!l->table || !aligned16(l->table)) return BQ_ERR_INVALID_ARG;
-  if ((l->r > 1) != (l->O != nullptr)) return BQ_ERR_INVALID_ARG;
-  if (l->O && (reinterpret_cast<uintptr_t>(l->O) & 3u)) return BQ_ERR_INVALID_ARG;
-  return BQ_OK;
-}
-
 bq_status check_rows(const void* a, const void* b, int64_t rows) {
   if (rows < 0) return BQ_ERR_INVALID_ARG;
   if (rows == 0) return BQ_OK;
@@ -112,18 +98,10 @@ size_t bq_butterfly_bwd_workspace_size(int32_t m, int32_t num_layers, int64_t ro
 bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers, const void* x, bq_dtype xt, void* y,
                            bq_dtype yt, const float* dy, float* dx, float* dtheta, int64_t rows_per_layer,
                            void* workspace, size_t workspace_bytes, void* stream) {
-  if (!layers || num_layers < 1 || num_layers > kMaxBwdLayers) return BQ_ERR_INVALID_ARG;
-  if (!valid_dtype(xt) || !valid_dtype(yt)) return BQ_ERR_INVALID_ARG;
-  const int m = layers[0].m;
   KLayer kl[kMaxBwdLayers];
-  for (int l = 0; l < num_layers; ++l) {
-    bq_status s = check_layer(&layers[l]);
-    if (s != BQ_OK) return s;
-    if (layers[l].m != m) return BQ_ERR_INVALID_ARG;
-    if (layers[l].r != 1) return BQ_ERR_UNSUPPORTED;
-    kl[l] = make_klayer(layers[l]);
-  }
-  if (rows_per_layer < 1) return BQ_ERR_INVALID_ARG;
+  const bq_status s = check_bwd_layers(layers, num_layers, xt, yt, rows_per_layer, kl);
+  if (s != BQ_OK) return s;
+  const int m = layers[0].m;
   const void* ptrs[] = {x, y, dy, dx, dtheta, workspace};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return BQ_ERR_INVALID_ARG;

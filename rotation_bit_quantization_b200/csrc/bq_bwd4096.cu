@@ -516,17 +516,16 @@ bq_status run(const B4Args& A, cudaStream_t st) {
   auto kern = k_bwd4096<TI, TO>;
   constexpr int smem = (5 * kBuf + 4 * M) * static_cast<int>(sizeof(float));
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
-  static int sms_of[64] = {};
-  if (sms_of[dev] == 0) {
-    int sms = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return BQ_ERR_CUDA;
-    sms_of[dev] = sms;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!once_per_device(ready, dev, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return BQ_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return BQ_ERR_CUDA;
   long long grid = static_cast<long long>(A.layers) * A.chunks;
-  if (grid > sms_of[dev]) grid = sms_of[dev];
+  if (grid > sms) grid = sms;
   kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(A);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }

@@ -210,7 +210,6 @@ bq_status uniformity_bits(const float* y, long long groups, int group, float eps
   }
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 }  // namespace bq

@@ -30,10 +30,12 @@
 //    fma.rn.f32x2 where two pairs sit in adjacent registers; when the layer's
 //    scaled form is out of range (table header flag 0) the same kernel runs the
 //    plain cos/sin rotation instead.
-//  * One CTA per SM (all 512 TMEM columns), three row groups per CTA sharing
-//    the tensor-memory image (warps w, w+4, w+8 use the same lanes) for
-//    latency hiding; the next row's input is prefetched into registers while
-//    the current row is processed.
+//  * One CTA per SM (all 512 TMEM columns) with kSlots row groups sharing the
+//    tensor-memory image (warps w, w + 4, ... use the same lanes).  The row is
+//    latency-bound (tensor-memory loads, transposes, the group barrier, the
+//    epilogue's reduction chain), so the kernel trades registers for resident
+//    warps: each thread reads one stage's coefficients at a time
+//    (kDoubleBuf false) and the next row's input is prefetched into registers.
 #include <cfloat>
 
 #include "bq_rtn.cuh"
@@ -43,10 +45,32 @@ namespace {
 
 constexpr int M = 4096;
 constexpr int kGroupThreads = 128;
-constexpr int kSlots = 3;
-constexpr int kThreads = kSlots * kGroupThreads;
 constexpr int kColB = 160, kColC = 320, kColS = 384;
-constexpr int kFillChunks = kImageCols / 16;  // 26 chunks of 16 columns, dealt round-robin to the slots
+constexpr int kFillChunks = kImageCols / 16;  // 26 chunks of 16 columns
+
+// forward kernel: kSlots row groups, each with an A -> B buffer, two alternating
+// B -> C buffers and the epilogue's parameter slots
+#ifndef BQ_FWD_SLOTS
+#define BQ_FWD_SLOTS 4
+#endif
+#ifndef BQ_FWD_DOUBLE_BUF
+#define BQ_FWD_DOUBLE_BUF 0
+#endif
+constexpr int kSlots = BQ_FWD_SLOTS;
+constexpr bool kDoubleBuf = BQ_FWD_DOUBLE_BUF != 0;
+constexpr int kThreads = kSlots * kGroupThreads;
+constexpr int kBufFloats = M;
+constexpr int kParamFloats = 4 * 32 * 4;  // 4 warps x 32 slots x float4
+constexpr int kSlotFloats = 3 * kBufFloats + kParamFloats;
+constexpr int kFwdSmemBytes = kSlots * kSlotFloats * static_cast<int>(sizeof(float));
+static_assert(kFwdSmemBytes <= 227 * 1024, "shared memory per CTA");
+// image chunks a thread loads per round of the start-up fill: all of its chunks at
+// once where registers allow (three row groups: 9 chunks, 144 registers), four at a
+// time with four row groups (128 registers per thread)
+#ifndef BQ_FILL_ROUND
+#define BQ_FILL_ROUND (kSlots >= 4 ? 4 : (kFillChunks + kSlots - 1) / kSlots)
+#endif
+constexpr int kFillRound = BQ_FILL_ROUND;
 
 enum Mode { kOutF32 = 0, kOutBF16 = 1, kQuant = 2 };
 
@@ -97,18 +121,18 @@ __device__ __forceinline__ float u2f(uint32_t v) { return __uint_as_float(v); }
 
 // ------------------------------------------------------------------ one stage in registers
 //
-// a[r][q] holds register slots (2q, 2q+1) of row r.  For in-register bit SB the
-// thread's 16 pairs are (j_k, j_k | 2^SB), j_k = ((k >> SB) << (SB+1)) | (k & (2^SB-1)),
-// and coefficient column 4q + e belongs to the low element of pair 2q + e,
-// column 4q + 2 + e to its high element.
+// a[q] holds register slots (2q, 2q+1).  For in-register bit SB the thread's 16
+// pairs are (j_k, j_k | 2^SB), j_k = ((k >> SB) << (SB+1)) | (k & (2^SB-1)), and
+// coefficient column 4q + e belongs to the low element of pair 2q + e, column
+// 4q + 2 + e to its high element.
 
 template <int SB>
 __host__ __device__ constexpr int low_slot(int k) {
   return ((k >> SB) << (SB + 1)) | (k & ((1 << SB) - 1));
 }
 
-template <int SB, bool SCALED, int R>
-__device__ __forceinline__ void stage(float2 (&a)[2][16], const uint32_t (&c)[32]) {
+template <int SB, bool SCALED>
+__device__ __forceinline__ void stage(float2 (&a)[16], const uint32_t (&c)[32]) {
   if constexpr (SB == 0) {
     // pairs (2k, 2k+1) sit inside one float2: scalar FMAs
 #pragma unroll
@@ -117,16 +141,13 @@ __device__ __forceinline__ void stage(float2 (&a)[2][16], const uint32_t (&c)[32
       for (int e = 0; e < 2; ++e) {
         const int k = 2 * q + e;
         const float cl = u2f(c[4 * q + e]), ch = u2f(c[4 * q + 2 + e]);
-#pragma unroll
-        for (int r = 0; r < R; ++r) {
-          const float lo = a[r][k].x, hi = a[r][k].y;
-          if constexpr (SCALED) {
-            a[r][k].x = fmaf(cl, hi, lo);
-            a[r][k].y = fmaf(ch, lo, hi);
-          } else {
-            a[r][k].x = fmaf(-ch, hi, cl * lo);
-            a[r][k].y = fmaf(cl, hi, ch * lo);
-          }
+        const float lo = a[k].x, hi = a[k].y;
+        if constexpr (SCALED) {
+          a[k].x = fmaf(cl, hi, lo);
+          a[k].y = fmaf(ch, lo, hi);
+        } else {
+          a[k].x = fmaf(-ch, hi, cl * lo);
+          a[k].y = fmaf(cl, hi, ch * lo);
         }
       }
     }
@@ -138,30 +159,35 @@ __device__ __forceinline__ void stage(float2 (&a)[2][16], const uint32_t (&c)[32
       const int hq = lq + kHalf;
       const float2 cl = make_float2(u2f(c[4 * q]), u2f(c[4 * q + 1]));
       const float2 ch = make_float2(u2f(c[4 * q + 2]), u2f(c[4 * q + 3]));
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const float2 lo = a[r][lq], hi = a[r][hq];
-        if constexpr (SCALED) {
-          a[r][lq] = __ffma2_rn(cl, hi, lo);
-          a[r][hq] = __ffma2_rn(ch, lo, hi);
-        } else {
-          const float2 nch = make_float2(-ch.x, -ch.y);
-          a[r][lq] = __ffma2_rn(nch, hi, __fmul2_rn(cl, lo));
-          a[r][hq] = __ffma2_rn(cl, hi, __fmul2_rn(ch, lo));
-        }
+      const float2 lo = a[lq], hi = a[hq];
+      if constexpr (SCALED) {
+        a[lq] = __ffma2_rn(cl, hi, lo);
+        a[hq] = __ffma2_rn(ch, lo, hi);
+      } else {
+        const float2 nch = make_float2(-ch.x, -ch.y);
+        a[lq] = __ffma2_rn(nch, hi, __fmul2_rn(cl, lo));
+        a[hq] = __ffma2_rn(cl, hi, __fmul2_rn(ch, lo));
       }
     }
   }
 }
 
-// Computes one stage from the coefficient block in `cur` while the block at
-// `next_addr` streams into `nxt`; returns after `nxt` has arrived.
-template <int SB, bool SCALED, int R>
-__device__ __forceinline__ void stage_step(float2 (&a)[2][16], uint32_t (&cur)[32], uint32_t (&nxt)[32],
-                                           uint32_t next_addr) {
-  tmem_ld32(next_addr, nxt);
-  stage<SB, SCALED, R>(a, cur);
-  tmem_wait(nxt);
+// One stage.  Double-buffered: computes from `cur` while the block at `next_addr`
+// streams into `nxt` and returns after it has arrived.  Single-buffered: loads
+// this stage's block at `addr` into `cur` and waits for it first (other warps of
+// the SM cover the wait).
+template <int SB, bool SCALED>
+__device__ __forceinline__ void stage_step(float2 (&a)[16], uint32_t (&cur)[32], uint32_t (&nxt)[32],
+                                           uint32_t addr, uint32_t next_addr) {
+  if constexpr (kDoubleBuf) {
+    tmem_ld32(next_addr, nxt);
+    stage<SB, SCALED>(a, cur);
+    tmem_wait(nxt);
+  } else {
+    tmem_ld32(addr, cur);
+    tmem_wait(cur);
+    stage<SB, SCALED>(a, cur);
+  }
 }
 
 // ------------------------------------------------------------------ inputs
@@ -171,47 +197,86 @@ struct Prefetch;
 template <>
 struct Prefetch<__nv_bfloat16> {
   static constexpr int kVec = 4;  // 16-byte vectors per row per thread (32 bf16)
-  uint4 v[2][kVec];
+  uint4 v[kVec];
 };
 template <>
 struct Prefetch<float> {
   static constexpr int kVec = 8;
-  uint4 v[2][kVec];
+  uint4 v[kVec];
 };
 
+// Pass-A layout input of one row (if cnt > 0): thread tau holds positions 32 tau .. 32 tau + 31.
 template <typename TI>
 __device__ __forceinline__ void prefetch(Prefetch<TI>& p, const TI* x, long long row, int cnt, int tau) {
+  if (cnt > 0) {
+    const uint4* src = reinterpret_cast<const uint4*>(x + row * M + tau * 32);
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    if (r < cnt) {
-      const uint4* src = reinterpret_cast<const uint4*>(x + (row + r) * M + tau * 32);
-#pragma unroll
-      for (int i = 0; i < Prefetch<TI>::kVec; ++i) p.v[r][i] = src[i];
-    }
+    for (int i = 0; i < Prefetch<TI>::kVec; ++i) p.v[i] = src[i];
   }
 }
 
-template <int R>
-__device__ __forceinline__ void unpack_input(const Prefetch<__nv_bfloat16>& p, float2 (&a)[2][16]) {
+__device__ __forceinline__ void unpack_input(const Prefetch<__nv_bfloat16>& p, float2 (&a)[16]) {
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t w[4] = {p.v[i].x, p.v[i].y, p.v[i].z, p.v[i].w};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const uint32_t w[4] = {p.v[r][i].x, p.v[r][i].y, p.v[r][i].z, p.v[r][i].w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k)
-        a[r][4 * i + k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
-    }
+    for (int k = 0; k < 4; ++k)
+      a[4 * i + k] = make_float2(__uint_as_float(w[k] << 16), __uint_as_float(w[k] & 0xffff0000u));
+  }
 }
 
-template <int R>
-__device__ __forceinline__ void unpack_input(const Prefetch<float>& p, float2 (&a)[2][16]) {
+__device__ __forceinline__ void unpack_input(const Prefetch<float>& p, float2 (&a)[16]) {
 #pragma unroll
-  for (int r = 0; r < R; ++r)
+  for (int i = 0; i < 8; ++i) {
+    a[2 * i] = make_float2(__uint_as_float(p.v[i].x), __uint_as_float(p.v[i].y));
+    a[2 * i + 1] = make_float2(__uint_as_float(p.v[i].z), __uint_as_float(p.v[i].w));
+  }
+}
+
+// ------------------------------------------------------------------ transposes
+//
+// A -> B: pass-A thread t writes its 32 positions as 16-byte vectors at float
+// 32 t + 4 (c ^ (t & 7)); pass-B threads read single floats.  B -> C: pass-B
+// threads write single floats, pass-C threads read 16-byte vectors, the two
+// halves of each 8-position run swapped by bit 2 of the thread index.  Every
+// access of a warp covers distinct banks in each of its phases.
+
+__device__ __forceinline__ void xpose_ab(float2 (&a)[16], float* buf, int tau) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      a[r][2 * i] = make_float2(__uint_as_float(p.v[r][i].x), __uint_as_float(p.v[r][i].y));
-      a[r][2 * i + 1] = make_float2(__uint_as_float(p.v[r][i].z), __uint_as_float(p.v[r][i].w));
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<float4*>(buf + tau * 32 + 4 * (c ^ (tau & 7))) =
+        make_float4(a[2 * c].x, a[2 * c].y, a[2 * c + 1].x, a[2 * c + 1].y);
+  // pass-A thread t writes positions 32 t .. 32 t + 31; pass-B thread t reads the
+  // positions of pass-A threads 32 (t >> 5) .. 32 (t >> 5) + 31: position bits 10, 11
+  // are the warp index in both layouts, so this exchange stays inside the warp
+  __syncwarp();
+  const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
+#pragma unroll
+  for (int rb = 0; rb < 32; rb += 2) {
+    const float v0 = buf[base + 32 * rb + 4 * (cq ^ (rb & 7))];
+    const float v1 = buf[base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))];
+    a[rb >> 1] = make_float2(v0, v1);
+  }
+}
+
+__device__ __forceinline__ void xpose_bc_write(const float2 (&a)[16], float* buf, int tau) {
+  const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
+#pragma unroll
+  for (int rb = 0; rb < 32; rb += 2) {
+    buf[base + 32 * rb + 4 * (sw ^ 0)] = a[rb >> 1].x;
+    buf[base + 32 * (rb + 1) + 4 * (sw ^ 1)] = a[rb >> 1].y;
+  }
+}
+
+__device__ __forceinline__ void xpose_bc_read(float2 (&a)[16], const float* buf, int tau) {
+  const int sw = (tau >> 2) & 1;
+#pragma unroll
+  for (int h = 0; h < 4; ++h)
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      const float4 v = *reinterpret_cast<const float4*>(buf + h * 1024 + tau * 8 + 4 * (hh ^ sw));
+      a[4 * h + 2 * hh] = make_float2(v.x, v.y);
+      a[4 * h + 2 * hh + 1] = make_float2(v.z, v.w);
     }
 }
 
@@ -252,32 +317,35 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
   return d;
 }
 
-// Per-group asymmetric RTN of the R rows held in pass-C layout, packing and stores.
+// Per-group asymmetric RTN of the row held in pass-C layout, packing and stores.
 //
-// Group extremes: 3-input min / max over each 8-value set, then a recursive-halving
-// shuffle reduction after which lane l holds set bitrev(l & (S-1)) of its group.
-// Every lane computes that group's parameters (scale16, s, z, 1 / s and the tie
-// threshold, as in rtn_params); each set then takes them by shuffle from the lane
-// that holds them and is coded by rtn_codes8 (exact RTN: see bq_rtn.cuh).  One
-// reducing warp per row group with the parameters in shared memory issues fewer
-// instructions but adds two row-group barriers, and measured slower at 2048 rows.
-template <int BITS, int GLANES, int R>
-__device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const FastArgs& A, long long row0, int tau,
-                                               int lane) {
-  constexpr int S = 4 * R;               // (row, hi2) sets per thread
-  constexpr int LOGS = clog2<0>(S);
+// Each thread holds 4 sets of 8 consecutive values (position bits 10, 11 = h); a
+// group of GROUP = 8 GLANES positions spans GLANES lanes.  Group extremes: 3-input
+// min / max over each set, then a recursive-halving shuffle reduction after which
+// lane l holds set bitrev(l & 3) of its group, and plain xor levels for the
+// remaining group lanes.  Every lane computes the parameters of the set it holds
+// (as in rtn_params); one lane per (group, set) stores scale and zero and puts
+// (1/s, tie threshold, 1.5 2^23 + z, s) into the warp's parameter slots in shared
+// memory, from which every lane reads the parameters of each of its sets after a
+// warp barrier (one broadcast load per set instead of four shuffles).  The codes
+// then come from rtn_codes8 (exact RTN: see bq_rtn.cuh).
+template <int BITS, int GLANES>
+__device__ __forceinline__ void quant_epilogue(const float2 (&a)[16], const FastArgs& A, long long row, int tau,
+                                               int lane, float4* params) {
+  constexpr int S = 4;                    // sets per thread
+  constexpr int LOGS = 2;
   constexpr int LOGG = clog2<0>(GLANES);  // lanes sharing one group
+  static_assert(LOGS <= LOGG, "a group must span at least S lanes");
   constexpr int GROUP = 8 * GLANES;
   constexpr int GPR = M / GROUP;          // groups per row
   constexpr int QMAX = (1 << BITS) - 1;
   const float qmax = static_cast<float>(QMAX);
   float mn[S], mx[S];
 #pragma unroll
-  for (int k = 0; k < S; ++k) {
-    const int r = k >> 2, h = k & 3;
-    const float2 p0 = a[r][4 * h], p1 = a[r][4 * h + 1], p2 = a[r][4 * h + 2], p3 = a[r][4 * h + 3];
-    mn[k] = fminf(min3(p0.x, p0.y, p1.x), min3(p1.y, p2.x, min3(p2.y, p3.x, p3.y)));
-    mx[k] = fmaxf(max3(p0.x, p0.y, p1.x), max3(p1.y, p2.x, max3(p2.y, p3.x, p3.y)));
+  for (int h = 0; h < S; ++h) {
+    const float2 p0 = a[4 * h], p1 = a[4 * h + 1], p2 = a[4 * h + 2], p3 = a[4 * h + 3];
+    mn[h] = fminf(min3(p0.x, p0.y, p1.x), min3(p1.y, p2.x, min3(p2.y, p3.x, p3.y)));
+    mx[h] = fmaxf(max3(p0.x, p0.y, p1.x), max3(p1.y, p2.x, max3(p2.y, p3.x, p3.y)));
   }
   // recursive halving over lane bits 0..LOGS-1: afterwards lane l holds set bitrev(l & (S-1))
 #pragma unroll
@@ -297,47 +365,21 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
     mn[0] = fminf(mn[0], __shfl_xor_sync(0xffffffffu, mn[0], 1 << i));
     mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], 1 << i));
   }
-  const float lo = mn[0], hi = mx[0];
-  __half h16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), qmax));
-  float s = __half2float(h16);
-  if (hi == lo || s == 0.f) {
-    s = 1.f;
-    h16 = __float2half_rn(1.f);
+  const RtnParams P = rtn_params(mn[0], mx[0], qmax);
+  const int slot0 = (lane >> LOGG) * S;
+  if (((lane >> LOGS) & ((1 << (LOGG - LOGS)) - 1)) == 0) {
+    const int h = bitrev<S>(lane & (S - 1));
+    const int g = h * (1024 / GROUP) + (tau >> LOGG);
+    A.scale[row * GPR + g] = P.scale16;
+    A.zero[row * GPR + g] = P.zero16;
+    params[slot0 + h] = make_float4(P.inv, P.thr, P.mz, P.s);
   }
-  const float zraw = rintf(__fdiv_rn(-lo, s));
-  const float z = __fadd_rn(fminf(fmaxf(zraw, 0.f), qmax), 0.f);  // +0 for a zero point of 0
-  const float inv = __fdiv_rn(1.f, s);
-  // tie margin for the whole group: every |v| <= max(|lo|, |hi|) * inv * (1 + 2^-20)
-  const float vmax = fmaxf(fabsf(lo), fabsf(hi)) * inv * 1.000001f;
-  const float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
-  // codes are monotone in y: when the group's extremes quantize inside [0, qmax],
-  // no element needs clamping.  Division and rint are both odd functions, so the
-  // code of lo is z - rint(-lo/s) exactly: in range at the bottom iff
-  // rint(-lo/s) <= qmax.  The top is checked with one IEEE division.
-  const bool inrange = zraw <= qmax && __fadd_rn(rintf(__fdiv_rn(hi, s)), z) <= qmax;
-  const float thr_in = inrange ? thr : -1.f;  // -1 sends the whole set to the slow path
-  {
-    const int k = bitrev<S>(lane & (S - 1));
-    if (((lane >> LOGS) & ((1 << (LOGG - LOGS)) - 1)) == 0) {
-      const long long row = row0 + (k >> 2);
-      const int g = (k & 3) * (1024 / GROUP) + (tau >> LOGG);
-      A.scale[row * GPR + g] = __half_as_ushort(h16);
-      A.zero[row * GPR + g] = __half_as_ushort(__float2half_rn(z));
-    }
-  }
-  // codes of each set with its group's parameters (from the lane that reduced it)
-  const float mz = __fadd_rn(12582912.f, z);
+  __syncwarp();
 #pragma unroll
-  for (int k = 0; k < S; ++k) {
-    const int src = (lane & ~(S - 1)) | bitrev<S>(k);
-    const float invk = __shfl_sync(0xffffffffu, inv, src);
-    const float thrk = __shfl_sync(0xffffffffu, thr_in, src);
-    const float mzk = __shfl_sync(0xffffffffu, mz, src);
-    const float sk = __shfl_sync(0xffffffffu, s, src);
-    const int r = k >> 2, h = k & 3;
-    const float2 y[4] = {a[r][4 * h], a[r][4 * h + 1], a[r][4 * h + 2], a[r][4 * h + 3]};
-    const uint32_t word = rtn_codes8<BITS>(y, invk, thrk, mzk, sk);
-    const long long row = row0 + r;
+  for (int h = 0; h < S; ++h) {
+    const float4 q = params[slot0 + h];
+    const float2 y[4] = {a[4 * h], a[4 * h + 1], a[4 * h + 2], a[4 * h + 3]};
+    const uint32_t word = rtn_codes8<BITS>(y, q.x, q.y, q.z, q.w);
     if constexpr (BITS == 4) {
       *reinterpret_cast<uint32_t*>(A.codes + row * (M / 2) + h * 512 + tau * 4) = word;
     } else {
@@ -346,167 +388,128 @@ __device__ __forceinline__ void quant_epilogue(const float2 (&a)[2][16], const F
   }
 }
 
-template <int MODE, int R>
-__device__ __forceinline__ void store_epilogue(const float2 (&a)[2][16], const FastArgs& A, long long row0, int tau) {
+template <int MODE>
+__device__ __forceinline__ void store_epilogue(const float2 (&a)[16], const FastArgs& A, long long row, int tau) {
 #pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const long long off = (row0 + r) * M + h * 1024 + tau * 8;
-      if constexpr (MODE == kOutF32) {
-        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(A.y) + off);
-        dst[0] = make_float4(a[r][4 * h].x, a[r][4 * h].y, a[r][4 * h + 1].x, a[r][4 * h + 1].y);
-        dst[1] = make_float4(a[r][4 * h + 2].x, a[r][4 * h + 2].y, a[r][4 * h + 3].x, a[r][4 * h + 3].y);
-      } else {
-        uint4 w;
-        __nv_bfloat162 b0 = __floats2bfloat162_rn(a[r][4 * h].x, a[r][4 * h].y);
-        __nv_bfloat162 b1 = __floats2bfloat162_rn(a[r][4 * h + 1].x, a[r][4 * h + 1].y);
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(a[r][4 * h + 2].x, a[r][4 * h + 2].y);
-        __nv_bfloat162 b3 = __floats2bfloat162_rn(a[r][4 * h + 3].x, a[r][4 * h + 3].y);
-        w.x = *reinterpret_cast<uint32_t*>(&b0);
-        w.y = *reinterpret_cast<uint32_t*>(&b1);
-        w.z = *reinterpret_cast<uint32_t*>(&b2);
-        w.w = *reinterpret_cast<uint32_t*>(&b3);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(A.y) + off) = w;
-      }
+  for (int h = 0; h < 4; ++h) {
+    const long long off = row * M + h * 1024 + tau * 8;
+    if constexpr (MODE == kOutF32) {
+      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(A.y) + off);
+      dst[0] = make_float4(a[4 * h].x, a[4 * h].y, a[4 * h + 1].x, a[4 * h + 1].y);
+      dst[1] = make_float4(a[4 * h + 2].x, a[4 * h + 2].y, a[4 * h + 3].x, a[4 * h + 3].y);
+    } else {
+      uint4 w;
+      __nv_bfloat162 b0 = __floats2bfloat162_rn(a[4 * h].x, a[4 * h].y);
+      __nv_bfloat162 b1 = __floats2bfloat162_rn(a[4 * h + 1].x, a[4 * h + 1].y);
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(a[4 * h + 2].x, a[4 * h + 2].y);
+      __nv_bfloat162 b3 = __floats2bfloat162_rn(a[4 * h + 3].x, a[4 * h + 3].y);
+      w.x = *reinterpret_cast<uint32_t*>(&b0);
+      w.y = *reinterpret_cast<uint32_t*>(&b1);
+      w.z = *reinterpret_cast<uint32_t*>(&b2);
+      w.w = *reinterpret_cast<uint32_t*>(&b3);
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(A.y) + off) = w;
     }
+  }
 }
 
-// One group of R rows through all twelve stages and the epilogue.  On entry
-// c0 holds coefficient block 0 (waited for) and `pre` holds the rows' input;
-// on return c0 again holds block 0 and `pre` holds the next rows' input.
-template <typename TI, int MODE, int BITS, int GLANES, bool SCALED, int R>
-__device__ __forceinline__ void process(const FastArgs& A, long long row0, long long nrow, int ncnt, int slot,
-                                        int tau, int lane, uint32_t tb, float* bufAB, float* bufBC,
+// One row through all twelve stages and the epilogue.  On entry `pre` holds the
+// row's input (and, double-buffered, c0 holds coefficient block 0); on return
+// `pre` holds the next row's input (if ncnt > 0).
+template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
+__device__ __forceinline__ void process(const FastArgs& A, long long row, int ncnt, int slot, int tau, int lane,
+                                        uint32_t tb, float* bufAB, float* bufBC, float4* params,
                                         Prefetch<TI>& pre, uint32_t (&c0)[32], uint32_t (&c1)[32]) {
-  float2 a[2][16];
-  unpack_input<R>(pre, a);
-  prefetch(pre, static_cast<const TI*>(A.x), nrow, ncnt, tau);
+  float2 a[16];
+  unpack_input(pre, a);
+  prefetch(pre, static_cast<const TI*>(A.x), row + 1, ncnt, tau);
 
   // pass A: stages 0..4 on position bits 0..4
-  stage_step<0, SCALED, R>(a, c0, c1, tb + 32);
-  stage_step<1, SCALED, R>(a, c1, c0, tb + 64);
-  stage_step<2, SCALED, R>(a, c0, c1, tb + 96);
-  stage_step<3, SCALED, R>(a, c1, c0, tb + 128);
-  stage_step<4, SCALED, R>(a, c0, c1, tb + kColB);
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-      *reinterpret_cast<float4*>(bufAB + r * M + tau * 32 + 4 * (c ^ (tau & 7))) =
-          make_float4(a[r][2 * c].x, a[r][2 * c].y, a[r][2 * c + 1].x, a[r][2 * c + 1].y);
-  // pass-A thread t writes row t (positions 32t..32t+31); pass-B thread t reads rows
-  // 32(t >> 5) .. 32(t >> 5) + 31: position bits 10, 11 are the warp index in both
-  // layouts, so this exchange stays inside the warp
-  __syncwarp();
-  {
-    const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int rb = 0; rb < 32; rb += 2) {
-        const float v0 = bufAB[r * M + base + 32 * rb + 4 * (cq ^ (rb & 7))];
-        const float v1 = bufAB[r * M + base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))];
-        a[r][rb >> 1] = make_float2(v0, v1);
-      }
-  }
+  stage_step<0, SCALED>(a, c0, c1, tb, tb + 32);
+  stage_step<1, SCALED>(a, c1, c0, tb + 32, tb + 64);
+  stage_step<2, SCALED>(a, c0, c1, tb + 64, tb + 96);
+  stage_step<3, SCALED>(a, c1, c0, tb + 96, tb + 128);
+  stage_step<4, SCALED>(a, c0, c1, tb + 128, tb + kColB);
+  xpose_ab(a, bufAB, tau);
   // pass B: stages 5..9 on position bits 5..9
-  stage_step<0, SCALED, R>(a, c1, c0, tb + kColB + 32);
-  stage_step<1, SCALED, R>(a, c0, c1, tb + kColB + 64);
-  stage_step<2, SCALED, R>(a, c1, c0, tb + kColB + 96);
-  stage_step<3, SCALED, R>(a, c0, c1, tb + kColB + 128);
-  stage_step<4, SCALED, R>(a, c1, c0, tb + kColC);
-  {
-    const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int rb = 0; rb < 32; rb += 2) {
-        bufBC[r * M + base + 32 * rb + 4 * (sw ^ 0)] = a[r][rb >> 1].x;
-        bufBC[r * M + base + 32 * (rb + 1) + 4 * (sw ^ 1)] = a[r][rb >> 1].y;
-      }
-  }
+  stage_step<0, SCALED>(a, c1, c0, tb + kColB, tb + kColB + 32);
+  stage_step<1, SCALED>(a, c0, c1, tb + kColB + 32, tb + kColB + 64);
+  stage_step<2, SCALED>(a, c1, c0, tb + kColB + 64, tb + kColB + 96);
+  stage_step<3, SCALED>(a, c0, c1, tb + kColB + 96, tb + kColB + 128);
+  stage_step<4, SCALED>(a, c1, c0, tb + kColB + 128, tb + kColC);
+  xpose_bc_write(a, bufBC, tau);
   group_sync(slot);
-  {
-    const int sw = (tau >> 2) & 1;
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int h = 0; h < 4; ++h)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const float4 v = *reinterpret_cast<const float4*>(bufBC + r * M + h * 1024 + tau * 8 + 4 * (hh ^ sw));
-          a[r][4 * h + 2 * hh] = make_float2(v.x, v.y);
-          a[r][4 * h + 2 * hh + 1] = make_float2(v.z, v.w);
-        }
-  }
+  xpose_bc_read(a, bufBC, tau);
   // pass C: stages 10, 11 on slot bits 3, 4 (position bits 10, 11)
-  stage_step<3, SCALED, R>(a, c0, c1, tb + kColC + 32);
-  stage_step<4, SCALED, R>(a, c1, c0, tb + kColS);
-  // output scale (1 for the plain rotation), then start loading the next group's block 0
-#pragma unroll
-  for (int r = 0; r < R; ++r)
-#pragma unroll
-    for (int q = 0; q < 16; ++q) a[r][q] = __fmul2_rn(a[r][q], make_float2(u2f(c0[2 * q]), u2f(c0[2 * q + 1])));
-  tmem_ld32(tb, c0);
-  if constexpr (MODE == kQuant) {
-    quant_epilogue<BITS, GLANES, R>(a, A, row0, tau, lane);
-  } else {
-    store_epilogue<MODE, R>(a, A, row0, tau);
+  stage_step<3, SCALED>(a, c0, c1, tb + kColC, tb + kColC + 32);
+  stage_step<4, SCALED>(a, c1, c0, tb + kColC + 32, tb + kColS);
+  // output scale (1 for the plain rotation)
+  if constexpr (!kDoubleBuf) {
+    tmem_ld32(tb + kColS, c0);
+    tmem_wait(c0);
   }
-  tmem_wait(c0);
+#pragma unroll
+  for (int q = 0; q < 16; ++q) a[q] = __fmul2_rn(a[q], make_float2(u2f(c0[2 * q]), u2f(c0[2 * q + 1])));
+  if constexpr (kDoubleBuf) tmem_ld32(tb, c0);  // block 0 of the next row
+  if constexpr (MODE == kQuant) {
+    quant_epilogue<BITS, GLANES>(a, A, row, tau, lane, params);
+  } else {
+    store_epilogue<MODE>(a, A, row, tau);
+  }
+  if constexpr (kDoubleBuf) tmem_wait(c0);
 }
 
 template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
 __device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long long re, int slot, int tau, int lane,
-                                         uint32_t tb, float* bufAB, float* bufBC, Prefetch<TI>& pre,
+                                         uint32_t tb, float* bufAB, float* bufBC, float4* params, Prefetch<TI>& pre,
                                          uint32_t (&c0)[32], uint32_t (&c1)[32]) {
   // the B -> C buffer alternates between rows: with only a warp-level sync before
   // the next row's B -> C writes, row i's readers and row i+2's writers are kept
   // apart by row i+1's row-group barrier
 #pragma unroll 1
   for (long long row = rb; row < re; ++row)
-    process<TI, MODE, BITS, GLANES, SCALED, 1>(A, row, row + 1, row + 1 < re ? 1 : 0, slot, tau, lane, tb, bufAB,
-                                               bufBC + ((row - rb) & 1) * M, pre, c0, c1);
+    process<TI, MODE, BITS, GLANES, SCALED>(A, row, row + 1 < re ? 1 : 0, slot, tau, lane, tb, bufAB,
+                                            bufBC + ((row - rb) & 1) * kBufFloats, params, pre, c0, c1);
 }
 
 // Copies this thread's share of a tensor-memory image (NCHUNK chunks of 16
-// columns, dealt round-robin to the slots) into its lane: all loads in flight
-// first (each warp load is one contiguous 512-byte run of the [column/4][lane]
-// image), then the stores.  Every CTA reads the same image at the same moment,
-// so each starts at a different chunk (block index mod NCHUNK): the requests in
-// flight then spread over the L2 slices instead of queueing on the same few.
-// (Sharing one L2 read per CTA pair through distributed shared memory was
-// slower: gathering 208 KB per SM that way costs more than the L2 reads saved.)
-template <int NCHUNK>
+// columns, dealt round-robin to the NSLOT row groups) into its lane, ROUND chunks
+// at a time: all loads of a round in flight first (each warp load is one
+// contiguous 512-byte run of the [column/4][lane] image), then the stores.  Every
+// CTA reads the same image at the same moment, so each starts at a different
+// chunk (block index mod NCHUNK): the requests in flight then spread over the L2
+// slices instead of queueing on the same few.
+template <int NCHUNK, int NSLOT, int ROUND>
 __device__ __forceinline__ void fill_tmem(const float* image, uint32_t tb, int slot, int tau) {
   const float4* src = reinterpret_cast<const float4*>(image) + tau;  // block q of lane tau at [q * 128]
-  constexpr int kMine = (NCHUNK + kSlots - 1) / kSlots;
-  float4 f[kMine * 4];
+  constexpr int kMine = (NCHUNK + NSLOT - 1) / NSLOT;
   const int rot = blockIdx.x % NCHUNK;
 #pragma unroll
-  for (int i = 0; i < kMine; ++i) {
-    const int c0 = slot + i * kSlots;
-    if (c0 < NCHUNK) {
-      const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
+  for (int base = 0; base < kMine; base += ROUND) {
+    float4 f[ROUND * 4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
-    }
-  }
+    for (int i = 0; i < ROUND; ++i) {
+      const int c0 = slot + (base + i) * NSLOT;
+      if (base + i < kMine && c0 < NCHUNK) {
+        const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
 #pragma unroll
-  for (int i = 0; i < kMine; ++i) {
-    const int c0 = slot + i * kSlots;
-    if (c0 < NCHUNK) {
-      const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
-      uint32_t v[16];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        v[4 * j] = __float_as_uint(f[4 * i + j].x);
-        v[4 * j + 1] = __float_as_uint(f[4 * i + j].y);
-        v[4 * j + 2] = __float_as_uint(f[4 * i + j].z);
-        v[4 * j + 3] = __float_as_uint(f[4 * i + j].w);
+        for (int j = 0; j < 4; ++j) f[4 * i + j] = src[(4 * c + j) * kImageLanes];
       }
-      tmem_st16(tb + 16 * c, v);
+    }
+#pragma unroll
+    for (int i = 0; i < ROUND; ++i) {
+      const int c0 = slot + (base + i) * NSLOT;
+      if (base + i < kMine && c0 < NCHUNK) {
+        const int c = c0 + rot < NCHUNK ? c0 + rot : c0 + rot - NCHUNK;
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[4 * j] = __float_as_uint(f[4 * i + j].x);
+          v[4 * j + 1] = __float_as_uint(f[4 * i + j].y);
+          v[4 * j + 2] = __float_as_uint(f[4 * i + j].z);
+          v[4 * j + 3] = __float_as_uint(f[4 * i + j].w);
+        }
+        tmem_st16(tb + 16 * c, v);
+      }
     }
   }
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
@@ -518,8 +521,10 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __shared__ uint32_t s_tmem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
-  float* bufAB = smem + slot * (3 * M);
-  float* bufBC = bufAB + M;  // two buffers, used alternately
+  float* sbase = smem + slot * kSlotFloats;
+  float* bufAB = sbase;
+  float* bufBC = sbase + kBufFloats;  // two buffers, used alternately
+  float4* params = reinterpret_cast<float4*>(sbase + 3 * kBufFloats) + wq * 32;
   const long long G = static_cast<long long>(gridDim.x) * kSlots;
   const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
@@ -536,19 +541,21 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  fill_tmem<kFillChunks>(A.image, tb, slot, tau);
+  fill_tmem<kFillChunks, kSlots, kFillRound>(A.image, tb, slot, tau);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
   const bool scaled = A.hdr[0] == 1.f;
   uint32_t c0[32], c1[32];
-  tmem_ld32(tb, c0);
-  tmem_wait(c0);
+  if constexpr (kDoubleBuf) {
+    tmem_ld32(tb, c0);
+    tmem_wait(c0);
+  }
   if (scaled)
-    run_rows<TI, MODE, BITS, GLANES, true>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, pre, c0, c1);
+    run_rows<TI, MODE, BITS, GLANES, true>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, params, pre, c0, c1);
   else
-    run_rows<TI, MODE, BITS, GLANES, false>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, pre, c0, c1);
+    run_rows<TI, MODE, BITS, GLANES, false>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, params, pre, c0, c1);
 
   tc_fence_before();
   __syncthreads();
@@ -561,23 +568,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
 template <typename TI, int MODE, int BITS, int GLANES>
 bq_status launch(const FastArgs& A, cudaStream_t st) {
   auto kern = k_fast4096<TI, MODE, BITS, GLANES>;
-  const int smem = kSlots * 3 * M * static_cast<int>(sizeof(float));
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
-  // per device: the shared-memory opt-in and the SM count, set up on first use
-  static int sms_of[64] = {};
-  if (sms_of[dev] == 0) {
-    int sms = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return BQ_ERR_CUDA;
-    sms_of[dev] = sms;
-  }
-  const int sms = sms_of[dev];
+  if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!once_per_device(ready, dev, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmemBytes) ==
+               cudaSuccess;
+      }))
+    return BQ_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return BQ_ERR_CUDA;
   long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(A);
+  kern<<<static_cast<unsigned>(grid), kThreads, kFwdSmemBytes, st>>>(A);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -596,14 +600,18 @@ bq_status dispatch_quant(const FastArgs& A, int bits, int group, cudaStream_t st
 
 // ------------------------------------------------------------------ inverse
 //
-// x = Q^T y: stages 11 .. 0, each the transpose [[c, s], [-s, c]] of its rotation,
-// in the forward's thread layouts visited backwards (pass C, then B, then A) with
-// the two transposes reversed.  Coefficients: the plain (cos, sin) image, whose
-// stage-s block sits at column 32 s; the scaled form's [[1, alpha], [beta, 1]]
-// steps do not invert into steps of the same shape.
+// x = Q^T y: stages 11 .. 0, each the transposed rotation, in the forward's thread
+// layouts visited backwards (pass C, then B, then A) with the two transposes
+// reversed.  The rotation by -theta has the same scaled two-FMA form as the
+// forward, with its own coefficients and output scale prepared by
+// bq_precompute_cs (table header[3]); the image holds them in the forward's
+// columns (stage s at column 32 s, the output scale of the pass-A positions at
+// column 384), or (cos, sin) when that form is out of range, in which case the
+// plain transposed rotation [[c, s], [-s, c]] runs.  Same row groups, buffers
+// and coefficient loads as the forward.
 
 template <int SB>
-__device__ __forceinline__ void stage_inv(float2 (&a)[2][16], const uint32_t (&c)[32]) {
+__device__ __forceinline__ void stage_inv_plain(float2 (&a)[16], const uint32_t (&c)[32]) {
   if constexpr (SB == 0) {
 #pragma unroll
     for (int q = 0; q < 8; ++q)
@@ -611,9 +619,9 @@ __device__ __forceinline__ void stage_inv(float2 (&a)[2][16], const uint32_t (&c
       for (int e = 0; e < 2; ++e) {
         const int k = 2 * q + e;
         const float cl = u2f(c[4 * q + e]), ch = u2f(c[4 * q + 2 + e]);
-        const float lo = a[0][k].x, hi = a[0][k].y;
-        a[0][k].x = fmaf(ch, hi, cl * lo);
-        a[0][k].y = fmaf(-ch, lo, cl * hi);
+        const float lo = a[k].x, hi = a[k].y;
+        a[k].x = fmaf(ch, hi, cl * lo);
+        a[k].y = fmaf(-ch, lo, cl * hi);
       }
   } else {
 #pragma unroll
@@ -623,19 +631,29 @@ __device__ __forceinline__ void stage_inv(float2 (&a)[2][16], const uint32_t (&c
       const int hq = lq + kHalf;
       const float2 cl = make_float2(u2f(c[4 * q]), u2f(c[4 * q + 1]));
       const float2 ch = make_float2(u2f(c[4 * q + 2]), u2f(c[4 * q + 3]));
-      const float2 lo = a[0][lq], hi = a[0][hq];
-      a[0][lq] = __ffma2_rn(ch, hi, __fmul2_rn(cl, lo));
-      a[0][hq] = __ffma2_rn(make_float2(-ch.x, -ch.y), lo, __fmul2_rn(cl, hi));
+      const float2 lo = a[lq], hi = a[hq];
+      a[lq] = __ffma2_rn(ch, hi, __fmul2_rn(cl, lo));
+      a[hq] = __ffma2_rn(make_float2(-ch.x, -ch.y), lo, __fmul2_rn(cl, hi));
     }
   }
 }
 
-// stage S of the inverse from `cur`, while the block of stage S - 1 streams into `nxt`
-template <int S, int SB>
-__device__ __forceinline__ void inv_step(float2 (&a)[2][16], uint32_t (&cur)[32], uint32_t (&nxt)[32], uint32_t tb) {
-  if constexpr (S > 0) tmem_ld32(tb + 32 * (S - 1), nxt);
-  stage_inv<SB>(a, cur);
-  if constexpr (S > 0) tmem_wait(nxt);
+// Stage S (in-register bit SB) of the inverse; the next stage in visiting order
+// is S - 1 (after stage 0: stage 11 of the next row).
+template <int S, int SB, bool SCALED>
+__device__ __forceinline__ void inv_step(float2 (&a)[16], uint32_t (&cur)[32], uint32_t (&nxt)[32], uint32_t tb) {
+  if constexpr (kDoubleBuf) {
+    tmem_ld32(tb + 32 * (S > 0 ? S - 1 : 11), nxt);
+  } else {
+    tmem_ld32(tb + 32 * S, cur);
+    tmem_wait(cur);
+  }
+  if constexpr (SCALED) {
+    stage<SB, true>(a, cur);
+  } else {
+    stage_inv_plain<SB>(a, cur);
+  }
+  if constexpr (kDoubleBuf) tmem_wait(nxt);
 }
 
 // Pass-C layout input: thread tau holds positions 8 tau + 1024 h + (0..7), h < 4.
@@ -647,21 +665,21 @@ __device__ __forceinline__ void prefetch_c(Prefetch<TI>& p, const TI* x, long lo
     for (int h = 0; h < 4; ++h) {
       const uint4* src = reinterpret_cast<const uint4*>(x + row * M + h * 1024 + tau * 8);
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) p.v[0][kPer * h + i] = src[i];
+      for (int i = 0; i < kPer; ++i) p.v[kPer * h + i] = src[i];
     }
   }
 }
 
-template <typename TI, typename TO>
+template <typename TI, typename TO, bool SCALED>
 __device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int ncnt, int slot, int tau, uint32_t tb,
                                         float* bufAB, float* bufBC, Prefetch<TI>& pre, uint32_t (&c0)[32],
                                         uint32_t (&c1)[32]) {
-  float2 a[2][16];
-  unpack_input<1>(pre, a);
+  float2 a[16];
+  unpack_input(pre, a);
   prefetch_c(pre, static_cast<const TI*>(A.x), row + 1, ncnt, tau);
-  // pass C: stages 11, 10 (slot bits 4, 3); c0 holds block 11 on entry
-  inv_step<11, 4>(a, c0, c1, tb);
-  inv_step<10, 3>(a, c1, c0, tb);
+  // pass C: stages 11, 10 (slot bits 4, 3); double-buffered, c0 holds block 11 on entry
+  inv_step<11, 4, SCALED>(a, c0, c1, tb);
+  inv_step<10, 3, SCALED>(a, c1, c0, tb);
   {
     const int sw = (tau >> 2) & 1;
 #pragma unroll
@@ -669,50 +687,55 @@ __device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int nc
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
         *reinterpret_cast<float4*>(bufBC + h * 1024 + tau * 8 + 4 * (hh ^ sw)) =
-            make_float4(a[0][4 * h + 2 * hh].x, a[0][4 * h + 2 * hh].y, a[0][4 * h + 2 * hh + 1].x,
-                        a[0][4 * h + 2 * hh + 1].y);
+            make_float4(a[4 * h + 2 * hh].x, a[4 * h + 2 * hh].y, a[4 * h + 2 * hh + 1].x, a[4 * h + 2 * hh + 1].y);
   }
   group_sync(slot);
   {
     const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
 #pragma unroll
     for (int rb = 0; rb < 32; rb += 2)
-      a[0][rb >> 1] = make_float2(bufBC[base + 32 * rb + 4 * sw], bufBC[base + 32 * (rb + 1) + 4 * (sw ^ 1)]);
+      a[rb >> 1] = make_float2(bufBC[base + 32 * rb + 4 * sw], bufBC[base + 32 * (rb + 1) + 4 * (sw ^ 1)]);
   }
   // pass B: stages 9 .. 5
-  inv_step<9, 4>(a, c0, c1, tb);
-  inv_step<8, 3>(a, c1, c0, tb);
-  inv_step<7, 2>(a, c0, c1, tb);
-  inv_step<6, 1>(a, c1, c0, tb);
-  inv_step<5, 0>(a, c0, c1, tb);
+  inv_step<9, 4, SCALED>(a, c0, c1, tb);
+  inv_step<8, 3, SCALED>(a, c1, c0, tb);
+  inv_step<7, 2, SCALED>(a, c0, c1, tb);
+  inv_step<6, 1, SCALED>(a, c1, c0, tb);
+  inv_step<5, 0, SCALED>(a, c0, c1, tb);
   {
     const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
 #pragma unroll
     for (int rb = 0; rb < 32; rb += 2) {
-      bufAB[base + 32 * rb + 4 * (cq ^ (rb & 7))] = a[0][rb >> 1].x;
-      bufAB[base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))] = a[0][rb >> 1].y;
+      bufAB[base + 32 * rb + 4 * (cq ^ (rb & 7))] = a[rb >> 1].x;
+      bufAB[base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))] = a[rb >> 1].y;
     }
   }
   __syncwarp();  // the B -> A exchange stays inside the warp (position bits 10, 11)
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     const float4 v = *reinterpret_cast<const float4*>(bufAB + tau * 32 + 4 * (c ^ (tau & 7)));
-    a[0][2 * c] = make_float2(v.x, v.y);
-    a[0][2 * c + 1] = make_float2(v.z, v.w);
+    a[2 * c] = make_float2(v.x, v.y);
+    a[2 * c + 1] = make_float2(v.z, v.w);
   }
-  // pass A: stages 4 .. 0, then block 11 again for the next row
-  inv_step<4, 4>(a, c1, c0, tb);
-  inv_step<3, 3>(a, c0, c1, tb);
-  inv_step<2, 2>(a, c1, c0, tb);
-  inv_step<1, 1>(a, c0, c1, tb);
-  tmem_ld32(tb + 32 * 11, c0);
-  stage_inv<0>(a, c1);
+  // pass A: stages 4 .. 0 (double-buffered, the last one loads block 11 of the next row)
+  inv_step<4, 4, SCALED>(a, c1, c0, tb);
+  inv_step<3, 3, SCALED>(a, c0, c1, tb);
+  inv_step<2, 2, SCALED>(a, c1, c0, tb);
+  inv_step<1, 1, SCALED>(a, c0, c1, tb);
+  inv_step<0, 0, SCALED>(a, c1, c0, tb);
+  if constexpr (SCALED) {
+    // output scale of the pass-A positions; then block 11 again for the next row
+    tmem_ld32(tb + kColS, c1);
+    tmem_wait(c1);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) a[q] = __fmul2_rn(a[q], make_float2(u2f(c1[2 * q]), u2f(c1[2 * q + 1])));
+  }
   // pass-A layout output: 32 consecutive positions at 32 tau
   const long long off = row * M + tau * 32;
   if constexpr (sizeof(TO) == 4) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(A.y) + off);
 #pragma unroll
-    for (int c = 0; c < 8; ++c) dst[c] = make_float4(a[0][2 * c].x, a[0][2 * c].y, a[0][2 * c + 1].x, a[0][2 * c + 1].y);
+    for (int c = 0; c < 8; ++c) dst[c] = make_float4(a[2 * c].x, a[2 * c].y, a[2 * c + 1].x, a[2 * c + 1].y);
   } else {
     uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(A.y) + off);
 #pragma unroll
@@ -720,13 +743,12 @@ __device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int nc
       uint32_t w[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        __nv_bfloat162 b = __floats2bfloat162_rn(a[0][4 * c + k].x, a[0][4 * c + k].y);
+        __nv_bfloat162 b = __floats2bfloat162_rn(a[4 * c + k].x, a[4 * c + k].y);
         w[k] = *reinterpret_cast<uint32_t*>(&b);
       }
       dst[c] = make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
-  tmem_wait(c0);
 }
 
 template <typename TI, typename TO>
@@ -735,8 +757,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   __shared__ uint32_t s_tmem;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
-  float* bufAB = smem + slot * (3 * M);
-  float* bufBC = bufAB + M;  // two buffers, used alternately
+  float* bufAB = smem + slot * kSlotFloats;
+  float* bufBC = bufAB + kBufFloats;  // two buffers, used alternately
   const long long G = static_cast<long long>(gridDim.x) * kSlots;
   const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
@@ -752,19 +774,30 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
-  fill_tmem<kImageInvCols / 16>(A.image, tb, slot, tau);
+  fill_tmem<kImageInvCols / 16, kSlots, kFillRound>(A.image, tb, slot, tau);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
 
+  const bool scaled = A.hdr[3] == 1.f;
   uint32_t c0[32], c1[32];
-  tmem_ld32(tb + 32 * 11, c0);
-  tmem_wait(c0);
+  if constexpr (kDoubleBuf) {
+    tmem_ld32(tb + 32 * 11, c0);
+    tmem_wait(c0);
+  }
   // the C -> B buffer alternates between rows (row i's readers and row i+2's
   // writers are kept apart by row i+1's barrier)
+  if (scaled) {
 #pragma unroll 1
-  for (long long row = rb; row < re; ++row)
-    inv_row<TI, TO>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * M, pre, c0, c1);
+    for (long long row = rb; row < re; ++row)
+      inv_row<TI, TO, true>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * kBufFloats,
+                            pre, c0, c1);
+  } else {
+#pragma unroll 1
+    for (long long row = rb; row < re; ++row)
+      inv_row<TI, TO, false>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * kBufFloats,
+                             pre, c0, c1);
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -777,21 +810,20 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
 template <typename TI, typename TO>
 bq_status launch_inv(const FastArgs& A, cudaStream_t st) {
   auto kern = k_inv4096<TI, TO>;
-  const int smem = kSlots * 3 * M * static_cast<int>(sizeof(float));
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
-  static int sms_of[64] = {};
-  if (sms_of[dev] == 0) {
-    int sms = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return BQ_ERR_CUDA;
-    sms_of[dev] = sms;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!once_per_device(ready, dev, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmemBytes) ==
+               cudaSuccess;
+      }))
+    return BQ_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return BQ_ERR_CUDA;
   long long grid = (A.rows + kSlots - 1) / kSlots;
-  if (grid > sms_of[dev]) grid = sms_of[dev];
+  if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, smem, st>>>(A);
+  kern<<<static_cast<unsigned>(grid), kThreads, kFwdSmemBytes, st>>>(A);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 

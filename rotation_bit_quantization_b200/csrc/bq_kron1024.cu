@@ -462,16 +462,15 @@ bq_status kron_launch(const KronArgs& A, cudaStream_t st) {
   auto kern = k_kron1024<TI, MODE, BITS, R>;
   constexpr int smem = kron_smem_bytes<R>();
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
-  static int sms_of[64] = {};
-  if (sms_of[dev] == 0) {
-    int sms = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return BQ_ERR_CUDA;
-    sms_of[dev] = sms;
-  }
-  long long grid = static_cast<long long>(sms_of[dev]) * 4;  // four row CTAs per SM
+  if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!once_per_device(ready, dev, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return BQ_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return BQ_ERR_CUDA;
+  long long grid = static_cast<long long>(sms) * 4;  // four row CTAs per SM
   if (grid > A.rows) grid = A.rows;
   if (grid < 1) grid = 1;
   kern<<<static_cast<unsigned>(grid), kT, smem, st>>>(A);
@@ -739,16 +738,15 @@ bq_status kron_inv_launch(const KronArgs& A, cudaStream_t st) {
   auto kern = k_kron1024_inv<TI, TO, R>;
   constexpr int smem = kron_smem_bytes<R>();
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return BQ_ERR_CUDA;
-  static int sms_of[64] = {};
-  if (sms_of[dev] == 0) {
-    int sms = 0;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-      return BQ_ERR_CUDA;
-    sms_of[dev] = sms;
-  }
-  long long grid = static_cast<long long>(sms_of[dev]) * 4;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!once_per_device(ready, dev, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) == cudaSuccess;
+      }))
+    return BQ_ERR_CUDA;
+  const int sms = device_sm_count(dev);
+  if (sms <= 0) return BQ_ERR_CUDA;
+  long long grid = static_cast<long long>(sms) * 4;
   if (grid > A.rows) grid = A.rows;
   if (grid < 1) grid = 1;
   kern<<<static_cast<unsigned>(grid), kT, smem, st>>>(A);

@@ -19,7 +19,6 @@ namespace bq {
 namespace {
 
 constexpr size_t kScratchBytes = size_t(8) << 20;  // 8 MiB (BQ_NOALLOC_SCRATCH_BYTES)
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scratch[kScratchBytes];
 
@@ -42,9 +41,6 @@ bq_status scratch_for_current_device(void** out) {
   return BQ_OK;
 }
 
-bool valid_width(int m) { return m >= 2 && m <= kMaxM && (m & (m - 1)) == 0; }
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 }  // namespace
 }  // namespace bq
 
@@ -53,17 +49,11 @@ using namespace bq;
 extern "C" bq_status bq_butterfly_bwd_noalloc(const bq_layer* layers, int32_t num_layers, const void* x, bq_dtype xt,
                                               void* y, bq_dtype yt, const float* dy, float* dx, float* dtheta,
                                               int64_t rows_per_layer, void* stream) {
-  if (!layers || num_layers < 1 || num_layers > kMaxBwdLayers) return BQ_ERR_INVALID_ARG;
-  if ((xt != BQ_F32 && xt != BQ_BF16) || (yt != BQ_F32 && yt != BQ_BF16)) return BQ_ERR_INVALID_ARG;
-  const int m = layers[0].m;
+  // the same layer and dtype checks, in the same order, as bq_butterfly_bwd
   KLayer kl[kMaxBwdLayers];
-  for (int l = 0; l < num_layers; ++l) {
-    const bq_layer& L = layers[l];
-    if (!valid_width(L.m) || L.m != m || L.n != L.m || !L.table || !aligned16(L.table)) return BQ_ERR_INVALID_ARG;
-    if (L.r != 1 || L.O != nullptr) return L.r != 1 ? BQ_ERR_UNSUPPORTED : BQ_ERR_INVALID_ARG;
-    kl[l] = make_klayer(L);
-  }
-  if (rows_per_layer < 1) return BQ_ERR_INVALID_ARG;
+  const bq_status s = check_bwd_layers(layers, num_layers, xt, yt, rows_per_layer, kl);
+  if (s != BQ_OK) return s;
+  const int m = layers[0].m;
   const void* ptrs[] = {x, y, dy, dx, dtheta};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return BQ_ERR_INVALID_ARG;

@@ -19,47 +19,48 @@
 //    When any scale leaves [2^-60, 1] or any coefficient exceeds 2^60 (angles
 //    near +-pi/2 chained over many stages), header[0] is cleared and the
 //    kernels use the plain cos/sin form for this layer.
+//  * the same scaled form of the inverse Q^T (stages L-1 .. 0, each rotation by
+//    the negated angle), with its own coefficients, output scale and flag
+//    (header[3]).
 #include "bq_internal.cuh"
 
 namespace bq {
 
 namespace {
 
-__global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ table, TableLayout tl) {
-  extern __shared__ double d[];  // running scale of every position
-  __shared__ int bad;
+// One sweep of the scaled form over all stages: forward (stages 0 .. L-1, angle
+// theta) or inverse (stages L-1 .. 0, angle -theta: the transposed rotation).  The
+// running scale of every position starts at 1 and is multiplied by the pair's
+// cosine at every stage; the coefficients of the pair (i, j) at that stage are
+// alpha = -t d_j / d_i (position i) and beta = t d_i / d_j (position j), with
+// t = tan of the stage's angle (negated for the inverse), both applied to the old
+// values.  Returns (in *bad) 1 when a coefficient exceeds 2^60 or a scale falls
+// below 2^-60 (or is NaN).
+template <typename CS>
+__device__ void scaled_sweep(CS cs_of, const TableLayout& tl, bool inverse, float* __restrict__ fast,
+                             float* __restrict__ sigma, double* d, int* bad) {
   const int m = tl.m, L = tl.L, half = m / 2;
   const int tid = threadIdx.x, T = blockDim.x;
-  float2* cs = reinterpret_cast<float2*>(table + tl.off_cs);
-  float* fast = table + tl.off_fast;
-  float* sigma = table + tl.off_sigma;
-
-  for (int k = tid; k < L * half; k += T) {
-    double sn, c;
-    sincos(static_cast<double>(theta[k]), &sn, &c);
-    cs[k] = make_float2(static_cast<float>(c), static_cast<float>(sn));
-  }
   for (int i = tid; i < m; i += T) d[i] = 1.0;
-  if (tid == 0) bad = 0;
   __syncthreads();
-
   const double kCoefMax = 0x1p60, kScaleMin = 0x1p-60;
-  for (int s = 0; s < L; ++s) {
+  for (int k = 0; k < L; ++k) {
+    const int s = inverse ? L - 1 - k : k;
     for (int p = tid; p < half; p += T) {
       const int lowmask = (1 << s) - 1;
       const int i = ((p >> s) << (s + 1)) | (p & lowmask);
       const int j = i + (1 << s);
       double sn, c;
-      sincos(static_cast<double>(theta[s * half + p]), &sn, &c);
+      cs_of(s, p, sn, c);
       const double di = d[i], dj = d[j];
-      const double t = sn / c;
+      const double t = inverse ? -sn / c : sn / c;
       const double alpha = -t * dj / di;
       const double beta = t * di / dj;
-      if (!(fabs(alpha) <= kCoefMax && fabs(beta) <= kCoefMax)) bad = 1;  // also NaN
+      if (!(fabs(alpha) <= kCoefMax && fabs(beta) <= kCoefMax)) *bad = 1;  // also NaN
       fast[size_t(s) * m + i] = static_cast<float>(alpha);
       fast[size_t(s) * m + j] = static_cast<float>(beta);
       const double ndi = di * c, ndj = dj * c;
-      if (!(fabs(ndi) >= kScaleMin && fabs(ndj) >= kScaleMin)) bad = 1;
+      if (!(fabs(ndi) >= kScaleMin && fabs(ndj) >= kScaleMin)) *bad = 1;
       d[i] = ndi;
       d[j] = ndj;
     }
@@ -67,13 +68,38 @@ __global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ t
   }
   for (int i = tid; i < m; i += T) sigma[i] = static_cast<float>(d[i]);
   __syncthreads();
+}
+
+__device__ __forceinline__ void write_header(float* table, const TableLayout& tl, int bad, int bad_inv) {
+  const int tid = threadIdx.x;
   if (tid < 16) {
     float v = 0.f;
     if (tid == 0) v = bad ? 0.f : 1.f;
-    if (tid == 1) v = static_cast<float>(m);
-    if (tid == 2) v = static_cast<float>(L);
+    if (tid == 1) v = static_cast<float>(tl.m);
+    if (tid == 2) v = static_cast<float>(tl.L);
+    if (tid == 3) v = bad_inv ? 0.f : 1.f;
     table[tid] = v;
   }
+}
+
+__global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ table, TableLayout tl) {
+  extern __shared__ double d[];  // running scale of every position
+  __shared__ int bad, bad_inv;
+  const int half = tl.m / 2;
+  const int tid = threadIdx.x, T = blockDim.x;
+  float2* cs = reinterpret_cast<float2*>(table + tl.off_cs);
+
+  for (int k = tid; k < tl.L * half; k += T) {
+    double sn, c;
+    sincos(static_cast<double>(theta[k]), &sn, &c);
+    cs[k] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+  }
+  if (tid == 0) bad = bad_inv = 0;
+  __syncthreads();
+  auto cs_of = [&](int s, int p, double& sn, double& c) { sincos(static_cast<double>(theta[s * half + p]), &sn, &c); };
+  scaled_sweep(cs_of, tl, false, table + tl.off_fast, table + tl.off_sigma, d, &bad);
+  scaled_sweep(cs_of, tl, true, table + tl.off_fast_inv, table + tl.off_sigma_inv, d, &bad_inv);
+  write_header(table, tl, bad, bad_inv);
 }
 
 // Hadamard presets.  H_n is the butterfly at particular angles (explainer
@@ -85,39 +111,35 @@ __global__ void k_prepare(const float* __restrict__ theta, float* __restrict__ t
 // float64 here (not float32 angles through sincos), so t = s / c is +-1, every
 // coefficient of the scaled form is exactly +-1 (all positions carry the same
 // |scale| at each stage) and the output scale is +-(1/sqrt(2))^L: the forward
-// kernels then compute the butterfly with exact coefficient products.
+// and inverse kernels then compute the butterfly with exact coefficient products.
 __global__ void k_prepare_hadamard(const uint8_t* __restrict__ quadrant, float* __restrict__ table,
                                    float* __restrict__ theta_out, TableLayout tl) {
   extern __shared__ double d[];
-  const int m = tl.m, L = tl.L, half = m / 2;
+  __shared__ int bad, bad_inv;
+  const int half = tl.m / 2;
   const int tid = threadIdx.x, T = blockDim.x;
   float2* cs = reinterpret_cast<float2*>(table + tl.off_cs);
-  float* fast = table + tl.off_fast;
-  float* sigma = table + tl.off_sigma;
   const double r = 0.70710678118654752440;  // 1 / sqrt(2)
   const double kPi = 3.14159265358979323846;
-  for (int i = tid; i < m; i += T) d[i] = 1.0;
-  __syncthreads();
-  for (int s = 0; s < L; ++s) {
-    for (int p = tid; p < half; p += T) {
-      const int k = quadrant ? (quadrant[s * half + p] & 3) : 0;
-      const double c = (k == 0 || k == 3) ? r : -r;   // cos(pi/4 + k pi/2)
-      const double sn = (k <= 1) ? r : -r;            // sin(pi/4 + k pi/2)
-      cs[s * half + p] = make_float2(static_cast<float>(c), static_cast<float>(sn));
-      if (theta_out) theta_out[s * half + p] = static_cast<float>(kPi / 4 + (k < 2 ? k : k - 4) * (kPi / 2));
-      const int i = ((p >> s) << (s + 1)) | (p & ((1 << s) - 1));
-      const int j = i + (1 << s);
-      const double di = d[i], dj = d[j], t = sn / c;
-      fast[size_t(s) * m + i] = static_cast<float>(-t * dj / di);
-      fast[size_t(s) * m + j] = static_cast<float>(t * di / dj);
-      d[i] = di * c;
-      d[j] = dj * c;
-    }
-    __syncthreads();
+  auto cs_of = [&](int s, int p, double& sn, double& c) {
+    const int k = quadrant ? (quadrant[s * half + p] & 3) : 0;
+    c = (k == 0 || k == 3) ? r : -r;   // cos(pi/4 + k pi/2)
+    sn = (k <= 1) ? r : -r;            // sin(pi/4 + k pi/2)
+  };
+  for (int q = tid; q < tl.L * half; q += T) {
+    double sn, c;
+    cs_of(q / half, q % half, sn, c);
+    cs[q] = make_float2(static_cast<float>(c), static_cast<float>(sn));
+    const int k = quadrant ? (quadrant[q] & 3) : 0;
+    if (theta_out) theta_out[q] = static_cast<float>(kPi / 4 + (k < 2 ? k : k - 4) * (kPi / 2));
   }
-  for (int i = tid; i < m; i += T) sigma[i] = static_cast<float>(d[i]);
+  if (tid == 0) bad = bad_inv = 0;
   __syncthreads();
-  if (tid < 16) table[tid] = tid == 0 ? 1.f : tid == 1 ? static_cast<float>(m) : tid == 2 ? static_cast<float>(L) : 0.f;
+  // every coefficient of both sweeps is exactly +-1 (t = +-1 and all positions carry
+  // the same |scale| at each stage), so the range checks always pass
+  scaled_sweep(cs_of, tl, false, table + tl.off_fast, table + tl.off_sigma, d, &bad);
+  scaled_sweep(cs_of, tl, true, table + tl.off_fast_inv, table + tl.off_sigma_inv, d, &bad_inv);
+  write_header(table, tl, bad, bad_inv);
 }
 
 // Position held in register slot e by thread t of a 128-thread row group, for
@@ -135,11 +157,13 @@ __device__ __forceinline__ int pos_pass(int pass, int t, int e) {
 //   columns [160,320): pass 1 stages 5..9
 //   columns [320,384): pass 2 stages 10, 11
 //   columns [384,416): output scale of the 32 positions thread t ends with
+//                      (pass-2 layout for the forward, pass-0 for the inverse)
 // Inside a stage block, column 4q + e (e = 0, 1) is the coefficient of the low
 // element of the thread's (2q + e)-th pair and column 4q + 2 + e that of its
 // high element: (alpha, beta) of the scaled form, or (cos, sin) when the
 // scaled form is out of range (header flag 0; the output scale is then 1).
-// The inverse image (columns [0, 384) only) always holds (cos, sin).
+// The inverse image has the same stage columns, filled from the inverse's own
+// scaled form (header[3]) or with (cos, sin).
 __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
   const bool inv = idx >= kImageLanes * kImageCols;
@@ -147,13 +171,13 @@ __global__ void k_image4096(float* __restrict__ table, TableLayout tl) {
   if (idx >= kImageLanes * (inv ? kImageInvCols : kImageCols)) return;
   const int ncol = inv ? kImageInvCols : kImageCols;
   const int t = idx / ncol, col = idx % ncol;
-  const bool scaled = !inv && table[0] == 1.f;
+  const bool scaled = inv ? table[3] == 1.f : table[0] == 1.f;
   const float2* cs = reinterpret_cast<const float2*>(table + tl.off_cs);
-  const float* fast = table + tl.off_fast;
-  const float* sigma = table + tl.off_sigma;
+  const float* fast = table + (inv ? tl.off_fast_inv : tl.off_fast);
+  const float* sigma = table + (inv ? tl.off_sigma_inv : tl.off_sigma);
   float v;
   if (col >= 384) {
-    v = scaled ? sigma[pos_pass(2, t, col - 384)] : 1.f;
+    v = scaled ? sigma[pos_pass(inv ? 0 : 2, t, col - 384)] : 1.f;
   } else {
     int pass, stage, sb;
     if (col < 160) { pass = 0; stage = col / 32; sb = stage; }

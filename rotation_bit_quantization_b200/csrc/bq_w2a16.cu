@@ -940,7 +940,6 @@ bool encode_2d(CUtensorMap* map, CUtensorMapDataType type, const void* ptr, uint
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 template <int BITS, bool BF16>
 bq_status run_gemm(const CUtensorMap& mx, const CUtensorMap& mc, const GemmArgs& a, int grid, cudaStream_t st) {

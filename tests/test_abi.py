@@ -128,6 +128,32 @@ def test_bwd_rejects_bad_arguments(lib):
     assert lib.bq_butterfly_bwd(kron, 1, *args, ws, None) == _lib.BQ_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("layer,status", [
+    (_layer(64, 64, 0, table=FAKE), _lib.BQ_ERR_INVALID_ARG),          # r = 0
+    (_layer(64 * 9, 64, 9, table=FAKE, O=FAKE), _lib.BQ_ERR_INVALID_ARG),  # r above the limit
+    (_layer(320, 64, 5, table=FAKE, O=FAKE), _lib.BQ_ERR_UNSUPPORTED),  # a valid composite: no backward
+    (_layer(320, 64, 5, table=FAKE), _lib.BQ_ERR_INVALID_ARG),          # r > 1 without O
+    (_layer(64, 64, 1, table=FAKE, O=FAKE), _lib.BQ_ERR_INVALID_ARG),   # O with r == 1
+    (_layer(64, 64, 1, table=FAKE + 4), _lib.BQ_ERR_INVALID_ARG),       # misaligned table
+])
+def test_both_backward_entry_points_reject_bad_layers_alike(lib, layer, status):
+    """The allocation-free backward validates its layers exactly as bq_butterfly_bwd does."""
+    L = (_lib.BQLayer * 1)(layer)
+    args = [FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, 10]
+    ws = 1 << 30
+    assert lib.bq_butterfly_bwd(L, 1, *args, FAKE, ws, None) == status
+    assert lib.bq_butterfly_bwd_noalloc(L, 1, *args, None) == status
+
+
+def test_noalloc_rejects_what_does_not_fit_its_scratch(lib):
+    # 86 layers of width 4096 need more than the 8 MiB of fixed scratch even at one
+    # token chunk per layer (98,304 bytes of partials each); nothing is launched
+    L = (_lib.BQLayer * 86)(*[_layer(4096, 4096, 1, table=FAKE) for _ in range(86)])
+    args = [FAKE, 0, FAKE, 0, FAKE, FAKE, FAKE, 10]
+    assert lib.bq_butterfly_bwd_noalloc(L, 86, *args, None) == _lib.BQ_ERR_WORKSPACE
+    assert lib.bq_butterfly_bwd_noalloc(L, 0, *args, None) == _lib.BQ_ERR_INVALID_ARG
+
+
 def test_precompute_rejects_bad_width(lib):
     assert lib.bq_precompute_cs(FAKE, 12, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
     assert lib.bq_precompute_cs(None, 16, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
