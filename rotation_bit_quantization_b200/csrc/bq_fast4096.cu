@@ -31,11 +31,9 @@
 //    scaled form is out of range (table header flag 0) the same kernel runs the
 //    plain cos/sin rotation instead.
 //  * One CTA per SM (all 512 TMEM columns) with kSlots row groups sharing the
-//    tensor-memory image (warps w, w + 4, ... use the same lanes).  The row is
-//    latency-bound (tensor-memory loads, transposes, the group barrier, the
-//    epilogue's reduction chain), so the kernel trades registers for resident
-//    warps: each thread reads one stage's coefficients at a time
-//    (kDoubleBuf false) and the next row's input is prefetched into registers.
+//    tensor-memory image (warps w, w + 4, ... use the same lanes); each thread
+//    reads the next stage's coefficients while it computes the current one
+//    (kDoubleBuf) and the next row's input is prefetched into registers.
 #include <cfloat>
 
 #include "bq_rtn.cuh"
@@ -50,14 +48,11 @@ constexpr int kFillChunks = kImageCols / 16;  // 26 chunks of 16 columns
 
 // forward kernel: kSlots row groups, each with an A -> B buffer, two alternating
 // B -> C buffers and the epilogue's parameter slots
-#ifndef BQ_FWD_SLOTS
-#define BQ_FWD_SLOTS 4
-#endif
-#ifndef BQ_FWD_DOUBLE_BUF
-#define BQ_FWD_DOUBLE_BUF 0
-#endif
-constexpr int kSlots = BQ_FWD_SLOTS;
-constexpr bool kDoubleBuf = BQ_FWD_DOUBLE_BUF != 0;
+// Three row groups with double-buffered coefficient loads (168 registers) and four
+// with single-buffered loads (128 registers) measured the same at 16384 rows; three
+// were 6% faster at 2048 rows and for the inverse.
+constexpr int kSlots = 3;
+constexpr bool kDoubleBuf = true;
 constexpr int kThreads = kSlots * kGroupThreads;
 constexpr int kBufFloats = M;
 constexpr int kParamFloats = 4 * 32 * 4;  // 4 warps x 32 slots x float4
@@ -66,11 +61,8 @@ constexpr int kFwdSmemBytes = kSlots * kSlotFloats * static_cast<int>(sizeof(flo
 static_assert(kFwdSmemBytes <= 227 * 1024, "shared memory per CTA");
 // image chunks a thread loads per round of the start-up fill: all of its chunks at
 // once where registers allow (three row groups: 9 chunks, 144 registers), four at a
-// time with four row groups (128 registers per thread)
-#ifndef BQ_FILL_ROUND
-#define BQ_FILL_ROUND (kSlots >= 4 ? 4 : (kFillChunks + kSlots - 1) / kSlots)
-#endif
-constexpr int kFillRound = BQ_FILL_ROUND;
+// time with more row groups
+constexpr int kFillRound = kSlots >= 4 ? 4 : (kFillChunks + kSlots - 1) / kSlots;
 
 enum Mode { kOutF32 = 0, kOutBF16 = 1, kQuant = 2 };
 

@@ -35,6 +35,19 @@ struct RtnParams {
   uint16_t scale16, zero16;
 };
 
+// rint(RN(-lo / s)) and rint(RN(hi / s)) of a group's extremes, by the same
+// exact-RTN argument as rtn_codes8 (fast path: one packed FMA pair and the tie
+// test; IEEE division only when either quotient is near a half-integer).
+__device__ __forceinline__ float2 rint_extremes(float lo, float hi, float s, float inv, float thr) {
+  const float2 v = make_float2(-lo, hi);
+  const float2 m2 = make_float2(12582912.f, 12582912.f);   // 1.5 * 2^23
+  const float2 t = __ffma2_rn(v, make_float2(inv, inv), m2);
+  const float2 r = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 e = __ffma2_rn(v, make_float2(-inv, -inv), r);
+  if (fmaxf(fabsf(e.x), fabsf(e.y)) < thr) return r;        // also false for a NaN
+  return make_float2(rintf(__fdiv_rn(-lo, s)), rintf(__fdiv_rn(hi, s)));
+}
+
 __device__ __forceinline__ RtnParams rtn_params(float lo, float hi, float qmax) {
   RtnParams p;
   __half h16 = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), qmax));
@@ -43,14 +56,15 @@ __device__ __forceinline__ RtnParams rtn_params(float lo, float hi, float qmax) 
     s = 1.f;
     h16 = __float2half_rn(1.f);
   }
-  const float zraw = rintf(__fdiv_rn(-lo, s));
-  const float z = __fadd_rn(fminf(fmaxf(zraw, 0.f), qmax), 0.f);  // +0 for a zero point of 0
-  const float inv = __fdiv_rn(1.f, s);
+  const float inv = __frcp_rn(s);  // correctly rounded 1 / s
   const float vmax = fmaxf(fabsf(lo), fabsf(hi)) * inv * 1.000001f;
   const float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
+  const float2 ext = rint_extremes(lo, hi, s, inv, thr);
+  const float zraw = ext.x;
+  const float z = __fadd_rn(fminf(fmaxf(zraw, 0.f), qmax), 0.f);  // +0 for a zero point of 0
   // codes are monotone in y: the group needs no clamping iff its extremes land in
   // [0, qmax]; the bottom is z - rint(-lo / s) (division and rint are odd functions)
-  const bool inrange = zraw <= qmax && __fadd_rn(rintf(__fdiv_rn(hi, s)), z) <= qmax;
+  const bool inrange = zraw <= qmax && __fadd_rn(ext.y, z) <= qmax;
   p.inv = inv;
   p.thr = inrange ? thr : -1.f;
   p.mz = __fadd_rn(12582912.f, z);

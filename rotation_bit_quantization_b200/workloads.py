@@ -169,30 +169,47 @@ def backward_layer_host(layer: int, tokens: int, m: int = 4096) -> Workload:
                     dy=dy.astype(np.float32))
 
 
-def backward_angles(layers: int, m: int = 4096) -> np.ndarray:
-    """Per-layer angles of the backward workload, float32 (layers, log2 m, m/2)."""
-    return np.stack([uniform_angles(np.random.default_rng([5, l, 0]), m) for l in range(layers)])
+def _layer_ids(layers):
+    return list(range(layers)) if isinstance(layers, (int, np.integer)) else [int(l) for l in layers]
 
 
-def backward_inputs_device(layers: int, tokens: int, m: int, device, seed: int = 5):
-    """Device-resident X (layers, tokens, m) bf16 and dY (layers, tokens, m) fp32 drawn with a
-    seeded torch.Generator; t(nu=3) = z / sqrt(chi2_3 / 3) built from normal draws.
+def backward_angles(layers, m: int = 4096) -> np.ndarray:
+    """Per-layer angles of the backward workload, float32 (len, log2 m, m/2), for layers
+    0..layers-1 (an int) or the given layer indices; layer l's angles depend on l only."""
+    return np.stack([uniform_angles(np.random.default_rng([5, l, 0]), m) for l in _layer_ids(layers)])
+
+
+def shard_layers(num_layers: int, world: int, rank: int):
+    """Layer indices of one rank when the backward's independent layers are split across
+    ranks: rank r takes layers r, r + world, r + 2 world, ..."""
+    if world <= 0 or not (0 <= rank < world) or num_layers < 0:
+        raise ValueError("bad world/rank/layers")
+    return list(range(rank, num_layers, world))
+
+
+def backward_inputs_device(layers, tokens: int, m: int, device, seed: int = 5):
+    """Device-resident X (len, tokens, m) bf16 and dY (len, tokens, m) fp32 for layers
+    0..layers-1 (an int) or the given layer indices, drawn with a seeded torch.Generator
+    per layer (layer l's draws depend on seed and l only, so a rank holding a subset of
+    the layers draws exactly those layers of the full workload); t(nu=3) =
+    z / sqrt(chi2_3 / 3) built from normal draws.
 
     Used where host generation of ~50 GB is impractical; callers copy the layers
     they check back to the host.
     """
     import torch
 
+    ids = _layer_ids(layers)
     gen = torch.Generator(device=device)
-    x = torch.empty((layers, tokens, m), dtype=torch.bfloat16, device=device)
-    dy = torch.empty((layers, tokens, m), dtype=torch.float32, device=device)
-    for l in range(layers):
+    x = torch.empty((len(ids), tokens, m), dtype=torch.bfloat16, device=device)
+    dy = torch.empty((len(ids), tokens, m), dtype=torch.float32, device=device)
+    for k, l in enumerate(ids):
         gen.manual_seed(seed * 1_000_003 + l)
         z = torch.randn((tokens, m), generator=gen, device=device)
         c = torch.randn((3, tokens, m), generator=gen, device=device).square_().sum(0).div_(3.0).sqrt_()
-        x[l].copy_(z.div_(c))
+        x[k].copy_(z.div_(c))
         del z, c
-        dy[l].normal_(generator=gen)
+        dy[k].normal_(generator=gen)
     return x, dy
 
 
