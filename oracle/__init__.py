@@ -31,6 +31,12 @@ What it computes, and where the method is stated:
   and the reconstruction loss of a quantized layer with a straight-through
   estimator.  The estimators and smoothing are readings listed in the module
   docstring.
+* ``blockq``     - the block-wise transform of the WUSH workload (WUSH technical
+  summary, section 2: per-block G x G linear transforms of the activations,
+  fused with an AbsMax-scaled round-to-nearest block quantizer in FP or INT
+  formats) and its MXFP4, NVFP4 and symmetric INT4 quantizers; pinned in
+  ``tests/test_oracle_blockq_pins.py`` (dense block-diagonal product, exact
+  rational E2M1 rounding, torch's FP8 E4M3 conversion, brute force, fixtures).
 * ``w2a16``      - the W2A16 consumer GEMM (explainer article, section "training
   & results": 2-bit weights, 16-bit activations; abstract: y = (W Q^T)(Q x)):
   bfloat16 activations times the bfloat16-rounded dequantized codes, summed
