@@ -64,6 +64,10 @@ def workload_spec(name: str):
         return dict(make=None, kind="gemm", rows=2048, n=4096, bits=2, group=128, out_features=11008,
                     label="W2A16 linear: rotated activations 2048 x 4096 bf16 times INT2 g128 weights 11008 x 4096 "
                           "-> 2048 x 11008 bf16 (LLaMA-2-7B MLP up-projection shape)")
+    if name == "wush4096":
+        return dict(make=None, kind="block", rows=2048, n=4096, bits=4, group=32, fmt="mxfp4",
+                    label="block transform + MXFP4: 2048 x 4096 bf16 activations, 128 per-block 32 x 32 transforms "
+                          "(tcgen05), E2M1 codes with E8M0 scales per 32 (WUSH workload shape)")
     if name == "act5120":
         return dict(make=lambda rank: wl.act_5120(8192), kind="quant", rows=8192, n=5120, bits=4, group=128,
                     label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> INT4 RTN g128 (LLaMA-2-13B shape)")
@@ -687,6 +691,136 @@ def oracle_gemm_rate(x_bits, codes, s16, z16, bits, group, tokens_sample):
     return flops / el, el
 
 
+def run_block_bench(args, spec, rank, world, local_rank):
+    """The block transform + MXFP4 quantizer (bq_block_transform_quantize) over a batch of
+    activations, timed like the transform line: K launches in one CUDA graph over input
+    sets cycled so that every step reads an input that is not in L2."""
+    import torch
+    import torch.distributed as dist
+
+    import rotation_bit_quantization_b200 as bq
+    from rotation_bit_quantization_b200 import build as bq_build
+    from rotation_bit_quantization_b200 import workloads as wl
+
+    bq_build.build()
+    bq.load()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    rows, C, G, fmt = spec["rows"], spec["n"], spec["group"], spec["fmt"]
+    w = wl.act_4096(rows, seed_offset=rank)
+    x_host = torch.from_numpy(w.x.view(np.int16)).view(torch.bfloat16)
+    x = x_host.to(dev)
+    Tb = wl.block_transforms(C, G)
+    T = torch.from_numpy(Tb.view(np.int16)).to(dev).view(torch.bfloat16).view(C // G, G, G)
+    bt = bq.BlockTransform(T)
+    out_bytes = C // 2 + C // G
+    set_bytes = rows * (C * 2 + out_bytes)
+    NS = max(2, int(np.ceil(2 * L2_BYTES / set_bytes)))
+    xs = [x] + [x.clone() for _ in range(NS - 1)]
+    outs = [bq.block_outputs(rows, C, fmt, dev) for _ in range(NS)]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        bq.bq_block_transform_quantize(bt, xs[i % NS], fmt, *outs[i % NS], status=status)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream()
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            for i in range(args.steps):
+                step(i)
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id_for(dev))
+    t_busy = time.perf_counter()
+    while time.perf_counter() - t_busy < 0.5:
+        graph.replay()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    graph.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop()
+    del graph
+    if int(status.item()) != 0:
+        raise SystemExit(f"block kernel reported a wait timeout (status {int(status.item())})")
+    t = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item()) / args.steps
+    by_launch = rows * (C * 2 + out_bytes)
+    flops = 2.0 * rows * C * G
+    peaks, peak_src = load_peaks()
+    gbs = by_launch / (ms * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        codes, scales = outs[0]
+        x_pin = x_host.pin_memory()
+        c_pin = torch.empty(codes.shape, dtype=codes.dtype).pin_memory()
+        s_pin = torch.empty(scales.shape, dtype=scales.dtype).pin_memory()
+        x_dev = torch.empty_like(x)
+
+        def e2e_step():
+            x_dev.copy_(x_pin, non_blocking=True)
+            bq.bq_block_transform_quantize(bt, x_dev, fmt, codes, scales, status=status)
+            c_pin.copy_(codes, non_blocking=True)
+            s_pin.copy_(scales, non_blocking=True)
+
+        for _ in range(args.warmup):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        f1.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([f0.elapsed_time(f1) / args.steps], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s",
+               "h2d_bytes_per_step": int(x_pin.numel() * 2),
+               "d2h_bytes_per_step": int(c_pin.numel() + s_pin.numel() * s_pin.element_size())}
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import blockq as obq
+        xs_h = wl.f32_from_bf16_bits(w.x[:256]).astype(np.float64)
+        Tf = wl.f32_from_bf16_bits(Tb).astype(np.float64)
+        t0 = time.perf_counter()
+        obq.quantize(obq.block_transform(Tf, xs_h).astype(np.float32), fmt)
+        el = time.perf_counter() - t0
+        cpu = {"value": 256 / el, "unit": "rows/s", "cores": 1, "kind": "oracle",
+               "sample": f"256 rows (float64 numpy einsum + the MXFP4 quantizer), {el:.2f} s"}
+    return {
+        "metric": "block transform + MXFP4 rows/s, n=4096 (per-block 32 x 32 transforms on tcgen05)",
+        "value": rows * world / (ms * 1e-3), "unit": "rows/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 operands, f32 accumulate", "data": "synthetic (seeded)",
+        "config": {"workload": spec["label"], "rows": rows, "C": C, "G": G, "format": fmt,
+                   "l2": f"inputs larger than L2: {NS} input/output sets cycled ({NS * set_bytes / 1e6:.0f} MB)",
+                   "timing": f"{args.steps} launches in one CUDA graph between two CUDA events"},
+        "gbs": gbs,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None, "peak_source": peak_src,
+                     "algorithmic_bytes_per_launch": by_launch, "algorithmic_flops_per_launch": flops,
+                     "tensor_tflops": flops / (ms * 1e-3) / 1e12, "kernel": "k_blockq<MXFP4, G=32>"},
+        "e2e": e2e, "cpu_baseline": cpu, "gpu_launches": args.steps, "clocks": clocks,
+    }
+
+
 def run_gemm_bench(args, spec, rank, world, local_rank):
     """The W2A16 consumer GEMM (bq_w2a16_gemm) on the LLaMA-2-7B MLP shape."""
     import torch
@@ -898,6 +1032,25 @@ def run_reference(args, spec):
                                "TFLOP/s", statistics.median(rates), el, 1,
                                "256 tokens x 4096 x 11008 per step (float64 numpy, the whole weight matrix dequantized)",
                                {"workload": spec["label"], "tokens": spec["rows"], "out_features": spec["out_features"]})
+    if kind == "block":
+        from oracle import blockq as obq
+        from rotation_bit_quantization_b200 import workloads as wl
+        C, G, fmt = spec["n"], spec["group"], spec["fmt"]
+        Tf = wl.f32_from_bf16_bits(wl.block_transforms(C, G)).astype(np.float64)
+        w = wl.act_4096(256)
+        xs = wl.f32_from_bf16_bits(w.x).astype(np.float64)
+        obq.quantize(obq.block_transform(Tf, xs[:16]).astype(np.float32), fmt)
+        rates = []
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            ts = time.perf_counter()
+            obq.quantize(obq.block_transform(Tf, xs).astype(np.float32), fmt)
+            rates.append(xs.shape[0] / (time.perf_counter() - ts))
+        el = time.perf_counter() - t0
+        return _reference_line(args, spec, "block transform + MXFP4 rows/s, n=4096 (per-block 32 x 32 transforms on tcgen05)",
+                               "rows/s", statistics.median(rates), el, 1,
+                               "256 rows per step (float64 numpy einsum + the MXFP4 quantizer)",
+                               {"workload": spec["label"], "rows": spec["rows"]})
     raise SystemExit(f"no reference arm for workload kind {kind}")
 
 
@@ -910,7 +1063,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="act4096",
-                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity", "w2a16"])
+                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity", "w2a16",
+                             "wush4096"])
     ap.add_argument("--rows", type=int, default=0, help="override the workload's rows (tokens per layer for bwd)")
     ap.add_argument("--layers", type=int, default=0, help="override the backward workload's layer count")
     ap.add_argument("--no-e2e", action="store_true")
@@ -927,7 +1081,7 @@ def main():
         # that has to fit the profiling size rules; never the bench line's size
         from rotation_bit_quantization_b200 import workloads as wl
         rows = args.rows or spec["rows"]
-        if spec["kind"] in ("bwd", "uniformity", "gemm"):
+        if spec["kind"] in ("bwd", "uniformity", "gemm", "block"):
             spec = dict(spec, rows=rows, layers=args.layers or spec.get("layers", 1))
         else:
             base = {"act4096": lambda r, k: wl.act_4096(r, seed_offset=k), "fwd4096": lambda r, k: wl.act_4096(r, seed_offset=k),
@@ -955,6 +1109,8 @@ def main():
             res = run_bwd_bench(args, spec, rank, world, local_rank)
         elif spec["kind"] == "uniformity":
             res = run_uniformity_bench(args, spec, rank, world, local_rank)
+        elif spec["kind"] == "block":
+            res = run_block_bench(args, spec, rank, world, local_rank)
         elif spec["kind"] == "gemm":
             res = run_gemm_bench(args, spec, rank, world, local_rank)
         else:

@@ -292,6 +292,53 @@ bq_status bq_w2a16_linear(const bq_layer* layer, const void* x, bq_dtype xt, int
                           int64_t out_features, int32_t bits, int32_t group, void* out, bq_dtype out_t,
                           void* workspace, size_t workspace_bytes, int32_t* status, void* stream);
 
+/* ---------------------------------------------------------------------------
+ * Block-wise transform fused with AbsMax block quantization (WUSH technical
+ * summary, section 2 "method": per-block G x G linear transforms of the
+ * activations, an AbsMax-scaled round-to-nearest block quantizer in FP and INT
+ * formats; "implementation": the transform fused with activation quantization
+ * on the GPU).  Per row and block b of G channels:
+ *   y[b G + o] = sum_k T[b][o][k] x[b G + k]   (bf16 operands, float32 sums),
+ * then one of:
+ *   BQ_BLOCK_MXFP4 (G = 32): X = floor(log2 max|y|) - 2 clamped to [-127, 127]
+ *     (-127 for an all-zero block), scale byte X + 127 (E8M0); codes
+ *     E2M1(y / 2^X): magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} as codes 0..7, sign
+ *     in bit 3, round to nearest even, saturating at 6;
+ *   BQ_BLOCK_NVFP4 (G = 16): scale = E4M3(max|y| / 6) (round to nearest even,
+ *     saturating at 448), stored as its FP8 byte; codes E2M1(y / (scale *
+ *     gscale)) with the product and the division in IEEE float32 (all +0
+ *     when the scale is 0);
+ *   BQ_BLOCK_INT4 (G = 32): scale16 = fp16(max|y| / 7) (1.0 for an all-zero or
+ *     underflowing block), codes clamp(rint(y / scale), -7, 7) in IEEE float32,
+ *     half to even, as 4-bit two's complement;
+ *   BQ_BLOCK_NONE (G = 16 or 32): y itself, float32 or bfloat16.
+ * Codes are [rows][C / 2] bytes, two per byte, lowest channel in the low nibble;
+ * scales [rows][C / G] (bytes for MXFP4 and NVFP4, fp16 bits for INT4). */
+typedef enum { BQ_BLOCK_NONE = 0, BQ_BLOCK_MXFP4 = 1, BQ_BLOCK_NVFP4 = 2, BQ_BLOCK_INT4 = 3 } bq_block_format;
+
+/* Bytes of the prepared transform table for C channels in blocks of G (16 or 32);
+ * 0 when C is not a positive multiple of 64 or G is not 16 or 32.  Host only. */
+size_t bq_block_table_bytes(int32_t C, int32_t G);
+
+/* Prepare the transform table from T: [C / G][G][G] bfloat16 (T[b][o][k] maps
+ * input channel b G + k to output channel b G + o), device, 2-byte aligned; table:
+ * device, 16-byte aligned, bq_block_table_bytes(C, G) bytes, written with each
+ * 64-channel tile's blocks side by side (the layout the kernel copies).  Async. */
+bq_status bq_block_prepare(const uint16_t* T, int32_t C, int32_t G, uint16_t* table, void* stream);
+
+/* The fused block transform and quantization of x: [rows][C] bfloat16 (device,
+ * 16-byte aligned).  table from bq_block_prepare with the same C and G; format
+ * one of the above with its G; gscale > 0 (NVFP4 only).  BQ_BLOCK_NONE writes
+ * y: [rows][C] of yt (16-byte aligned) and ignores codes / scales; the others
+ * write codes (16-byte aligned) and scales (2-byte aligned).  status: NULL, or a
+ * device int32 the caller zeroes; the kernel ORs a nonzero code into it if any
+ * of its barrier waits gave up after one second (it then stops early and its
+ * outputs are incomplete).  Runs on the tensor cores (tcgen05, operands copied
+ * by the tensor memory accelerator).  Async. */
+bq_status bq_block_transform_quantize(const uint16_t* table, int32_t C, int32_t G, const void* x, int64_t rows,
+                                      bq_block_format format, float gscale, void* y, bq_dtype yt,
+                                      uint8_t* codes, void* scales, int32_t* status, void* stream);
+
 /* The library's last CUDA runtime error (a cudaError_t value, 0 for none),
  * cleared by the call: after BQ_ERR_CUDA it says which CUDA call or launch
  * failed.  Host only; launches nothing. */

@@ -7,7 +7,10 @@ include/bq.h); this package only marshals arguments to it (``_lib``), builds it
 
 from ._lib import (  # noqa: F401
     BQError,
+    BlockTransform,
     Layer,
+    block_outputs,
+    bq_block_transform_quantize,
     bq_butterfly_bwd,
     bq_butterfly_bwd_noalloc,
     bq_butterfly_bwd_workspace_size,

@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(HERE, "libbq.so")
 
 BQ_OK, BQ_ERR_INVALID_ARG, BQ_ERR_UNSUPPORTED, BQ_ERR_WORKSPACE, BQ_ERR_CUDA = range(5)
 BQ_F32, BQ_BF16 = 0, 1
+BQ_BLOCK_NONE, BQ_BLOCK_MXFP4, BQ_BLOCK_NVFP4, BQ_BLOCK_INT4 = range(4)
+BLOCK_FORMATS = {"none": BQ_BLOCK_NONE, "mxfp4": BQ_BLOCK_MXFP4, "nvfp4": BQ_BLOCK_NVFP4, "int4": BQ_BLOCK_INT4}
 
 EXPORTED = (
     "bq_table_floats",
@@ -37,6 +39,9 @@ EXPORTED = (
     "bq_w2a16_gemm_workspace_size",
     "bq_w2a16_linear_workspace_size",
     "bq_w2a16_linear",
+    "bq_block_table_bytes",
+    "bq_block_prepare",
+    "bq_block_transform_quantize",
     "bq_status_string",
     "bq_cuda_last_error",
     "bq_cuda_error_string",
@@ -88,6 +93,9 @@ def load(path: str | None = None):
         "bq_w2a16_gemm_workspace_size": (sz, [i64, i32, i64]),
         "bq_w2a16_linear_workspace_size": (sz, [i32, i64, i64]),
         "bq_w2a16_linear": (i32, [lp, vp, i32, i64, vp, vp, vp, i64, i32, i32, vp, i32, vp, sz, vp, vp]),
+        "bq_block_table_bytes": (sz, [i32, i32]),
+        "bq_block_prepare": (i32, [vp, i32, i32, vp, vp]),
+        "bq_block_transform_quantize": (i32, [vp, i32, i32, vp, i64, i32, ctypes.c_float, vp, i32, vp, vp, vp, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
         "bq_cuda_last_error": (i32, []),
         "bq_cuda_error_string": (ctypes.c_char_p, [i32]),
@@ -361,3 +369,57 @@ def bq_w2a16_linear(layer: Layer, x, codes, scale, zero, bits: int, group: int, 
                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(status),
                                   _stream(stream)))
     return out
+
+
+# ----------------------------------------------------------------------------- block transform + quantize
+
+class BlockTransform:
+    """Per-block G x G transforms of C channels, prepared for the fused kernel.
+
+    T: bfloat16 CUDA tensor (C/G, G, G), T[b, o, k] mapping input channel b G + k to
+    output channel b G + o.  The prepared table (bq_block_prepare) is kept alive here."""
+
+    def __init__(self, T, stream=None):
+        torch = _torch()
+        lib = load()
+        _dev(T, "T")
+        if T.dtype != torch.bfloat16 or T.dim() != 3 or T.shape[1] != T.shape[2]:
+            raise ValueError("T must be bfloat16 of shape (C/G, G, G)")
+        self.G = int(T.shape[1])
+        self.C = int(T.shape[0]) * self.G
+        nbytes = lib.bq_block_table_bytes(self.C, self.G)
+        if nbytes == 0:
+            raise ValueError(f"unsupported block shape C={self.C}, G={self.G}")
+        self.T = T
+        self.table = torch.empty(nbytes // 2, dtype=torch.int16, device=T.device)
+        _check("bq_block_prepare", lib.bq_block_prepare(_ptr(T), self.C, self.G, _ptr(self.table), _stream(stream)))
+
+
+def block_outputs(rows: int, C: int, fmt: str, device):
+    """Empty (codes, scales) tensors of a block-quantized batch."""
+    torch = _torch()
+    G = {"mxfp4": 32, "nvfp4": 16, "int4": 32}[fmt]
+    codes = torch.empty((rows, C // 2), dtype=torch.uint8, device=device)
+    scales = torch.empty((rows, C // G), dtype=torch.int16 if fmt == "int4" else torch.uint8, device=device)
+    return codes, scales
+
+
+def bq_block_transform_quantize(bt: BlockTransform, x, fmt: str, codes=None, scales=None, y=None, gscale: float = 1.0,
+                                status=None, stream=None):
+    """x: bfloat16 (rows, C).  fmt "mxfp4" / "nvfp4" / "int4" writes codes and scales (see
+    block_outputs); "none" writes y (float32 or bfloat16, (rows, C))."""
+    _dev(x, "x")
+    rows = x.numel() // bt.C
+    f = BLOCK_FORMATS[fmt]
+    if f == BQ_BLOCK_NONE:
+        _dev(y, "y")
+        yt = _dtype_code(y)
+    else:
+        _dev(codes, "codes"); _dev(scales, "scales")
+        yt = BQ_F32
+    if status is not None:
+        _dev(status, "status")
+    _check("bq_block_transform_quantize",
+           load().bq_block_transform_quantize(_ptr(bt.table), bt.C, bt.G, _ptr(x), rows, f, float(gscale), _ptr(y), yt,
+                                              _ptr(codes), _ptr(scales), _ptr(status), _stream(stream)))
+    return (y,) if f == BQ_BLOCK_NONE else (codes, scales)

@@ -243,3 +243,12 @@ def w2a16_4096(tokens: int = 2048, out_features: int = 11008, seed: int = 6):
     x = bf16_bits_from_f32((0.5 * student_t(rng, 3.0, (tokens, 4096))).astype(np.float32))
     codes, s16, z16 = packed_weights(np.random.default_rng([seed, 2]), out_features, 4096, 2, 128)
     return x, codes, s16, z16, 2, 128
+
+
+def block_transforms(C: int, G: int, seed: int = 7) -> np.ndarray:
+    """Seeded per-block G x G transforms, bf16 bits (C/G, G, G): identity plus N(0, 0.3^2/G)
+    entries (well conditioned, not orthogonal), standing in for transforms built offline
+    from calibration statistics."""
+    rng = np.random.default_rng([7, seed, C, G])
+    T = np.eye(G)[None] + 0.3 * rng.standard_normal((C // G, G, G)) / np.sqrt(G)
+    return bf16_bits_from_f32(T.astype(np.float32))

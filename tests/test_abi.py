@@ -363,3 +363,30 @@ def test_w2a16_workspace_plan(lib):
     assert lib.bq_w2a16_gemm_workspace_size(0, n, out) == 0
     assert lib.bq_w2a16_gemm_workspace_size(16, 100, out) == 0   # n not a multiple of 64
     assert lib.bq_w2a16_linear_workspace_size(n, 16, out) >= 16 * n * 2 + lib.bq_w2a16_gemm_workspace_size(16, n, out)
+
+
+def test_block_transform_rejects_bad_arguments(lib):
+    f = lib.bq_block_transform_quantize
+    assert lib.bq_block_table_bytes(4096, 32) == 4096 * 32 * 2
+    assert lib.bq_block_table_bytes(100, 32) == 0 and lib.bq_block_table_bytes(4096, 8) == 0
+    assert lib.bq_block_prepare(FAKE, 100, 32, FAKE, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_block_prepare(FAKE, 128, 32, FAKE + 4, None) == _lib.BQ_ERR_INVALID_ARG
+    args = dict(table=FAKE, C=256, G=32, x=FAKE, rows=4, fmt=_lib.BQ_BLOCK_MXFP4, gscale=1.0, y=None, yt=0,
+                codes=FAKE, scales=FAKE, status=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return f(a["table"], a["C"], a["G"], a["x"], a["rows"], a["fmt"], a["gscale"], a["y"], a["yt"], a["codes"],
+                 a["scales"], a["status"], None)
+
+    assert call(fmt=_lib.BQ_BLOCK_NVFP4) == _lib.BQ_ERR_INVALID_ARG            # NVFP4 needs G = 16
+    assert call(G=16, fmt=_lib.BQ_BLOCK_INT4) == _lib.BQ_ERR_INVALID_ARG       # INT4 needs G = 32
+    assert call(C=96) == _lib.BQ_ERR_INVALID_ARG
+    assert call(rows=-1) == _lib.BQ_ERR_INVALID_ARG
+    assert call(codes=None) == _lib.BQ_ERR_INVALID_ARG
+    assert call(x=FAKE + 8) == _lib.BQ_ERR_INVALID_ARG
+    assert call(fmt=_lib.BQ_BLOCK_NONE) == _lib.BQ_ERR_INVALID_ARG             # no y
+    assert call(fmt=_lib.BQ_BLOCK_NONE, y=FAKE, yt=7) == _lib.BQ_ERR_INVALID_ARG
+    assert call(G=16, fmt=_lib.BQ_BLOCK_NVFP4, gscale=0.0) == _lib.BQ_ERR_INVALID_ARG
+    assert call(fmt=9) == _lib.BQ_ERR_INVALID_ARG
+    assert call(rows=0, table=None, x=None) == _lib.BQ_OK                      # empty: nothing launched
