@@ -17,10 +17,10 @@
 //    tcgen05.mma.cta_group::1.kind::f16 (M = 128 rows, N = G outputs, bf16
 //    operands from shared memory, fp32 accumulate) into a tensor-memory
 //    accumulator (64 columns per unit, two accumulators alternating);
-//  * four epilogue warps read the accumulator (thread = row: tcgen05.ld of the
-//    row's 64 outputs), compute each block's absolute maximum and scale in
-//    registers (a quantization group is one thread's run of G values: no
-//    cross-lane reduction) and convert two values per instruction with
+//  * eight epilogue warps read the accumulator (thread = row and half of the 64
+//    columns: tcgen05.ld of 32 outputs), compute each block's absolute maximum
+//    and scale in registers (a quantization group is one thread's run of G
+//    values: no cross-lane reduction) and convert two values per instruction with
 //    cvt.rn.satfinite.e2m1x2.f32 (exact for MXFP4: the division by a power of
 //    two is exact; NVFP4 divides by the E4M3 scale in IEEE float32 first) or
 //    the exact RTN path of the INT4 codes.
@@ -39,19 +39,25 @@ namespace {
 
 constexpr int kBM = 128;   // rows per unit (the MMA's M)
 constexpr int kBC = 64;    // channels per unit (one 128-byte swizzle row of bf16)
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kAStageBytes = kBM * kBC * 2;  // 16 KB
 constexpr int kBStageBytes = 32 * kBC * 2;   // up to G = 32 rows: 4 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;
 constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;  // 1024-byte alignment slack, barriers
-constexpr int kThreads = 192;                      // 4 epilogue warps, TMA warp, MMA warp
-constexpr int kTmaWarp = 4, kMmaWarp = 5;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(16 * kStages + 16 + 16 + 8 + 4 + 4 <= 256, "barrier block");
+constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter: 32 columns each
+constexpr int kThreads = 32 * (kEpiWarps + 2);     // epilogue warps, TMA warp, MMA warp
+constexpr int kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
 constexpr int kTmemCols = 128;                     // two accumulators of 64 columns
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
-// barrier block (byte offsets from kBarOff)
-constexpr int kFull = 0, kEmpty = 32, kAccFull = 64, kAccEmpty = 80, kDrain = 96, kTmemSlot = 104, kAbort = 108;
+// barrier block (byte offsets from kBarOff): a full and an empty barrier per stage,
+// a full and an empty barrier per accumulator, the drain barrier, the TMEM slot and
+// the abort flag
+constexpr int kFull = 0, kEmpty = 8 * kStages, kAccFull = 16 * kStages, kAccEmpty = kAccFull + 16,
+              kDrain = kAccEmpty + 16, kTmemSlot = kDrain + 8, kAbort = kTmemSlot + 4;
 constexpr int kStTma = 1, kStMma = 2, kStEpi = 4, kStDrain = 8;
 
 enum Format { kNone = 0, kMxfp4 = 1, kNvfp4 = 2, kInt4 = 3 };
@@ -168,23 +174,14 @@ __device__ __forceinline__ void tmem_ld32(uint32_t addr, float (&r)[32]) {
       : "r"(addr));
 }
 
-__device__ __forceinline__ void tmem_wait_ld(float (&a)[32], float (&b)[32]) {
+__device__ __forceinline__ void tmem_wait_ld1(float (&a)[32]) {
   uint32_t (&u)[32] = reinterpret_cast<uint32_t (&)[32]>(a);
-  uint32_t (&v)[32] = reinterpret_cast<uint32_t (&)[32]>(b);
   asm volatile("tcgen05.wait::ld.sync.aligned;"
                : "+r"(u[0]), "+r"(u[1]), "+r"(u[2]), "+r"(u[3]), "+r"(u[4]), "+r"(u[5]), "+r"(u[6]), "+r"(u[7]),
                  "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]), "+r"(u[12]), "+r"(u[13]), "+r"(u[14]),
                  "+r"(u[15]), "+r"(u[16]), "+r"(u[17]), "+r"(u[18]), "+r"(u[19]), "+r"(u[20]), "+r"(u[21]),
                  "+r"(u[22]), "+r"(u[23]), "+r"(u[24]), "+r"(u[25]), "+r"(u[26]), "+r"(u[27]), "+r"(u[28]),
                  "+r"(u[29]), "+r"(u[30]), "+r"(u[31])
-               :
-               : "memory");
-  asm volatile(""
-               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
-                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
-                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
-                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
-                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
                :
                : "memory");
 }
@@ -335,13 +332,13 @@ __device__ __forceinline__ void quant_int4(const float* v, uint4& codes, uint32_
 }
 
 template <int FMT, int G>
-__device__ __forceinline__ void epilogue_row(const BlkArgs& a, long long row, int c0, const float* v) {
-  // v: this row's outputs c0 .. c0 + 63
+__device__ __forceinline__ void epilogue_half(const BlkArgs& a, long long row, int c0, const float* v) {
+  // v: this row's outputs c0 .. c0 + 31
   if constexpr (FMT == kNone) {
     if (a.y_bf16) {
       uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + row * a.C + c0);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
+      for (int q = 0; q < 4; ++q) {
         uint32_t w[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -353,23 +350,20 @@ __device__ __forceinline__ void epilogue_row(const BlkArgs& a, long long row, in
     } else {
       float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.y) + row * a.C + c0);
 #pragma unroll
-      for (int q = 0; q < 16; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     }
   } else {
     uint8_t* crow = a.codes + row * (a.C / 2) + c0 / 2;
     const long long srow = row * (a.C / G) + c0 / G;
     if constexpr (FMT == kMxfp4) {
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint4 c;
-        uint32_t sc;
-        quant_mxfp4(v + 32 * g, c, sc);
-        reinterpret_cast<uint4*>(crow)[g] = c;
-        static_cast<uint8_t*>(a.scales)[srow + g] = static_cast<uint8_t>(sc);
-      }
+      uint4 c;
+      uint32_t sc;
+      quant_mxfp4(v, c, sc);
+      *reinterpret_cast<uint4*>(crow) = c;
+      static_cast<uint8_t*>(a.scales)[srow] = static_cast<uint8_t>(sc);
     } else if constexpr (FMT == kNvfp4) {
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
+      for (int g = 0; g < 2; ++g) {
         uint2 c;
         uint32_t sc;
         quant_nvfp4(v + 16 * g, a.gscale, c, sc);
@@ -377,14 +371,11 @@ __device__ __forceinline__ void epilogue_row(const BlkArgs& a, long long row, in
         static_cast<uint8_t*>(a.scales)[srow + g] = static_cast<uint8_t>(sc);
       }
     } else {
-#pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint4 c;
-        uint32_t sc;
-        quant_int4(v + 32 * g, c, sc);
-        reinterpret_cast<uint4*>(crow)[g] = c;
-        static_cast<uint16_t*>(a.scales)[srow + g] = static_cast<uint16_t>(sc);
-      }
+      uint4 c;
+      uint32_t sc;
+      quant_int4(v, c, sc);
+      *reinterpret_cast<uint4*>(crow) = c;
+      static_cast<uint16_t*>(a.scales)[srow] = static_cast<uint16_t>(sc);
     }
   }
 }
@@ -415,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bars + kAccFull + 8 * a, 1);
-      mbar_init(bars + kAccEmpty + 8 * a, 128);
+      mbar_init(bars + kAccEmpty + 8 * a, 32 * kEpiWarps);
     }
     mbar_init(bars + kDrain, 1);
     *abort_flag = 0;
@@ -493,25 +484,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
   } else {
-    // ---------------------------------------------------------------- epilogue (warps 0..3: thread = row)
-    const uint32_t lane_base = static_cast<uint32_t>(32 * warp) << 16;
+    // ---------------------------------------------------------------- epilogue
+    // warp w: rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns 32 (w >> 2) .. + 31
+    const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
+    const int half = warp >> 2;
     int i = 0;
     for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++i) {
       const int acc = i & 1;
       if (!wait_bar(bars + kAccFull + 8 * acc, (i >> 1) & 1, abort_flag, args.status, kStEpi)) break;
       tc_fence_after();
-      float v[64];
-      float (&v0)[32] = *reinterpret_cast<float (*)[32]>(v);
-      float (&v1)[32] = *reinterpret_cast<float (*)[32]>(v + 32);
-      const uint32_t t0 = tmem + lane_base + static_cast<uint32_t>(64 * acc);
-      tmem_ld32(t0, v0);
-      tmem_ld32(t0 + 32, v1);
-      tmem_wait_ld(v0, v1);
+      float v[32];
+      tmem_ld32(tmem + lane_base + static_cast<uint32_t>(64 * acc + 32 * half), v);
+      tmem_wait_ld1(v);
       tc_fence_before();
       mbar_arrive(bars + kAccEmpty + 8 * acc);
       const int rt = u % row_tiles, ct = u / row_tiles;
-      const long long row = static_cast<long long>(rt) * kBM + 32 * warp + lane;
-      if (row < args.rows) epilogue_row<FMT, G>(args, row, ct * kBC, v);
+      const long long row = static_cast<long long>(rt) * kBM + 32 * (warp & 3) + lane;
+      if (row < args.rows) epilogue_half<FMT, G>(args, row, ct * kBC + 32 * half, v);
     }
   }
 
