@@ -8,22 +8,28 @@
 // symmetric INT4 (fp16 scale, G = 32); or written out unquantized.
 //
 // Design (B200, sm_100a): the transform is a dense contraction, so it runs on the
-// tensor cores.  A work unit is 128 rows x 64 channels (64 / G blocks):
-//  * one thread issues the tensor-memory-accelerator copies of the unit's
-//    activation tile (128 x 64 bf16, 128-byte swizzle) and of the blocks'
+// tensor cores.  A work unit is 128 rows x 256 channels, loaded as four
+// 64-channel sub-tiles (the last unit of a row may have fewer):
+//  * one thread issues the tensor-memory-accelerator copies of each sub-tile's
+//    activations (128 x 64 bf16, 128-byte swizzle) and of its blocks'
 //    transforms (G x 64 bf16: the prepared table puts the 64 / G blocks of a
 //    64-channel tile side by side) into a ring of shared-memory stages;
 //  * one thread issues, per block and per 16 channels of K,
 //    tcgen05.mma.cta_group::1.kind::f16 (M = 128 rows, N = G outputs, bf16
 //    operands from shared memory, fp32 accumulate) into a tensor-memory
-//    accumulator (64 columns per unit, two accumulators alternating);
-//  * eight epilogue warps read the accumulator (thread = row and half of the 64
-//    columns: tcgen05.ld of 32 outputs), compute each block's absolute maximum
-//    and scale in registers (a quantization group is one thread's run of G
-//    values: no cross-lane reduction) and convert two values per instruction with
+//    accumulator (256 columns per unit, two accumulators alternating);
+//  * eight (MXFP4) or sixteen (NVFP4, INT4, unquantized output) epilogue warps
+//    read the accumulator (thread = row and a half or a quarter of the unit's
+//    columns: tcgen05.ld of 32 outputs at a time), compute each block's absolute
+//    maximum and scale in registers (a quantization group is one thread's run of
+//    G values: no cross-lane reduction) and write its code bytes of the unit with
+//    32-byte stores and its scales with one store: the wide unit is what
+//    keeps the scale stores few (per-row scale runs of 1 or 2 bytes cost as much
+//    store bandwidth as the codes); they convert two values per instruction with
 //    cvt.rn.satfinite.e2m1x2.f32 (exact for MXFP4: the division by a power of
-//    two is exact; NVFP4 divides by the E4M3 scale in IEEE float32 first) or
-//    the exact RTN path of the INT4 codes.
+//    two is exact; NVFP4 takes the codes of the IEEE float32 quotient by the E4M3
+//    scale through a checked reciprocal product) or the exact RTN path of the INT4
+//    codes.
 // Every barrier wait gives up after one second: the CTA raises its abort flag,
 // records the role in the caller's status word and leaves its loop after the
 // work already issued has completed; the caller checks the status word.
@@ -38,8 +44,13 @@ namespace bq {
 namespace {
 
 constexpr int kBM = 128;   // rows per unit (the MMA's M)
-constexpr int kBC = 64;    // channels per unit (one 128-byte swizzle row of bf16)
-constexpr int kStages = 6;
+constexpr int kBC = 64;    // channels per sub-tile (one 128-byte swizzle row of bf16)
+#ifndef BQ_BLOCK_SUB
+#define BQ_BLOCK_SUB 4
+#endif
+constexpr int kSub = BQ_BLOCK_SUB;  // sub-tiles per unit
+constexpr int kUC = kBC * kSub;    // channels per unit
+constexpr int kStages = 6;         // sub-tile stages
 constexpr int kAStageBytes = kBM * kBC * 2;  // 16 KB
 constexpr int kBStageBytes = 32 * kBC * 2;   // up to G = 32 rows: 4 KB
 constexpr int kStageBytes = kAStageBytes + kBStageBytes;
@@ -47,10 +58,8 @@ constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kSmemBytes = 1024 + kBarOff + 256;  // 1024-byte alignment slack, barriers
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(16 * kStages + 16 + 16 + 8 + 4 + 4 <= 256, "barrier block");
-constexpr int kEpiWarps = 8;                        // two per TMEM lane quarter: 32 columns each
-constexpr int kThreads = 32 * (kEpiWarps + 2);     // epilogue warps, TMA warp, MMA warp
-constexpr int kTmaWarp = kEpiWarps, kMmaWarp = kEpiWarps + 1;
-constexpr int kTmemCols = 128;                     // two accumulators of 64 columns
+constexpr int kTmemCols = 2 * kUC;                 // two accumulators
+static_assert(kTmemCols <= 512 && (kTmemCols & (kTmemCols - 1)) == 0, "tensor memory allocation");
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // barrier block (byte offsets from kBarOff): a full and an empty barrier per stage,
@@ -61,6 +70,21 @@ constexpr int kFull = 0, kEmpty = 8 * kStages, kAccFull = 16 * kStages, kAccEmpt
 constexpr int kStTma = 1, kStMma = 2, kStEpi = 4, kStDrain = 8;
 
 enum Format { kNone = 0, kMxfp4 = 1, kNvfp4 = 2, kInt4 = 3 };
+
+// Epilogue shape per format: warps per TMEM lane quarter (each takes kUC / parts
+// columns of a unit).  MXFP4's codes are cheap (a power-of-two scale, one conversion
+// per two values): two warps per quarter keep up and leave the smaller CTA; the
+// NVFP4 and INT4 epilogues do more arithmetic per value, and the unquantized output
+// more stores, and take four.
+template <int FMT>
+struct Epi {
+  static constexpr int kParts = FMT == kMxfp4 ? 2 : 4;
+  static constexpr int kWarps = 4 * kParts;
+  static constexpr int kCols = kUC / kParts;        // columns of a unit per epilogue thread
+  static constexpr int kChunks = kCols / 32;        // tcgen05.ld of 32 columns each
+  static constexpr int kThreads = 32 * (kWarps + 2);  // epilogue warps, TMA warp, MMA warp
+  static_assert(kChunks >= 1 && kCols % 32 == 0, "epilogue columns");
+};
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -186,6 +210,27 @@ __device__ __forceinline__ void tmem_wait_ld1(float (&a)[32]) {
                : "memory");
 }
 
+// 32-byte store (one full L2 sector); p 32-byte aligned
+__device__ __forceinline__ void st_global_32B(void* p, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+               "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
+// keeps the registers of a chunk loaded before the preceding wait::ld from being
+// read earlier (the wait itself is issued once, by tmem_wait_ld1)
+__device__ __forceinline__ void tmem_bind(float (&a)[32]) {
+  uint32_t (&u)[32] = reinterpret_cast<uint32_t (&)[32]>(a);
+  asm volatile(""
+               : "+r"(u[0]), "+r"(u[1]), "+r"(u[2]), "+r"(u[3]), "+r"(u[4]), "+r"(u[5]), "+r"(u[6]), "+r"(u[7]),
+                 "+r"(u[8]), "+r"(u[9]), "+r"(u[10]), "+r"(u[11]), "+r"(u[12]), "+r"(u[13]), "+r"(u[14]),
+                 "+r"(u[15]), "+r"(u[16]), "+r"(u[17]), "+r"(u[18]), "+r"(u[19]), "+r"(u[20]), "+r"(u[21]),
+                 "+r"(u[22]), "+r"(u[23]), "+r"(u[24]), "+r"(u[25]), "+r"(u[26]), "+r"(u[27]), "+r"(u[28]),
+                 "+r"(u[29]), "+r"(u[30]), "+r"(u[31])
+               :
+               : "memory");
+}
+
 // two float32 -> one byte of two E2M1 codes (hi in bits 4..7), round to nearest even,
 // saturating at +-6
 __device__ __forceinline__ uint32_t e2m1x2(float hi, float lo) {
@@ -220,7 +265,7 @@ __device__ __forceinline__ float absmax(const float* v, int n) {
 
 struct BlkArgs {
   int rows, C, G;
-  int col_tiles, units;
+  int col_tiles, col_units, units;  // 64-channel sub-tiles, units per row tile, all units
   float gscale;           // NVFP4 per-tensor scale
   void* y;                // kNone: [rows][C] float32 or bf16
   int y_bf16;
@@ -251,11 +296,27 @@ __device__ __forceinline__ void quant_mxfp4(const float* v, uint4& codes, uint32
   codes = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// NVFP4: 16 values -> 8 code bytes and the E4M3 scale byte.
+// NVFP4: 16 values -> 8 code bytes and the E4M3 scale byte.  The codes are those of
+// RN32(y / den).  Fast path: q = RN32(y * RN32(1 / den)) is within 1.5 ulp of the
+// correctly rounded quotient (two roundings of relative size 2^-24 each), so when
+// q (1 - 2^-20) and q (1 + 2^-20) receive the same E2M1 code, that code -- the code is
+// monotone in the value -- is also the code of RN32(y / den); elements where the two
+// differ (a quotient within about 2^-20 relative of a rounding boundary of the E2M1
+// grid), and groups whose den or quotients leave the range where those error bounds
+// hold, take IEEE division.
 __device__ __forceinline__ void quant_nvfp4(const float* v, float gscale, uint2& codes, uint32_t& scale) {
   const float amax = absmax(v, 16);
   scale = e4m3_byte(__fdiv_rn(amax, 6.f));
   const float den = __fmul_rn(e4m3_value(scale), gscale);
+  if (den == 0.f) {
+    codes = make_uint2(0u, 0u);
+    return;
+  }
+  const float r = __frcp_rn(den);
+  bool ok = den >= 0x1p-100f && den <= 0x1p100f && amax * r < 0x1p100f;
+  const float2 up = make_float2(1.00000095367431640625f, 1.00000095367431640625f);   // 1 + 2^-20
+  const float2 dn = make_float2(0.99999904632568359375f, 0.99999904632568359375f);   // 1 - 2^-20
+  const float2 r2 = make_float2(r, r);
   uint32_t w[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
@@ -263,54 +324,36 @@ __device__ __forceinline__ void quant_nvfp4(const float* v, float gscale, uint2&
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       const int k = 8 * q + 2 * b;
-      const float hi = den == 0.f ? 0.f : __fdiv_rn(v[k + 1], den);
-      const float lo = den == 0.f ? 0.f : __fdiv_rn(v[k], den);
-      word |= e2m1x2(hi, lo) << (8 * b);
+      const float2 qv = __fmul2_rn(make_float2(v[k], v[k + 1]), r2);
+      const float2 qu = __fmul2_rn(qv, up), qd = __fmul2_rn(qv, dn);
+      const uint32_t cu = e2m1x2(qu.y, qu.x), cd = e2m1x2(qd.y, qd.x);
+      ok = ok && cu == cd;
+      word |= cu << (8 * b);
     }
     w[q] = word;
+  }
+  if (!ok) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int k = 8 * q + 2 * b;
+        word |= e2m1x2(__fdiv_rn(v[k + 1], den), __fdiv_rn(v[k], den)) << (8 * b);
+      }
+      w[q] = word;
+    }
   }
   codes = make_uint2(w[0], w[1]);
 }
 
-// Symmetric INT4 codes of 8 values (two's complement nibbles, lowest element in the
-// lowest bits): rint(y / s) by the exact RTN path of rtn_codes8 with the offset 8
-// (codes 1..15 for -7..7, XOR 8 gives the nibble); IEEE division and clamping when
-// a value is near a tie or the group's extreme lands outside [-7, 7].
-__device__ __noinline__ uint32_t int4sym_codes8_slow(float y0, float y1, float y2, float y3, float y4, float y5,
-                                                     float y6, float y7, float s) {
-  const float y[8] = {y0, y1, y2, y3, y4, y5, y6, y7};
-  uint32_t word = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const float t = fminf(fmaxf(rintf(__fdiv_rn(y[e], s)), -7.f), 7.f);
-    word |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xfu) << (4 * e);
-  }
-  return word;
-}
-
-__device__ __forceinline__ uint32_t int4sym_codes8(const float* y, float inv, float thr, float s) {
-  const float2 iv = make_float2(inv, inv), niv = make_float2(-inv, -inv);
-  const float2 m2 = make_float2(12582920.f, 12582920.f);   // 1.5 * 2^23 + 8
-  const float2 nm2 = make_float2(-12582920.f, -12582920.f);
-  uint32_t b[8];
-  float emax = 0.f;
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float2 yv = make_float2(y[2 * q], y[2 * q + 1]);
-    const float2 t = __ffma2_rn(yv, iv, m2);
-    const float2 r = __fadd2_rn(t, nm2);
-    const float2 e = __ffma2_rn(yv, niv, r);
-    emax = max_nan3(emax, fabsf(e.x), fabsf(e.y));
-    b[2 * q] = __float_as_uint(t.x);
-    b[2 * q + 1] = __float_as_uint(t.y);
-  }
-  uint32_t word = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) word |= ((b[e] & 0xfu) ^ 8u) << (4 * e);
-  if (!(emax < thr)) word = int4sym_codes8_slow(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7], s);
-  return word;
-}
-
+// Symmetric INT4 codes of 32 values (two's complement nibbles, lowest element in the
+// lowest bits): rint(y / s) as in the exact RTN path of the asymmetric quantizer, with
+// the offset 8 (codes 1..15 for -7..7; XOR 8 gives the nibble).  y * inv + (1.5 2^23 + 8)
+// rounds to the integer rint(y inv) + 8 in the low mantissa bits; the residual
+// e = rint - y inv, taken with one rounding, shows how far y inv is from a tie.  The
+// group takes IEEE division and clamping when a residual comes within the error bound
+// of the product of a tie, or the group's extreme lands outside [-7, 7].
 __device__ __forceinline__ void quant_int4(const float* v, uint4& codes, uint32_t& scale16) {
   const float amax = absmax(v, 32);
   __half h16 = __float2half_rn(__fdiv_rn(amax, 7.f));
@@ -325,68 +368,133 @@ __device__ __forceinline__ void quant_int4(const float* v, uint4& codes, uint32_
   float thr = vmax < 4194304.f ? 0.5f - vmax * 9.5367431640625e-7f : -1.f;  // 2^22, 2^-20
   // |y| <= amax: no code leaves [-7, 7] when rint(amax / s) <= 7
   if (!(rintf(__fdiv_rn(amax, s)) <= 7.f)) thr = -1.f;
+  const float2 iv = make_float2(inv, inv), niv = make_float2(-inv, -inv);
+  const float2 m2 = make_float2(12582920.f, 12582920.f);   // 1.5 * 2^23 + 8
+  const float2 nm2 = make_float2(-12582920.f, -12582920.f);
+  float emax = 0.f;
   uint32_t w[4];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) w[q] = int4sym_codes8(v + 8 * q, inv, thr, s);
+  for (int g = 0; g < 4; ++g) {
+    uint32_t b[8];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 yv = make_float2(v[8 * g + 2 * q], v[8 * g + 2 * q + 1]);
+      const float2 t = __ffma2_rn(yv, iv, m2);
+      const float2 rr = __fadd2_rn(t, nm2);
+      const float2 e = __ffma2_rn(yv, niv, rr);
+      emax = max_nan3(emax, fabsf(e.x), fabsf(e.y));
+      b[2 * q] = __float_as_uint(t.x);
+      b[2 * q + 1] = __float_as_uint(t.y);
+    }
+    // low byte of t = rint + 8 in 1..15: two codes per byte, then the four bytes
+    const uint32_t p0 = b[0] + (b[1] << 4), p1 = b[2] + (b[3] << 4);
+    const uint32_t p2 = b[4] + (b[5] << 4), p3 = b[6] + (b[7] << 4);
+    w[g] = __byte_perm(__byte_perm(p0, p1, 0x0040), __byte_perm(p2, p3, 0x0040), 0x5410) ^ 0x88888888u;
+  }
+  if (!(emax < thr)) {
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      uint32_t word = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float t = fminf(fmaxf(rintf(__fdiv_rn(v[8 * g + e], s)), -7.f), 7.f);
+        word |= (static_cast<uint32_t>(static_cast<int>(t)) & 0xfu) << (4 * e);
+      }
+      w[g] = word;
+    }
+  }
   codes = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-template <int FMT, int G>
-__device__ __forceinline__ void epilogue_half(const BlkArgs& a, long long row, int c0, const float* v) {
-  // v: this row's outputs c0 .. c0 + 31
+// 32 outputs -> 16 code bytes and their scales: one byte (MXFP4), two bytes (NVFP4:
+// two groups of 16) or the fp16 bits (INT4)
+template <int FMT>
+__device__ __forceinline__ void chunk_quant(const float* v, float gscale, uint4& codes, uint32_t& scales) {
+  if constexpr (FMT == kMxfp4) {
+    quant_mxfp4(v, codes, scales);
+  } else if constexpr (FMT == kNvfp4) {
+    uint2 c0, c1;
+    uint32_t s0, s1;
+    quant_nvfp4(v, gscale, c0, s0);
+    quant_nvfp4(v + 16, gscale, c1, s1);
+    codes = make_uint4(c0.x, c0.y, c1.x, c1.y);
+    scales = s0 | (s1 << 8);
+  } else {
+    quant_int4(v, codes, scales);
+  }
+}
+
+// One row's outputs c0 .. c0 + 32 nch - 1 (v[c] holds c0 + 32 c ..), nch <= kChunks.
+template <int FMT, int G, int kChunks>
+__device__ __forceinline__ void epilogue_part(const BlkArgs& a, long long row, int c0, float (&v)[kChunks][32],
+                                              int nch) {
   if constexpr (FMT == kNone) {
-    if (a.y_bf16) {
-      uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + row * a.C + c0);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t w[4];
+    for (int c = 0; c < kChunks; ++c) {
+      if (c >= nch) break;
+      if (a.y_bf16) {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.y) + row * a.C + c0 + 32 * c);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * q + 2 * k], v[8 * q + 2 * k + 1]);
-          w[k] = *reinterpret_cast<uint32_t*>(&h);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            __nv_bfloat162 h = __floats2bfloat162_rn(v[c][8 * q + 2 * k], v[c][8 * q + 2 * k + 1]);
+            w[k] = *reinterpret_cast<uint32_t*>(&h);
+          }
+          dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        dst[q] = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    } else {
-      float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.y) + row * a.C + c0);
+      } else {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.y) + row * a.C + c0 + 32 * c);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        for (int q = 0; q < 8; ++q)
+          dst[q] = make_float4(v[c][4 * q], v[c][4 * q + 1], v[c][4 * q + 2], v[c][4 * q + 3]);
+      }
     }
   } else {
-    uint8_t* crow = a.codes + row * (a.C / 2) + c0 / 2;
-    const long long srow = row * (a.C / G) + c0 / G;
-    if constexpr (FMT == kMxfp4) {
-      uint4 c;
-      uint32_t sc;
-      quant_mxfp4(v, c, sc);
-      *reinterpret_cast<uint4*>(crow) = c;
-      static_cast<uint8_t*>(a.scales)[srow] = static_cast<uint8_t>(sc);
-    } else if constexpr (FMT == kNvfp4) {
+    constexpr int kSb = FMT == kMxfp4 ? 1 : 2;   // scale bytes per 32 outputs
+    constexpr int kBytes = kSb * kChunks;
+    uint4* crow = reinterpret_cast<uint4*>(a.codes + row * (a.C / 2) + c0 / 2);
+    uint8_t* sp = static_cast<uint8_t*>(a.scales) + (row * (a.C / G) + c0 / G) * (FMT == kInt4 ? 2 : 1);
+    uint64_t sc = 0;
+    uint4 q[kChunks];
 #pragma unroll
-      for (int g = 0; g < 2; ++g) {
-        uint2 c;
-        uint32_t sc;
-        quant_nvfp4(v + 16 * g, a.gscale, c, sc);
-        reinterpret_cast<uint2*>(crow)[g] = c;
-        static_cast<uint8_t*>(a.scales)[srow + g] = static_cast<uint8_t>(sc);
+    for (int c = 0; c < kChunks; ++c) {
+      if (c >= nch) break;
+      uint32_t s;
+      chunk_quant<FMT>(v[c], a.gscale, q[c], s);
+      sc |= static_cast<uint64_t>(s) << (8 * kSb * c);
+    }
+    // codes: 32-byte stores (whole sectors) where the run allows
+    const bool wide = (reinterpret_cast<uintptr_t>(crow) & 31u) == 0;
+#pragma unroll
+    for (int c = 0; c < kChunks; c += 2) {
+      if (c >= nch) break;
+      if (c + 1 < nch && wide) {
+        st_global_32B(crow + c, q[c], q[c + 1]);
+      } else {
+        crow[c] = q[c];
+        if (c + 1 < nch) crow[c + 1] = q[c + 1];
       }
+    }
+    if (nch == kChunks && (reinterpret_cast<uintptr_t>(sp) & (kBytes - 1)) == 0) {
+      if constexpr (kBytes == 8) *reinterpret_cast<uint64_t*>(sp) = sc;
+      else if constexpr (kBytes == 4) *reinterpret_cast<uint32_t*>(sp) = static_cast<uint32_t>(sc);
+      else if constexpr (kBytes == 2) *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(sc);
+      else *sp = static_cast<uint8_t>(sc);
     } else {
-      uint4 c;
-      uint32_t sc;
-      quant_int4(v, c, sc);
-      *reinterpret_cast<uint4*>(crow) = c;
-      static_cast<uint16_t*>(a.scales)[srow] = static_cast<uint16_t>(sc);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        if (c >= nch) break;
+        if constexpr (kSb == 1) sp[c] = static_cast<uint8_t>(sc >> (8 * c));
+        else reinterpret_cast<uint16_t*>(sp)[c] = static_cast<uint16_t>(sc >> (16 * c));
+      }
     }
   }
 }
 
-// ------------------------------------------------------------------ kernel
-//
-// Work unit u: row tile fastest (consecutive units of a CTA share the transform
-// blocks of one 64-channel tile), then the column tile.
-
 template <int FMT, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Epi<FMT>::kThreads, 1)
     k_blockq(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_t, const BlkArgs args) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -395,6 +503,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t bars = base + kBarOff;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(gbase + kBarOff + kAbort);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + kBarOff + kTmemSlot);
+  using E = Epi<FMT>;
+  constexpr int kTmaWarp = E::kWarps, kMmaWarp = E::kWarps + 1;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row_tiles = (args.rows + kBM - 1) / kBM;
   constexpr uint32_t kTx = kAStageBytes + G * kBC * 2;  // bytes a stage's two copies deliver
@@ -406,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bars + kAccFull + 8 * a, 1);
-      mbar_init(bars + kAccEmpty + 8 * a, 32 * kEpiWarps);
+      mbar_init(bars + kAccEmpty + 8 * a, 32 * E::kWarps);
     }
     mbar_init(bars + kDrain, 1);
     *abort_flag = 0;
@@ -431,18 +541,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---------------------------------------------------------------- loads
     if (lane == 0) {
       uint32_t s = 0, par = 0, issued = 0, last_parity = 0;
-      for (int u = blockIdx.x; u < args.units; u += gridDim.x) {
-        if (!wait_bar(bars + kEmpty + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) break;
-        const int rt = u % row_tiles, ct = u / row_tiles;
-        const uint32_t st = base + s * kStageBytes;
-        mbar_expect_tx(bars + kFull + 8 * s, kTx);
-        tma_2d(st, &map_x, ct * kBC, rt * kBM, bars + kFull + 8 * s);
-        tma_2d(st + kAStageBytes, &map_t, 0, ct * G, bars + kFull + 8 * s);
-        issued |= 1u << s;
-        last_parity = (last_parity & ~(1u << s)) | (par << s);
-        if (++s == kStages) {
-          s = 0;
-          par ^= 1u;
+      bool stop = false;
+      for (int u = blockIdx.x; u < args.units && !stop; u += gridDim.x) {
+        const int rt = u % row_tiles, cu = u / row_tiles;
+        const int nsub = min(kSub, args.col_tiles - kSub * cu);
+        for (int j = 0; j < nsub; ++j) {
+          if (!wait_bar(bars + kEmpty + 8 * s, par ^ 1u, abort_flag, args.status, kStTma)) {
+            stop = true;
+            break;
+          }
+          const int ct = kSub * cu + j;
+          const uint32_t st = base + s * kStageBytes;
+          mbar_expect_tx(bars + kFull + 8 * s, kTx);
+          tma_2d(st, &map_x, ct * kBC, rt * kBM, bars + kFull + 8 * s);
+          tma_2d(st + kAStageBytes, &map_t, 0, ct * G, bars + kFull + 8 * s);
+          issued |= 1u << s;
+          last_parity = (last_parity & ~(1u << s)) | (par << s);
+          if (++s == kStages) {
+            s = 0;
+            par ^= 1u;
+          }
         }
       }
       // copies still in flight land before the CTA exits
@@ -455,28 +573,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       uint32_t s = 0, par = 0;
       int i = 0;
-      for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++i) {
+      bool stop = false;
+      for (int u = blockIdx.x; u < args.units && !stop; u += gridDim.x, ++i) {
         const int acc = i & 1;
         if (!wait_bar(bars + kAccEmpty + 8 * acc, ((i >> 1) & 1) ^ 1, abort_flag, args.status, kStMma)) break;
-        if (!wait_bar(bars + kFull + 8 * s, par, abort_flag, args.status, kStMma)) break;
-        tc_fence_after();
-        const uint32_t st = base + s * kStageBytes;
-        const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + kAStageBytes);
-        const uint32_t d0 = tmem + static_cast<uint32_t>(64 * acc);
+        const int nsub = min(kSub, args.col_tiles - kSub * (u / row_tiles));
+        for (int j = 0; j < nsub; ++j) {
+          if (!wait_bar(bars + kFull + 8 * s, par, abort_flag, args.status, kStMma)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = base + s * kStageBytes;
+          const uint64_t ad = sw128_desc(st), bd = sw128_desc(st + kAStageBytes);
+          const uint32_t d0 = tmem + static_cast<uint32_t>(kUC * acc + kBC * j);
 #pragma unroll
-        for (int b = 0; b < kBC / G; ++b) {
+          for (int b = 0; b < kBC / G; ++b) {
 #pragma unroll
-          for (int kk = 0; kk < G / 16; ++kk) {
-            const uint64_t koff = static_cast<uint64_t>((b * G + 16 * kk) * 2 / 16);  // +32 bytes per 16 of K
-            umma_ss(d0 + static_cast<uint32_t>(b * G), ad + koff, bd + koff, args.idesc, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < G / 16; ++kk) {
+              const uint64_t koff = static_cast<uint64_t>((b * G + 16 * kk) * 2 / 16);  // +32 bytes per 16 of K
+              umma_ss(d0 + static_cast<uint32_t>(b * G), ad + koff, bd + koff, args.idesc, kk > 0 ? 1u : 0u);
+            }
+          }
+          umma_commit(bars + kEmpty + 8 * s);
+          if (++s == kStages) {
+            s = 0;
+            par ^= 1u;
           }
         }
-        umma_commit(bars + kEmpty + 8 * s);
+        if (stop) break;
         umma_commit(bars + kAccFull + 8 * acc);
-        if (++s == kStages) {
-          s = 0;
-          par ^= 1u;
-        }
       }
       // every MMA issued has completed before the tensor memory is freed
       umma_commit(bars + kDrain);
@@ -485,22 +611,30 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    // warp w: rows 32 (w & 3) .. + 31 (its TMEM lane quarter), columns 32 (w >> 2) .. + 31
+    // warp w: rows 32 (w & 3) .. + 31 (its TMEM lane quarter), the unit's columns
+    // E::kCols (w >> 2) .. + E::kCols - 1
     const uint32_t lane_base = static_cast<uint32_t>(32 * (warp & 3)) << 16;
-    const int half = warp >> 2;
+    const int part = warp >> 2;
     int i = 0;
     for (int u = blockIdx.x; u < args.units; u += gridDim.x, ++i) {
       const int acc = i & 1;
       if (!wait_bar(bars + kAccFull + 8 * acc, (i >> 1) & 1, abort_flag, args.status, kStEpi)) break;
       tc_fence_after();
-      float v[32];
-      tmem_ld32(tmem + lane_base + static_cast<uint32_t>(64 * acc + 32 * half), v);
-      tmem_wait_ld1(v);
+      const int rt = u % row_tiles, cu = u / row_tiles;
+      const int valid = kBC * min(kSub, args.col_tiles - kSub * cu) - E::kCols * part;  // warp-uniform
+      const int nch = valid <= 0 ? 0 : min(E::kChunks, valid / 32);
+      float v[E::kChunks][32];
+      const uint32_t t0 = tmem + lane_base + static_cast<uint32_t>(kUC * acc + E::kCols * part);
+#pragma unroll
+      for (int c = 0; c < E::kChunks; ++c)
+        if (c < nch) tmem_ld32(t0 + 32 * c, v[c]);
+      tmem_wait_ld1(v[0]);
+#pragma unroll
+      for (int c = 1; c < E::kChunks; ++c) tmem_bind(v[c]);
       tc_fence_before();
       mbar_arrive(bars + kAccEmpty + 8 * acc);
-      const int rt = u % row_tiles, ct = u / row_tiles;
       const long long row = static_cast<long long>(rt) * kBM + 32 * (warp & 3) + lane;
-      if (row < args.rows) epilogue_half<FMT, G>(args, row, ct * kBC + 32 * half, v);
+      if (row < args.rows && nch > 0) epilogue_part<FMT, G, E::kChunks>(args, row, kUC * cu + E::kCols * part, v, nch);
     }
   }
 
@@ -566,7 +700,7 @@ bq_status run(const CUtensorMap& mx, const CUtensorMap& mt, const BlkArgs& a, in
         return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes) == cudaSuccess;
       }))
     return BQ_ERR_CUDA;
-  kern<<<grid, kThreads, kSmemBytes, st>>>(mx, mt, a);
+  kern<<<grid, Epi<FMT>::kThreads, kSmemBytes, st>>>(mx, mt, a);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -624,7 +758,8 @@ extern "C" bq_status bq_block_transform_quantize(const uint16_t* table, int32_t 
   a.C = C;
   a.G = G;
   a.col_tiles = C / kBC;
-  const long long units = ((rows + kBM - 1) / kBM) * static_cast<long long>(a.col_tiles);
+  a.col_units = (a.col_tiles + kSub - 1) / kSub;
+  const long long units = ((rows + kBM - 1) / kBM) * static_cast<long long>(a.col_units);
   if (units > 0x7fffffffLL) return BQ_ERR_UNSUPPORTED;
   a.units = static_cast<int>(units);
   a.gscale = gscale;
