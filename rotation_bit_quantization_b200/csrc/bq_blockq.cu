@@ -254,11 +254,41 @@ __device__ __forceinline__ float e4m3_value(uint32_t byte) {
   return __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xffffu)));
 }
 
-__device__ __forceinline__ float absmax(const float* v, int n) {
-  float m = 0.f;
+// eight float32 -> four bytes of E2M1 code pairs (element 2k in the low nibble of
+// byte k), round to nearest even, saturating at +-6
+__device__ __forceinline__ uint32_t e2m1x8(float2 a, float2 b, float2 c, float2 d) {
+  uint32_t w;
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+      " mov.b32 %0, {b0, b1, b2, b3};\n}"
+      : "=r"(w)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y), "f"(d.x), "f"(d.y));
+  return w;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// largest |v[k]| of N values (N even, N >= 8): three-input maxima in two chains
+template <int N>
+__device__ __forceinline__ float absmax(const float* v) {
+  float m0 = max3f(fabsf(v[0]), fabsf(v[1]), fabsf(v[2]));
+  float m1 = max3f(fabsf(v[3]), fabsf(v[4]), fabsf(v[5]));
+  int k = 6;
 #pragma unroll
-  for (int k = 0; k < n; k += 2) m = fmaxf(m, fmaxf(fabsf(v[k]), fabsf(v[k + 1])));
-  return m;
+  for (; k + 4 <= N; k += 4) {
+    m0 = max3f(m0, fabsf(v[k]), fabsf(v[k + 1]));
+    m1 = max3f(m1, fabsf(v[k + 2]), fabsf(v[k + 3]));
+  }
+#pragma unroll
+  for (; k < N; k += 2) m0 = max3f(m0, fabsf(v[k]), fabsf(v[k + 1]));
+  return fmaxf(m0, m1);
 }
 
 // ------------------------------------------------------------------ epilogue: one row's 64 outputs
@@ -277,21 +307,18 @@ struct BlkArgs {
 
 // MXFP4: 32 values -> 16 code bytes and the E8M0 scale byte.
 __device__ __forceinline__ void quant_mxfp4(const float* v, uint4& codes, uint32_t& scale) {
-  const float amax = absmax(v, 32);
+  const float amax = absmax<32>(v);
   const int biased = static_cast<int>((__float_as_uint(amax) >> 23) & 0xffu);
   const int X = biased - 129 > -127 ? biased - 129 : -127;   // floor(log2 amax) - 2, at least -127
   scale = static_cast<uint32_t>(X + 127);
   const float inv = __uint_as_float(static_cast<uint32_t>(127 - X) << 23);  // 2^-X, exact
+  const float2 iv = make_float2(inv, inv);
   uint32_t w[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
-    uint32_t word = 0;
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int k = 8 * q + 2 * b;
-      word |= e2m1x2(v[k + 1] * inv, v[k] * inv) << (8 * b);
-    }
-    w[q] = word;
+    const float* p = v + 8 * q;
+    w[q] = e2m1x8(__fmul2_rn(make_float2(p[0], p[1]), iv), __fmul2_rn(make_float2(p[2], p[3]), iv),
+                  __fmul2_rn(make_float2(p[4], p[5]), iv), __fmul2_rn(make_float2(p[6], p[7]), iv));
   }
   codes = make_uint4(w[0], w[1], w[2], w[3]);
 }
@@ -305,7 +332,7 @@ __device__ __forceinline__ void quant_mxfp4(const float* v, uint4& codes, uint32
 // grid), and groups whose den or quotients leave the range where those error bounds
 // hold, take IEEE division.
 __device__ __forceinline__ void quant_nvfp4(const float* v, float gscale, uint2& codes, uint32_t& scale) {
-  const float amax = absmax(v, 16);
+  const float amax = absmax<16>(v);
   scale = e4m3_byte(__fdiv_rn(amax, 6.f));
   const float den = __fmul_rn(e4m3_value(scale), gscale);
   if (den == 0.f) {
@@ -320,17 +347,15 @@ __device__ __forceinline__ void quant_nvfp4(const float* v, float gscale, uint2&
   uint32_t w[2];
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
-    uint32_t word = 0;
+    float2 qu[4], qd[4];
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      const int k = 8 * q + 2 * b;
-      const float2 qv = __fmul2_rn(make_float2(v[k], v[k + 1]), r2);
-      const float2 qu = __fmul2_rn(qv, up), qd = __fmul2_rn(qv, dn);
-      const uint32_t cu = e2m1x2(qu.y, qu.x), cd = e2m1x2(qd.y, qd.x);
-      ok = ok && cu == cd;
-      word |= cu << (8 * b);
+      const float2 qv = __fmul2_rn(make_float2(v[8 * q + 2 * b], v[8 * q + 2 * b + 1]), r2);
+      qu[b] = __fmul2_rn(qv, up);
+      qd[b] = __fmul2_rn(qv, dn);
     }
-    w[q] = word;
+    w[q] = e2m1x8(qu[0], qu[1], qu[2], qu[3]);
+    ok = ok && w[q] == e2m1x8(qd[0], qd[1], qd[2], qd[3]);
   }
   if (!ok) {
 #pragma unroll
@@ -355,7 +380,7 @@ __device__ __forceinline__ void quant_nvfp4(const float* v, float gscale, uint2&
 // group takes IEEE division and clamping when a residual comes within the error bound
 // of the product of a tie, or the group's extreme lands outside [-7, 7].
 __device__ __forceinline__ void quant_int4(const float* v, uint4& codes, uint32_t& scale16) {
-  const float amax = absmax(v, 32);
+  const float amax = absmax<32>(v);
   __half h16 = __float2half_rn(__fdiv_rn(amax, 7.f));
   float s = __half2float(h16);
   if (amax == 0.f || s == 0.f) {
