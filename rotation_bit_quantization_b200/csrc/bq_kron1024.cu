@@ -51,7 +51,9 @@ struct KronArgs {
   const float* fast;    // [10][1024] scaled-form coefficients
   const float* sigma;   // [1024]
   const float2* cs;     // [10][512] cos, sin
-  const float* hdr;     // header: hdr[0] == 1 when the scaled form is usable
+  const float* fast_inv;   // [10][1024] scaled-form coefficients of the inverse
+  const float* sigma_inv;  // [1024]
+  const float* hdr;     // header: hdr[0] (hdr[3]) == 1 when the scaled form (inverse) is usable
   const float* O;       // [R][R]
   uint8_t* codes;
   uint16_t* scale;
@@ -486,13 +488,19 @@ bq_status kron_dispatch(const KronArgs& A, bq_dtype yt, const QuantArgs* q, cuda
 
 // ------------------------------------------------------------------ inverse
 //
-// x = (B_1024^T (x) O_R^T) y: the forward's layouts visited backwards with plain
-// cos/sin (the scaled form's steps do not invert into steps of the same shape).
-// The row is read in element-order chunks into shared memory and picked up in
-// pass-2 layout; stage 9 runs across lanes, stages 8..0 in registers with the
-// exchanges reversed; O_R^T is applied in pass 0, which stores contiguously.
-// Tensor-memory columns: 8 s for register stage s (cos, sin), 72 + e / 80 + e the
-// stage-9 (cos, -+sin) of element e: y = k1 x + k2 x'.
+// x = (B_1024^T (x) O_R^T) y: the forward's layouts visited backwards.  B^T is the
+// butterfly of the transposed rotations with the stages in reverse order, so it has
+// a scaled form of its own (the table's fast_inv / sigma_inv, prepared by the same
+// sweep over stages 9 .. 0): every stage is then two FMAs per pair, with sigma_inv
+// applied after stage 0.  When the table's inverse flag is clear the kernel runs
+// the plain cos/sin rotations.  The row is read in element-order chunks into shared
+// memory and picked up in pass-2 layout; stage 9 runs across lanes, stages 8..0 in
+// registers with the exchanges reversed; O_R^T is applied in pass 0, which stores
+// contiguously.
+// Tensor-memory columns: 8 s for register stage s, 80 + e the stage-9 coefficient
+// k2 of element e (pass-2 layout) and 72 + e either the stage-9 k1 (plain:
+// y = k1 x + k2 x', k1 = cos, k2 = +-sin) or, scaled (y = x + k2 x'), sigma_inv of
+// pass-0 element e.
 
 template <int SB, int R>
 __device__ __forceinline__ void stage_inv(float2 (&a)[R][4], const uint32_t (&c)[8]) {
@@ -559,6 +567,7 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
   float* xbuf = smem;              // [R][kPlane]
   float* nat = xbuf + R * kPlane;  // [N + 16]
   const int tau = threadIdx.x, l = tau & 31, w = tau >> 5;
+  const bool scaled = A.hdr[3] == 1.f;
 
   if (w == 0) {
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
@@ -574,10 +583,16 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
       uint32_t c[8];
 #pragma unroll
       for (int pr = 0; pr < 4; ++pr) {
-        const int ilo = pos_pass(P, tau, e_low(pr, SB));
-        const float2 t = A.cs[s * (M1 / 2) + (((ilo >> (s + 1)) << s) | (ilo & ((1 << s) - 1)))];
-        c[pr] = __float_as_uint(t.x);
-        c[4 + pr] = __float_as_uint(t.y);
+        const int elo = e_low(pr, SB);
+        const int ilo = pos_pass(P, tau, elo);
+        if (scaled) {
+          c[pr] = __float_as_uint(A.fast_inv[s * M1 + ilo]);
+          c[4 + pr] = __float_as_uint(A.fast_inv[s * M1 + pos_pass(P, tau, elo | (1 << SB))]);
+        } else {
+          const float2 t = A.cs[s * (M1 / 2) + (((ilo >> (s + 1)) << s) | (ilo & ((1 << s) - 1)))];
+          c[pr] = __float_as_uint(t.x);
+          c[4 + pr] = __float_as_uint(t.y);
+        }
       }
       tst8(tb + 8 * s, c);
     }
@@ -585,9 +600,14 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       const int i1 = pos_pass(2, tau, e);
-      const float2 t = A.cs[9 * (M1 / 2) + (i1 & 511)];
-      k1[e] = __float_as_uint(t.x);
-      k2[e] = __float_as_uint(((i1 >> 9) & 1) ? -t.y : t.y);
+      if (scaled) {
+        k1[e] = __float_as_uint(A.sigma_inv[pos_pass(0, tau, e)]);
+        k2[e] = __float_as_uint(A.fast_inv[9 * M1 + i1]);
+      } else {
+        const float2 t = A.cs[9 * (M1 / 2) + (i1 & 511)];
+        k1[e] = __float_as_uint(t.x);
+        k2[e] = __float_as_uint(((i1 >> 9) & 1) ? -t.y : t.y);
+      }
     }
     tst8(tb + 72, k1);
     tst8(tb + 80, k2);
@@ -615,7 +635,9 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
   twait(ca);
 
 #define KISTEP(S, SB, CUR, NXT) \
-  tld8(tb + 8 * ((S) - 1), NXT); stage_inv<SB, R>(a, CUR); twait(NXT)
+  tld8(tb + 8 * ((S) - 1), NXT); \
+  if (scaled) stage<SB, true, R>(a, CUR); else stage_inv<SB, R>(a, CUR); \
+  twait(NXT)
 
 #pragma unroll 1
   for (long long row = blockIdx.x; row < A.rows; row += gridDim.x) {
@@ -641,8 +663,11 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
       for (int r = 0; r < R; ++r) {
         const float x0 = nat[nb + 64 * R * (2 * k) + r], x1 = nat[nb + 64 * R * (2 * k + 1) + r];
         const float p0 = __shfl_xor_sync(0xffffffffu, x0, 16), p1 = __shfl_xor_sync(0xffffffffu, x1, 16);
-        a[r][k] = make_float2(fmaf(u2f(ca[2 * k]), p0, u2f(cn[2 * k]) * x0),
-                              fmaf(u2f(ca[2 * k + 1]), p1, u2f(cn[2 * k + 1]) * x1));
+        if (scaled)
+          a[r][k] = make_float2(fmaf(u2f(ca[2 * k]), p0, x0), fmaf(u2f(ca[2 * k + 1]), p1, x1));
+        else
+          a[r][k] = make_float2(fmaf(u2f(ca[2 * k]), p0, u2f(cn[2 * k]) * x0),
+                                fmaf(u2f(ca[2 * k + 1]), p1, u2f(cn[2 * k + 1]) * x1));
       }
     tld8(tb + 64, ca);
     twait(ca);
@@ -680,9 +705,20 @@ __global__ void __launch_bounds__(kT, 4) k_kron1024_inv(const KronArgs A) {
       a[r][3] = make_float2(v.z, v.w);
     }
     KISTEP(2, 2, ca, cn); KISTEP(1, 1, cn, ca);
-    stage_inv<0, R>(a, ca);
-    tld8(tb + 72, cn);  // stage 9 of the next row
-    tld8(tb + 80, ca);
+    tld8(tb + 72, cn);  // sigma_inv (scaled) or stage 9's k1 of the next row (plain)
+    if (scaled) {
+      stage<0, true, R>(a, ca);
+      twait(cn);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 sg = make_float2(u2f(cn[2 * k]), u2f(cn[2 * k + 1]));
+#pragma unroll
+        for (int r = 0; r < R; ++r) a[r][k] = __fmul2_rn(a[r][k], sg);
+      }
+    } else {
+      stage_inv<0, R>(a, ca);
+    }
+    tld8(tb + 80, ca);  // stage 9's k2 of the next row
 
     // O_R^T on every group of R, then the pass-0 elements (contiguous) to memory
     float2 out[R][4];
@@ -769,6 +805,8 @@ bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, 
   A.rows = rows;
   A.fast = L.fast;
   A.sigma = L.sigma;
+  A.fast_inv = L.fast_inv;
+  A.sigma_inv = L.sigma_inv;
   A.cs = L.cs;
   A.hdr = L.hdr;
   A.O = L.O;
@@ -787,6 +825,8 @@ bq_status launch_kron1024_inv(const KLayer& L, const void* y, bq_dtype yt, void*
   A.rows = rows;
   A.fast = L.fast;
   A.sigma = L.sigma;
+  A.fast_inv = L.fast_inv;
+  A.sigma_inv = L.sigma_inv;
   A.cs = L.cs;
   A.hdr = L.hdr;
   A.O = L.O;

@@ -594,18 +594,36 @@ def test_kron5120_quant_groups(bq, bits, group):
 
 
 def test_kron5120_plain_form_fallback(bq):
-    """Angles whose scaled form leaves its range: the kernel's cos/sin path."""
+    """Angles whose scaled forms (forward and inverse) leave their range: the kernels'
+    cos/sin paths."""
     torch = H.torch()
     theta = np.full((10, 512), np.float32(np.pi / 2), np.float32)
     theta[:, ::3] = np.float32(0.3)
     O = wl.random_orthogonal(np.random.default_rng(3), 5)
     layer = make_layer(bq, theta, O)
-    assert not layer.fast_form
+    assert not layer.fast_form and not layer.fast_form_inverse
     x = np.random.default_rng(4).standard_normal((11, 5120)).astype(np.float32)
     y = run_fwd(bq, layer, H.dev_f32(x), torch.float32)
     ref = ob.kron_forward(theta, O.astype(np.float64), x.astype(np.float64), 1024)
     H.assert_f32_close(H.host(y), ref, x.astype(np.float64))
     check_quant(bq, layer, H.dev_f32(x), x.astype(np.float64), theta, 4, 128, O=O.astype(np.float64), m=1024)
+    ys = np.random.default_rng(5).standard_normal((13, 5120)).astype(np.float32)
+    ref_i = ob.kron_inverse(theta, O.astype(np.float64), ys.astype(np.float64), 1024)
+    x32 = torch.empty((13, 5120), dtype=torch.float32, device="cuda")
+    xb = torch.empty((13, 5120), dtype=torch.bfloat16, device="cuda")
+    bq.bq_butterfly_inv(layer, H.dev_f32(ys), x32)
+    bq.bq_butterfly_inv(layer, H.dev_f32(ys), xb)
+    torch.cuda.synchronize()
+    H.assert_f32_close(H.host(x32), ref_i, ys.astype(np.float64))
+    H.assert_bf16_output(H.host(xb), H.host(x32), ref_i, ys.astype(np.float64))
+
+
+def test_kron5120_inverse_uses_scaled_form(bq):
+    """Uniform angles: both scaled forms are in range, so the n = 5120 inverse runs the
+    two-FMA form of the transposed butterfly with its own output scale."""
+    theta, O, _ = _kron_case(41, 1)
+    layer = make_layer(bq, theta, O)
+    assert layer.fast_form and layer.fast_form_inverse
 
 
 def test_kron5120_exact_ties(bq):
