@@ -154,6 +154,10 @@ bq_status bq_butterfly_bwd(const bq_layer* layers, int32_t num_layers,
  * (num_layers * log2(m) * m/2 * 4 bytes + 512 > BQ_NOALLOC_SCRATCH_BYTES,
  * e.g. more than 85 layers of width 4096) it returns BQ_ERR_WORKSPACE and
  * launches nothing.  Nothing is allocated: no cudaMalloc, no cudaFree.
+ * Fewer chunks also mean fewer CTAs: at width 4096 the scratch holds 85
+ * (layer, chunk) slots, so at most 85 SMs work (32 layers get 64 CTAs, two
+ * chunks per layer) and the call takes about 2.3 times as long as
+ * bq_butterfly_bwd with a full-size workspace on a 148-SM B200.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
  * capture.  Every call shares the one array and clears the part that must

@@ -28,19 +28,22 @@ def bq():
 
 
 class Guarded:
-    """A device tensor of `shape`/`dtype` with sentinel-filled bands on both sides."""
+    """A device tensor of `shape`/`dtype` with sentinel-filled bands on both sides; `shift`
+    moves its start by that many bytes (to test outputs that meet only the documented
+    minimum alignment)."""
 
-    def __init__(self, shape, dtype):
+    def __init__(self, shape, dtype, shift=0):
         torch = H.torch()
         nbytes = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
         self.nbytes = nbytes
-        self.buf = torch.full((2 * PAD + nbytes,), SENTINEL, dtype=torch.uint8, device="cuda")
-        self.t = self.buf[PAD:PAD + nbytes].view(dtype).view(shape)
+        self.lo = PAD + shift
+        self.buf = torch.full((2 * PAD + nbytes + shift,), SENTINEL, dtype=torch.uint8, device="cuda")
+        self.t = self.buf[self.lo:self.lo + nbytes].view(dtype).view(shape)
 
     def check(self, name):
         b = self.buf.cpu().numpy()
-        assert np.all(b[:PAD] == SENTINEL), f"{name}: write before the buffer"
-        assert np.all(b[PAD + self.nbytes:] == SENTINEL), f"{name}: write past the end"
+        assert np.all(b[:self.lo] == SENTINEL), f"{name}: write before the buffer"
+        assert np.all(b[self.lo + self.nbytes:] == SENTINEL), f"{name}: write past the end"
 
 
 def _snap(*ts):
@@ -195,3 +198,36 @@ def test_hadamard_preset_stays_in_bounds(bq):
     torch.cuda.synchronize()
     table.check("table")
     theta.check("angles")
+
+
+@pytest.mark.parametrize("rows,C", [(1, 64), (131, 320), (300, 4096)])
+@pytest.mark.parametrize("shift", [0, 16])
+def test_block_transform_stays_in_bounds(bq, rows, C, shift):
+    """All block formats and both unquantized outputs on ragged rows, a last unit of one
+    64-channel sub-tile (C = 320), and outputs shifted to the documented minimum alignment
+    (codes 16 bytes, scales 2 bytes), which the kernel's wide stores must detect."""
+    torch = H.torch()
+    rng = np.random.default_rng(rows + C + shift)
+    x = H.dev_bf16_bits(wl.bf16_bits_from_f32(rng.standard_normal((rows, C)).astype(np.float32)))
+    keep = _snap(x)
+    for fmt, G in (("mxfp4", 32), ("nvfp4", 16), ("int4", 32), ("none", 16), ("none", 32)):
+        Tb = wl.block_transforms(C, G, 3)
+        bt = bq.BlockTransform(H.dev_bf16_bits(Tb.reshape(-1, G)).view(Tb.shape))
+        st = Guarded((1,), torch.int32)
+        st.t.zero_()
+        if fmt == "none":
+            for dt in (torch.float32, torch.bfloat16):
+                y = Guarded((rows, C), dt, shift)
+                bq.bq_block_transform_quantize(bt, x, "none", y=y.t, status=st.t)
+                torch.cuda.synchronize()
+                y.check(f"block output {dt}")
+        else:
+            c = Guarded((rows, C // 2), torch.uint8, shift)
+            sc = Guarded((rows, C // G), torch.int16 if fmt == "int4" else torch.uint8, 2 if shift else 0)
+            bq.bq_block_transform_quantize(bt, x, fmt, c.t, sc.t, gscale=0.5, status=st.t)
+            torch.cuda.synchronize()
+            c.check(f"{fmt} codes")
+            sc.check(f"{fmt} scales")
+        st.check("status")
+        assert int(st.t.item()) == 0
+    assert _same(keep, (x,))
