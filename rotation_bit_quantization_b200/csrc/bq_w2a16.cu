@@ -757,161 +757,174 @@ __global__ void __launch_bounds__(256) k_splitk_reduce(const float* __restrict__
   }
 }
 
-// ------------------------------------------------------------------ decode path (1-3 tokens)
+// ------------------------------------------------------------------ decode path (1-8 tokens)
 //
 // With a handful of tokens each dequantized weight feeds only T products, and the
-// tensor-core kernel is bound by its MMA issue rate (four instructions per K stage of
-// 128 features whatever N is).  This kernel does the same arithmetic on the CUDA
-// cores: lane l of the block's 8 warps owns output feature 32 b + l, warp w a
-// contiguous eighth of K; the weights are the same bf16((q - z) s) values (2-bit
-// codes by the byte tables, 4-bit codes by the exact float form), each product of
-// two bf16 values is exact in float32 and is added into one of eight interleaved
-// accumulation chains per token (64 terms each for n = 4096), and the chains and the
-// eight warps' slices are added in a fixed order.  The activations are staged once
-// per block as float32 in shared memory and read by broadcast; each warp keeps the
-// codes and group parameters of four steps ahead in registers.  At about 5.7
-// instructions per weight for one token it is instruction bound (the expansion to
-// bf16 pairs and their unpacking cost 2.7 of them), ahead of the tensor-core kernel
-// up to 3 tokens.
-constexpr int kGemvMaxTokens = 3;                        // at 4 tokens both paths take the same time
-constexpr int kGemvWarps = 8;
-constexpr int kGemvSmemFloats = 16384;                   // T x n activations, at most 64 KiB
+// tensor-core GEMM is bound by its MMA issue rate (four instructions per K stage of
+// 128 features whatever N is).  Here the weights are expanded in registers straight
+// into the A fragments of warp-level bf16 MMAs (mma.sync m16n8k16, float32
+// accumulation) with the tokens as N (an 8-token fragment), so the products
+// and sums leave the CUDA cores: what remains per weight is the expansion (about 1.5
+// instructions per weight for 2-bit codes: the byte tables' selectors and permutes).
+//
+// A block is four warps on 16 output features; warp w takes a quarter of K in windows
+// of 256, the next window's codes loading while one is expanded.  Lane (g, c) = (lane / 4, lane % 4) owns features f0 + g and f0 + g + 8 and,
+// in window j, the 64 channels k = 256 j + 64 c .. + 63, so that its codes of a
+// window are one contiguous 16- or 32-byte run per feature and its group parameters
+// one pair per feature (groups are multiples of 64).  The MMA's 16-wide K slice s of
+// the window maps its positions 2c, 2c + 1, 2c + 8, 2c + 9 to the channels
+// k + 4 s + 0, 1, 2, 3 of lane c's run; A (weights) and B (activations) use the same
+// map, so the contraction is the plain dot product.  The four warps' partial sums are
+// added in warp order: the result is reproducible bitwise, and its error stays within
+// one float32 rounding per 16 products plus the final adds (the GEMM's bound).
+constexpr int kDecMaxTokens = 8;
+constexpr int kDecWarps = 4;
 
-template <int BITS, int T, bool BF16>
-__global__ void __launch_bounds__(32 * kGemvWarps, 2)
-    k_w2a16_gemv(const __nv_bfloat16* __restrict__ x, const uint8_t* __restrict__ codes,
-                 const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, void* __restrict__ out,
-                 int n, int out_features, int group) {
-  extern __shared__ float xs[];                           // [T][n]
-  __shared__ float red[kGemvWarps][T][32];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < T * n / 2; i += 32 * kGemvWarps) {
-    const uint32_t w = reinterpret_cast<const uint32_t*>(x)[i];
-    xs[2 * i] = __uint_as_float(w << 16);
-    xs[2 * i + 1] = __uint_as_float(w & 0xffff0000u);
+
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// 16 consecutive codes of one feature (bits 2i or 4i of `c`: one word of 2-bit codes, or
+// the low / high half of two words of 4-bit codes) -> 8 words of bf16 pairs
+template <int BITS>
+__device__ __forceinline__ void expand16(const Expand<BITS>& ex, const uint32_t* c, uint32_t (&w)[8]) {
+  if constexpr (BITS == 2) {
+    ex.t.word(c[0], w);
+  } else {
+    ex.dq.half(c[0], w);
+    ex.dq.half(c[0] >> 16, w + 2);
+    ex.dq.half(c[1], w + 4);
+    ex.dq.half(c[1] >> 16, w + 6);
   }
-  __syncthreads();
-  const int o = blockIdx.x * 32 + lane;
-  const bool live = o < out_features;
-  const int kw = n / kGemvWarps, k0 = warp * kw;          // kw: a multiple of 64
-  const int steps = kw / 64;                              // 64 codes per step: inside one group (group >= 64)
+}
+
+template <int BITS, int NB, bool BF16>
+__global__ void __launch_bounds__(32 * kDecWarps)
+    k_w2a16_dec(const __nv_bfloat16* __restrict__ x, int tokens, const uint8_t* __restrict__ codes,
+                const uint16_t* __restrict__ scale, const uint16_t* __restrict__ zero, void* __restrict__ out, int n,
+                int out_features, int group) {
+  __shared__ float red[kDecWarps][16][8 * NB];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const int f0 = blockIdx.x * 16;
+  const int fa = f0 + g, fb = f0 + g + 8;
+  const bool la = fa < out_features, lb = fb < out_features;
+  const int nwin = n / 256;
+  const int j0 = (warp * nwin) / kDecWarps, j1 = ((warp + 1) * nwin) / kDecWarps;
+  constexpr int kRun = 64 * BITS / 8;  // code bytes of a lane's run
+  const size_t row_bytes = static_cast<size_t>(n) * BITS / 8;
+  const uint8_t* ca = codes + static_cast<size_t>(la ? fa : 0) * row_bytes;
+  const uint8_t* cb = codes + static_cast<size_t>(lb ? fb : 0) * row_bytes;
   const int gpr = n / group;
-  const uint8_t* row = codes + static_cast<size_t>(live ? o : 0) * (static_cast<size_t>(n) * BITS / 8);
-  // the codes and group parameters of step i + kPre are loaded while step i is expanded
-  constexpr int kPre = 4, kWords = BITS / 2;              // 16-byte words of codes per step
-  uint4 cr[kPre][kWords];
-  float sr[kPre], zr[kPre];
-  auto fetch = [&](int i, uint4 (&c)[kWords], float& sv, float& zv) {
+  // activations of token g (and g + 8): rows past the last token read token 0 and are
+  // never stored
+  const __nv_bfloat16* xr[NB];
 #pragma unroll
-    for (int q = 0; q < kWords; ++q) c[q] = make_uint4(0u, 0u, 0u, 0u);
-    sv = 0.f;
-    zv = 0.f;
-    if (live && i < steps) {
-      const int k = k0 + 64 * i;
-      const uint4* src = reinterpret_cast<const uint4*>(row + static_cast<size_t>(k) * BITS / 8);
+  for (int h = 0; h < NB; ++h) xr[h] = x + static_cast<size_t>(g + 8 * h < tokens ? g + 8 * h : 0) * n;
+
+  float d[NB][4];
 #pragma unroll
-      for (int q = 0; q < kWords; ++q) c[q] = __ldcs(src + q);
-      const size_t gi = static_cast<size_t>(o) * gpr + k / group;
-      sv = __half2float(__ushort_as_half(__ldg(scale + gi)));
-      zv = __half2float(__ushort_as_half(__ldg(zero + gi)));
+  for (int h = 0; h < NB; ++h) d[h][0] = d[h][1] = d[h][2] = d[h][3] = 0.f;
+
+  auto load_run = [&](const uint8_t* base, int j, uint32_t (&r)[kRun / 4]) {
+    const uint4* src = reinterpret_cast<const uint4*>(base + static_cast<size_t>(256 * j + 64 * c) * BITS / 8);
+#pragma unroll
+    for (int q = 0; q < kRun / 16; ++q) {
+      const uint4 v = __ldcs(src + q);
+      r[4 * q] = v.x;
+      r[4 * q + 1] = v.y;
+      r[4 * q + 2] = v.z;
+      r[4 * q + 3] = v.w;
     }
   };
-#pragma unroll
-  for (int p = 0; p < kPre; ++p) fetch(p, cr[p], sr[p], zr[p]);
-  float2 acc[T][4];
-#pragma unroll
-  for (int t = 0; t < T; ++t)
-#pragma unroll
-    for (int c = 0; c < 4; ++c) acc[t][c] = make_float2(0.f, 0.f);
-  Expand<BITS> ex;
+  uint32_t ra[kRun / 4], rb[kRun / 4];
+  if (j0 < j1) {
+    load_run(ca, j0, ra);
+    load_run(cb, j0, rb);
+  }
 #pragma unroll 1
-  for (int i = 0; i < steps; ++i) {
-    const int k = k0 + 64 * i;
-    ex.set(sr[0], zr[0]);
-    uint32_t wv[32];
-    if constexpr (BITS == 2) {
-      ex.t.word(cr[0][0].x, wv);
-      ex.t.word(cr[0][0].y, wv + 8);
-      ex.t.word(cr[0][0].z, wv + 16);
-      ex.t.word(cr[0][0].w, wv + 24);
-    } else {
-      const uint32_t cw[8] = {cr[0][0].x, cr[0][0].y, cr[0][0].z, cr[0][0].w,
-                              cr[0][1].x, cr[0][1].y, cr[0][1].z, cr[0][1].w};
+  for (int j = j0; j < j1; ++j) {
+    const int k = 256 * j + 64 * c;
+    const int gi = k / group;
+    Expand<BITS> ea, eb;
+    ea.set(la ? __half2float(__ushort_as_half(__ldg(scale + static_cast<size_t>(fa) * gpr + gi))) : 0.f,
+           la ? __half2float(__ushort_as_half(__ldg(zero + static_cast<size_t>(fa) * gpr + gi))) : 0.f);
+    eb.set(lb ? __half2float(__ushort_as_half(__ldg(scale + static_cast<size_t>(fb) * gpr + gi))) : 0.f,
+           lb ? __half2float(__ushort_as_half(__ldg(zero + static_cast<size_t>(fb) * gpr + gi))) : 0.f);
+    uint32_t qa[kRun / 4], qb[kRun / 4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        ex.dq.half(cw[c], wv + 4 * c);
-        ex.dq.half(cw[c] >> 16, wv + 4 * c + 2);
+    for (int i = 0; i < kRun / 4; ++i) {
+      qa[i] = ra[i];
+      qb[i] = rb[i];
+    }
+    if (j + 1 < j1) {  // the next window's codes in flight meanwhile
+      load_run(ca, j + 1, ra);
+      load_run(cb, j + 1, rb);
+    }
+#pragma unroll
+    for (int sub = 0; sub < 4; ++sub) {  // 16 channels: four K slices of the MMA
+      uint32_t wa[8], wb[8];
+      expand16<BITS>(ea, qa + sub * (BITS / 2), wa);
+      expand16<BITS>(eb, qb + sub * (BITS / 2), wb);
+      uint4 xv[NB][2];
+#pragma unroll
+      for (int h = 0; h < NB; ++h) {
+        const uint4* xs = reinterpret_cast<const uint4*>(xr[h] + k + 16 * sub);
+        xv[h][0] = __ldg(xs);
+        xv[h][1] = __ldg(xs + 1);
       }
-    }
 #pragma unroll
-    for (int p = 0; p + 1 < kPre; ++p) {
+      for (int s = 0; s < 4; ++s) {
 #pragma unroll
-      for (int q = 0; q < kWords; ++q) cr[p][q] = cr[p + 1][q];
-      sr[p] = sr[p + 1];
-      zr[p] = zr[p + 1];
-    }
-    fetch(i + kPre, cr[kPre - 1], sr[kPre - 1], zr[kPre - 1]);
-#pragma unroll
-    for (int j = 0; j < 32; j += 2) {                      // words j, j + 1: weights of k + 2j .. k + 2j + 3
-      const float2 w0 = make_float2(__uint_as_float(wv[j] << 16), __uint_as_float(wv[j] & 0xffff0000u));
-      const float2 w1 = make_float2(__uint_as_float(wv[j + 1] << 16), __uint_as_float(wv[j + 1] & 0xffff0000u));
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        const float4 xv = *reinterpret_cast<const float4*>(xs + t * n + k + 2 * j);
-        acc[t][j & 3] = __ffma2_rn(w0, make_float2(xv.x, xv.y), acc[t][j & 3]);
-        acc[t][(j + 1) & 3] = __ffma2_rn(w1, make_float2(xv.z, xv.w), acc[t][(j + 1) & 3]);
+        for (int h = 0; h < NB; ++h) {
+          const uint4& v = xv[h][s >> 1];
+          const uint32_t b0 = (s & 1) ? v.z : v.x, b1 = (s & 1) ? v.w : v.y;
+          mma_16816(d[h], wa[2 * s], wb[2 * s], wa[2 * s + 1], wb[2 * s + 1], b0, b1);
+        }
       }
     }
   }
+  // d[h]: (feature g, tokens 8 h + 2 c, + 1), (feature g + 8, the same tokens)
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const float a = ((acc[t][0].x + acc[t][0].y) + (acc[t][1].x + acc[t][1].y)) +
-                    ((acc[t][2].x + acc[t][2].y) + (acc[t][3].x + acc[t][3].y));
-    red[warp][t][lane] = a;
+  for (int h = 0; h < NB; ++h) {
+    red[warp][g][8 * h + 2 * c] = d[h][0];
+    red[warp][g][8 * h + 2 * c + 1] = d[h][1];
+    red[warp][g + 8][8 * h + 2 * c] = d[h][2];
+    red[warp][g + 8][8 * h + 2 * c + 1] = d[h][3];
   }
   __syncthreads();
-  if (warp == 0 && live) {
+  for (int e = threadIdx.x; e < 16 * 8 * NB; e += 32 * kDecWarps) {
+    const int t = e / 16, f = e % 16;  // features fastest: coalesced stores
+    if (t < tokens && f0 + f < out_features) {
+      float v = red[0][f][t];
 #pragma unroll
-    for (int t = 0; t < T; ++t) {
-      float v = red[0][t][lane];
-#pragma unroll
-      for (int w = 1; w < kGemvWarps; ++w) v += red[w][t][lane];
+      for (int w = 1; w < kDecWarps; ++w) v += red[w][f][t];
+      const size_t o = static_cast<size_t>(t) * out_features + f0 + f;
       if (BF16)
-        static_cast<__nv_bfloat16*>(out)[static_cast<size_t>(t) * out_features + o] = __float2bfloat16_rn(v);
+        static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(v);
       else
-        static_cast<float*>(out)[static_cast<size_t>(t) * out_features + o] = v;
+        static_cast<float*>(out)[o] = v;
     }
   }
 }
 
 template <int BITS, bool BF16>
-bq_status run_gemv_t(const void* x, int tokens, int n, const uint8_t* codes, const uint16_t* scale,
-                     const uint16_t* zero, void* out, int out_features, int group, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>((out_features + 31) / 32);
-  const size_t smem = static_cast<size_t>(tokens) * n * sizeof(float);
+bq_status run_dec(const void* x, int tokens, int n, const uint8_t* codes, const uint16_t* scale, const uint16_t* zero,
+                  void* out, int out_features, int group, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((out_features + 15) / 16);
   const auto* xb = static_cast<const __nv_bfloat16*>(x);
-#define BQ_GEMV_CASE(T)                                                                                      \
-  case T: {                                                                                                  \
-    auto kern = k_w2a16_gemv<BITS, T, BF16>;                                                                 \
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=   \
-        cudaSuccess)                                                                                         \
-      return BQ_ERR_CUDA;                                                                                    \
-    kern<<<grid, 32 * kGemvWarps, smem, st>>>(xb, codes, scale, zero, out, n, out_features, group);          \
-    break;                                                                                                   \
-  }
-  switch (tokens) {
-    BQ_GEMV_CASE(1)
-    BQ_GEMV_CASE(2)
-    BQ_GEMV_CASE(3)
-    default: return BQ_ERR_INVALID_ARG;
-  }
-#undef BQ_GEMV_CASE
+  k_w2a16_dec<BITS, 1, BF16><<<grid, 32 * kDecWarps, 0, st>>>(xb, tokens, codes, scale, zero, out, n, out_features,
+                                                               group);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
-bool gemv_applies(long long tokens, int n) {
-  return tokens >= 1 && tokens <= kGemvMaxTokens && n % (64 * kGemvWarps) == 0 && tokens * n <= kGemvSmemFloats;
-}
+bool dec_applies(long long tokens, int n) { return tokens >= 1 && tokens <= kDecMaxTokens && n % 256 == 0; }
 
 // ------------------------------------------------------------------ host side
 
@@ -996,7 +1009,7 @@ using namespace bq;
 
 extern "C" size_t bq_w2a16_gemm_workspace_size(int64_t tokens, int32_t n, int64_t out_features) {
   if (tokens <= 0 || out_features <= 0 || n <= 0 || n % kBK != 0) return 0;
-  if (gemv_applies(tokens, n)) return 0;
+  if (dec_applies(tokens, n)) return 0;
   const Plan p = plan_of(tokens, n, out_features, sm_count());
   return p.part_bytes;
 }
@@ -1012,14 +1025,14 @@ extern "C" bq_status bq_w2a16_gemm(const void* x, int64_t tokens, int32_t n, con
   if (!x || !codes || !scale_f16 || !zero_f16 || !out) return BQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(codes)) return BQ_ERR_INVALID_ARG;
   if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return BQ_ERR_INVALID_ARG;
-  if (gemv_applies(tokens, n)) {  // decode-sized: the CUDA-core kernel
+  if (dec_applies(tokens, n)) {  // decode-sized: warp-level MMAs, weights expanded in registers
     auto st = static_cast<cudaStream_t>(stream);
     const int t = static_cast<int>(tokens), of = static_cast<int>(out_features);
     if (bits == 2)
-      return out_t == BQ_BF16 ? run_gemv_t<2, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
-                              : run_gemv_t<2, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
-    return out_t == BQ_BF16 ? run_gemv_t<4, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
-                            : run_gemv_t<4, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
+      return out_t == BQ_BF16 ? run_dec<2, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
+                              : run_dec<2, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
+    return out_t == BQ_BF16 ? run_dec<4, true>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st)
+                            : run_dec<4, false>(x, t, n, codes, scale_f16, zero_f16, out, of, group, st);
   }
   const int sms = sm_count();
   Plan p = plan_of(tokens, n, out_features, sms);

@@ -232,6 +232,7 @@ def test_w2a16_rejects_bad_arguments(lib):
     assert call(ws=FAKE + 16, ws_bytes=1 << 20) == bad      # workspace not 256-byte aligned
     assert lib.bq_w2a16_gemm_workspace_size(0, 4096, 128) == 0
     assert lib.bq_w2a16_gemm_workspace_size(16, 4000, 128) == 0
+    assert lib.bq_w2a16_gemm_workspace_size(17, 4000, 128) == 0
     assert lib.bq_w2a16_linear_workspace_size(4096, 3, 0) == 4096 * 3 * 2
     assert lib.bq_w2a16_linear_workspace_size(256, 1, 0) == 512
     layer = _lib.BQLayer(256, 256, 1, FAKE, None)
@@ -346,14 +347,14 @@ def test_cuda_error_accessors(lib):
 
 def test_w2a16_workspace_plan(lib):
     """Host-side plan of the W2A16 GEMM (148 SMs when no device answers, the B200's
-    count): no workspace for 1-3 tokens (the decode kernel) or once the output tiles
+    count): no workspace for 1-8 tokens (the decode kernel) or once the output tiles
     fill the SMs; a split-K workspace of float32 partial rows in between, sized in
     whole 128-feature tiles; 0 for invalid shapes."""
     n, out = 4096, 11008
     f_tiles = (out + 127) // 128
-    for t in (1, 2, 3):
+    for t in range(1, 9):
         assert lib.bq_w2a16_gemm_workspace_size(t, n, out) == 0
-    for t in (4, 16, 64, 128):
+    for t in (9, 16, 64, 128):
         ws = lib.bq_w2a16_gemm_workspace_size(t, n, out)
         ntok = max(16, (t + 15) // 16 * 16)
         assert ws > 0 and ws % (f_tiles * 128 * ntok * 4) == 0
@@ -361,8 +362,8 @@ def test_w2a16_workspace_plan(lib):
         assert 2 <= ksplit <= n // 64 // 4                  # at least 4 K stages per slice
     assert lib.bq_w2a16_gemm_workspace_size(2048, n, out) == 0   # 688 tiles >= 148 SMs
     assert lib.bq_w2a16_gemm_workspace_size(0, n, out) == 0
-    assert lib.bq_w2a16_gemm_workspace_size(16, 100, out) == 0   # n not a multiple of 64
-    assert lib.bq_w2a16_linear_workspace_size(n, 16, out) >= 16 * n * 2 + lib.bq_w2a16_gemm_workspace_size(16, n, out)
+    assert lib.bq_w2a16_gemm_workspace_size(17, 100, out) == 0   # n not a multiple of 64
+    assert lib.bq_w2a16_linear_workspace_size(n, 32, out) >= 32 * n * 2 + lib.bq_w2a16_gemm_workspace_size(32, n, out)
 
 
 def test_block_transform_rejects_bad_arguments(lib):

@@ -116,16 +116,17 @@ def test_gemm_bf16_unsplit_drained_epilogue(bq, tokens, n, out, bits, group):
 
 @pytest.mark.parametrize("tokens,out,bits,group", [(1, 11008, 2, 128), (16, 11008, 2, 128), (7, 4096, 4, 128),
                                                   (40, 1000, 2, 64), (100, 2048, 4, 256), (2, 1000, 4, 64),
-                                                  (3, 130, 2, 256), (4, 4096, 4, 128), (1, 200, 4, 128)])
+                                                  (3, 130, 2, 256), (4, 4096, 4, 128), (1, 200, 4, 128),
+                                                  (9, 1001, 2, 64), (17, 700, 4, 128), (8, 24, 2, 256)])
 def test_gemm_decode_sizes(bq, tokens, out, bits, group):
-    """Few tokens: 1-3 tokens run on the CUDA-core decode kernel, 4 or more split K over
-    the SMs and add the slices in a fixed order; either way the result matches the
-    oracle, repeats bitwise, and agrees with the unsplit kernel to float32 summation
-    order."""
+    """Few tokens: 1-8 tokens run on the decode kernel (warp-level MMAs on weights
+    expanded in registers), more split K over the SMs and add the slices in a fixed
+    order; either way the result matches the oracle, repeats bitwise, and agrees with
+    the unsplit kernel to float32 summation order."""
     n = 4096
     xb, codes, s16, z16 = _inputs(tokens + out + 3 * bits, tokens, n, out, bits, group)
     torch = H.torch()
-    assert (bq.bq_w2a16_gemm_workspace_size(tokens, n, out) > 0) == (tokens > 3)
+    assert (bq.bq_w2a16_gemm_workspace_size(tokens, n, out) > 0) == (tokens > 8)
     got = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, False), False)
     again = _as_f64(_gemm(bq, xb, codes, s16, z16, bits, group, False), False)
     assert np.array_equal(got, again)
