@@ -154,6 +154,51 @@ def test_quantizer_edge_groups(bq, fmt):
     assert np.array_equal(codes, c_ref)
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_exact_rounding_ties(bq, fmt):
+    """Identity blocks and groups whose scale is exact but whose reciprocal is not (0.375):
+    every other value is a rounding tie of the format's grid (E2M1 midpoints for NVFP4,
+    half-integers of the INT4 step), so the kernels' reciprocal products sit next to the
+    boundary and must take IEEE division: codes bit-exact with the oracle."""
+    G = ob.FORMATS[fmt]
+    C = 256
+    Tb = np.broadcast_to(wl.bf16_bits_from_f32(np.eye(G, dtype=np.float32)), (C // G, G, G)).copy()
+    rng = np.random.default_rng(23)
+    s = 0.375
+    if fmt == "nvfp4":
+        ties = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])   # E2M1 midpoints, in units of the scale
+        amax = 6 * s                                             # scale = E4M3(amax / 6) = 0.375 exactly
+    else:
+        ties = np.arange(-7, 7) + 0.5                            # half-integers
+        amax = 7 * s                                             # scale = fp16(amax / 7) = 0.375 exactly
+    rows = []
+    for r in range(6):
+        v = s * rng.choice(ties, C) * rng.choice([-1.0, 1.0], C)
+        v[::G] = amax * (1 if r % 2 else -1)                     # each group's absolute maximum
+        v[1::2] = v[1::2] * (1 + 2.0 ** -7 * rng.choice([-1, 0, 1], C // 2))  # bf16 neighbours of ties
+        rows.append(v)
+    x = np.clip(np.stack(rows), -amax, amax).astype(np.float32)
+    xb = wl.bf16_bits_from_f32(x)
+    codes, scales = _run(bq, Tb, xb, fmt)
+    y32 = wl.f32_from_bf16_bits(xb)                              # the identity transform is exact
+    c_ref, s_ref = ob.quantize(y32, fmt)
+    assert np.array_equal(scales, s_ref)
+    assert np.array_equal(codes, c_ref)
+
+
+@pytest.mark.parametrize("gscale", [2.0 ** -120, 1e-20, 3.0, 1e20, 2.0 ** 110])
+def test_nvfp4_global_scale_extremes(bq, gscale):
+    """Per-tensor scales that push den = s8 * gscale (or the quotients) out of the range
+    where the reciprocal product is checked: those groups take IEEE division; codes and
+    scales stay bit-exact with the oracle."""
+    Tb, xb = _case(31, 64, 512, 16)
+    codes, scales = _run(bq, Tb, xb, "nvfp4", gscale=gscale)
+    y32 = _run(bq, Tb, xb, "none").astype(np.float32)
+    c_ref, s_ref = ob.quantize(y32, "nvfp4", gscale)
+    assert np.array_equal(scales, s_ref)
+    assert np.array_equal(codes, c_ref)
+
+
 def test_rejects_bad_shapes(bq):
     torch = H.torch()
     Tb, xb = _case(1, 4, 128, 32)
