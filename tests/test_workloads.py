@@ -124,3 +124,19 @@ def test_w2a16_layer():
     assert codes.shape == (256, 1024) and s16.shape == z16.shape == (256, 32)
     again = wl.w2a16_4096(tokens=32, out_features=256)
     assert all(np.array_equal(u, v) for u, v in zip((x, codes, s16, z16), again[:4]))
+
+
+def test_block_transforms_recipe():
+    """Block transforms of the WUSH workload: (C/G, G, G) bf16 bits, I + 0.3 N(0,1)/sqrt(G) per
+    block (diagonal near 1, off-diagonal spread 0.3/sqrt(G)), deterministic in the seed,
+    different seeds and block sizes giving different matrices."""
+    for C, G in ((4096, 32), (4096, 16), (320, 32)):
+        Tb = wl.block_transforms(C, G, 7)
+        assert Tb.shape == (C // G, G, G) and Tb.dtype == np.uint16
+        T = wl.f32_from_bf16_bits(Tb).astype(np.float64)
+        assert np.array_equal(wl.bf16_bits_from_f32(T.astype(np.float32)), Tb)   # bf16 values
+        off = T - np.eye(G)[None]
+        assert abs(off.std() - 0.3 / np.sqrt(G)) < 0.1 * 0.3 / np.sqrt(G)
+        assert abs(np.diagonal(T, axis1=1, axis2=2).mean() - 1.0) < 0.02
+        assert np.array_equal(wl.block_transforms(C, G, 7), Tb)
+        assert not np.array_equal(wl.block_transforms(C, G, 8), Tb)
