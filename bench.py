@@ -254,13 +254,15 @@ E2E_CHUNKS = 4
 
 
 def pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, steps, warmup, nchunk=E2E_CHUNKS):
-    """Milliseconds per step of `steps` end-to-end steps through the public API with host
-    buffers: every step copies its whole input from pinned host memory, runs `call` and
+    """(milliseconds per step, method) of `steps` end-to-end steps through the public API with
+    host buffers: every step copies its whole input from pinned host memory, runs `call` and
     copies every output back, all inside the timed region.  The batch goes in `nchunk` row
     chunks and three streams: the copy-in of chunk c, the call on it and the copy-out of its
     results are ordered by events, so the two PCIe directions and the kernels overlap,
     within a step and across steps; two device buffer sets alternate by step, each chunk's
-    reuse waiting for the call and the copy-out that last used it.
+    reuse waiting for the call and the copy-out that last used it.  The timed steps are
+    captured in one CUDA graph (copies, calls and their cross-stream dependencies), so that
+    host-side launch work stays out of the time; if the capture fails, they run eagerly.
 
     make_dev() -> (x_dev, [out_dev, ...]) with rows in dimension 0; outs_pin the matching
     pinned host outputs; call(x_chunk, [out_chunk, ...]) runs the library on the current
@@ -272,17 +274,20 @@ def pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, steps, wa
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     ev = {k: [[torch.cuda.Event() for _ in bounds] for _ in range(2)] for k in ("in", "cmp", "out")}
 
-    def one(step):
+    def one(step, fresh):
+        # fresh: the buffer set has no earlier use in this sequence (nothing to wait for)
         k = step % 2
         xd, od = sets[k]
         for c, (r0, r1) in enumerate(bounds):
             with torch.cuda.stream(s_in):
-                s_in.wait_event(ev["cmp"][k][c])       # the call two steps back has read this chunk
+                if not fresh:
+                    s_in.wait_event(ev["cmp"][k][c])   # the call two steps back has read this chunk
                 xd[r0:r1].copy_(x_pin[r0:r1], non_blocking=True)
                 ev["in"][k][c].record(s_in)
             with torch.cuda.stream(s_cmp):
                 s_cmp.wait_event(ev["in"][k][c])
-                s_cmp.wait_event(ev["out"][k][c])      # the copy-out two steps back has read its outputs
+                if not fresh:
+                    s_cmp.wait_event(ev["out"][k][c])  # the copy-out two steps back has read its outputs
                 call(xd[r0:r1], [o[r0:r1] for o in od])
                 ev["cmp"][k][c].record(s_cmp)
             with torch.cuda.stream(s_out):
@@ -291,20 +296,39 @@ def pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, steps, wa
                     h[r0:r1].copy_(o[r0:r1], non_blocking=True)
                 ev["out"][k][c].record(s_out)
 
-    for i in range(warmup):
-        one(i)
+    def run(n):
+        for s_ in (s_in, s_cmp, s_out):
+            s_.wait_stream(torch.cuda.current_stream())
+        for i in range(n):
+            one(i, i < 2)
+        for s_ in (s_in, s_cmp, s_out):
+            torch.cuda.current_stream().wait_stream(s_)
+
+    run(max(warmup, 2))
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    try:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            run(steps)
+        torch.cuda.synchronize()
+        method = "one CUDA graph of the timed steps (copies, calls, cross-stream dependencies)"
+    except RuntimeError as exc:  # capture refused: time the same steps eagerly
+        graph = None
+        torch.cuda.synchronize()
+        method = f"eager (graph capture failed: {str(exc).splitlines()[0][:80]})"
     e0.record(stream)
-    for s_ in (s_in, s_cmp, s_out):
-        s_.wait_stream(stream)
-    for i in range(steps):
-        one(warmup + i)
-    for s_ in (s_in, s_cmp, s_out):
-        stream.wait_stream(s_)
+    if graph is not None:
+        graph.replay()
+    else:
+        run(steps)
     e1.record(stream)
     torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / steps
+    del graph
+    return e0.elapsed_time(e1) / steps, method
 
 
 def run_ours(args, spec, rank, world, local_rank):
@@ -422,7 +446,8 @@ def run_ours(args, spec, rank, world, local_rank):
 
         if world > 1:
             dist.barrier()
-        e2e_ms = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps, args.warmup)
+        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
+                                           args.warmup)
         te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -432,7 +457,7 @@ def run_ours(args, spec, rank, world, local_rank):
                "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
                "ms_per_step": e2e_ms,
                "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
-                           f"copy-out), two device buffer sets alternating by step"}
+                           f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
 
     peaks, peak_src = load_peaks()
     fl_launch = flops_per_row(w.m, w.r) * rows
@@ -824,7 +849,8 @@ def run_block_bench(args, spec, rank, world, local_rank):
 
         if world > 1:
             dist.barrier()
-        e2e_ms = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps, args.warmup)
+        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
+                                           args.warmup)
         te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
@@ -833,7 +859,7 @@ def run_block_bench(args, spec, rank, world, local_rank):
                "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
                "ms_per_step": float(te.item()),
                "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
-                           f"copy-out), two device buffer sets alternating by step"}
+                           f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import blockq as obq
