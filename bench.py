@@ -957,29 +957,30 @@ def run_gemm_bench(args, spec, rank, world, local_rank):
     if not args.no_e2e:
         x_pin = x_host.pin_memory()
         o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        x_dev = torch.empty_like(x)
+        # token chunks of the same GEMM (the weights stay on the device, as for a served layer)
+        chunk_tokens = -(-tokens // E2E_CHUNKS)
+        ws_c = torch.empty(max(256, bq.bq_w2a16_gemm_workspace_size(chunk_tokens, n, out_f)), dtype=torch.uint8,
+                           device=dev)
 
-        def e2e_step():
-            x_dev.copy_(x_pin, non_blocking=True)
-            bq.bq_w2a16_gemm(x_dev, codes, scale, zero, bits, group, out, workspace=ws, status=status)
-            o_pin.copy_(out, non_blocking=True)
+        def make_dev():
+            return torch.empty_like(x), [torch.empty_like(out)]
 
-        for _ in range(args.warmup):
-            e2e_step()
-        torch.cuda.synchronize()
+        def call(xc, oc):
+            bq.bq_w2a16_gemm(xc, codes, scale, zero, bits, group, oc[0],
+                             workspace=ws_c if xc.shape[0] == chunk_tokens else None, status=status)
+
         if world > 1:
             dist.barrier()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / args.steps], dtype=torch.float64, device=dev)
+        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, [o_pin], make_dev, call, args.steps,
+                                           args.warmup)
+        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
         if world > 1:
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e = {"value": flops * world / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2}
+               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+               "ms_per_step": float(te.item()),
+               "pipeline": f"{E2E_CHUNKS} token chunks per step on three streams (copy-in, the GEMM, copy-out), "
+                           f"two device buffer sets alternating by step; timed as {e2e_method}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
