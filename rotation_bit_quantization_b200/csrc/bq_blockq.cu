@@ -45,10 +45,7 @@ namespace {
 
 constexpr int kBM = 128;   // rows per unit (the MMA's M)
 constexpr int kBC = 64;    // channels per sub-tile (one 128-byte swizzle row of bf16)
-#ifndef BQ_BLOCK_SUB
-#define BQ_BLOCK_SUB 4
-#endif
-constexpr int kSub = BQ_BLOCK_SUB;  // sub-tiles per unit
+constexpr int kSub = 4;            // sub-tiles per unit
 constexpr int kUC = kBC * kSub;    // channels per unit
 constexpr int kStages = 6;         // sub-tile stages
 constexpr int kAStageBytes = kBM * kBC * 2;  // 16 KB
