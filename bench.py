@@ -50,6 +50,12 @@ def workload_spec(name: str):
     if name == "fwd4096":
         return dict(make=lambda rank: wl.act_4096(2048, seed_offset=rank), kind="fwd", rows=2048, n=4096,
                     bits=4, group=128, label="act n=4096 rows=2048 bf16 -> Qx float32 (forward only)")
+    if name == "inv4096":
+        return dict(make=lambda rank: wl.act_4096(2048, seed_offset=rank), kind="inv", rows=2048, n=4096,
+                    bits=4, group=128, label="act n=4096 rows=2048 bf16 -> Q^T y bf16 (inverse)")
+    if name == "inv5120":
+        return dict(make=lambda rank: wl.act_5120(8192), kind="inv", rows=8192, n=5120, bits=4, group=128,
+                    label="act n=5120 = B_1024 (x) O_5, rows=8192 bf16 -> Q^T y bf16 (inverse)")
     if name == "weight4096":
         return dict(make=lambda rank: wl.weight_4096(11008), kind="quant", rows=11008, n=4096, bits=2, group=128,
                     label="weight n=4096 rows=11008 bf16 -> W Q^T + INT2 RTN g128 (W2A16)")
@@ -177,8 +183,9 @@ def gpu_id_for(device) -> str:
         return str(device.index if hasattr(device, "index") else 0)
 
 
-def cpu_oracle_rate(w, rows_target_s: float, max_rows: int):
-    """Rows/s of the float64 oracle (transform + float32-step quantizer) on the host cores."""
+def cpu_oracle_rate(w, rows_target_s: float, max_rows: int, inverse: bool = False):
+    """Rows/s of the float64 oracle (transform + float32-step quantizer, or the inverse
+    transform alone) on the host cores."""
     from concurrent.futures import ThreadPoolExecutor
 
     from oracle import butterfly as ob
@@ -193,6 +200,9 @@ def cpu_oracle_rate(w, rows_target_s: float, max_rows: int):
     def one(lo):
         xs = src[lo:lo + chunk]
         xf = (wl.f32_from_bf16_bits(xs) if dt == "bf16" else xs).astype(np.float64)
+        if inverse:
+            ob.inverse(w.theta, xf) if w.r == 1 else ob.kron_inverse(w.theta, w.O, xf, w.m)
+            return xs.shape[0]
         y = ob.forward(w.theta, xf) if w.r == 1 else ob.kron_forward(w.theta, w.O, xf, w.m)
         oq.quantize_pack(y.astype(np.float32), w.bits, w.group)
         return xs.shape[0]
@@ -353,22 +363,26 @@ def run_ours(args, spec, rank, world, local_rank):
     O = None if w.O is None else torch.from_numpy(w.O).to(dev)
     layer = bq.Layer(theta, O)
     fwd = spec["kind"] == "fwd"
+    inv = spec["kind"] == "inv"
+    out_row_bytes = n * 4 if fwd else (n * 2 if inv else bytes_per_row(n, 0, bits, group))
     # Every timed step reads an input set that is not in L2: NS copies of the batch
     # (and NS output sets), cycled, with NS sets together more than twice the L2.
-    set_bytes = rows * (n * 2 + (n * 4 if fwd else bytes_per_row(n, 0, bits, group)))
+    set_bytes = rows * (n * 2 + out_row_bytes)
     NS = max(2, int(np.ceil(2 * L2_BYTES / set_bytes)))
     xs = [x] + [x.clone() for _ in range(NS - 1)]
-    if fwd:
-        outs = [torch.empty((rows, n), dtype=torch.float32, device=dev) for _ in range(NS)]
+    if fwd or inv:
+        outs = [torch.empty((rows, n), dtype=torch.float32 if fwd else torch.bfloat16, device=dev)
+                for _ in range(NS)]
     else:
         outs = [bq.quant_outputs(rows, n, bits, group, dev) for _ in range(NS)]
-    codes, scale, zero = (None, None, None) if fwd else outs[0]
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
     def step(i):
         if fwd:
             bq.bq_butterfly_fwd(layer, xs[i % NS], outs[i % NS])
+        elif inv:
+            bq.bq_butterfly_inv(layer, xs[i % NS], outs[i % NS])
         else:
             bq.bq_transform_quantize(layer, xs[i % NS], bits, group, *outs[i % NS])
 
@@ -433,16 +447,24 @@ def run_ours(args, spec, rank, world, local_rank):
 
     # end to end through the public API with host buffers: H2D input, kernel, D2H codes/scale/zero
     e2e = None
-    if not args.no_e2e and not fwd:
-        codes, scale, zero = outs[0]
+    if not args.no_e2e:
         x_pin = x_host.pin_memory()
-        outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (codes, scale, zero)]
+        if fwd or inv:
+            outs_pin = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()]
 
-        def make_dev():
-            return torch.empty_like(x), list(bq.quant_outputs(rows, n, bits, group, dev))
+            def make_dev():
+                return torch.empty_like(x), [torch.empty_like(outs[0])]
 
-        def call(xc, oc):
-            bq.bq_transform_quantize(layer, xc, bits, group, *oc)
+            def call(xc, oc):
+                (bq.bq_butterfly_fwd if fwd else bq.bq_butterfly_inv)(layer, xc, oc[0])
+        else:
+            outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[0]]
+
+            def make_dev():
+                return torch.empty_like(x), list(bq.quant_outputs(rows, n, bits, group, dev))
+
+            def call(xc, oc):
+                bq.bq_transform_quantize(layer, xc, bits, group, *oc)
 
         if world > 1:
             dist.barrier()
@@ -461,7 +483,7 @@ def run_ours(args, spec, rank, world, local_rank):
 
     peaks, peak_src = load_peaks()
     fl_launch = flops_per_row(w.m, w.r) * rows
-    by_launch = (bytes_per_row(n, 2, bits, group) if not fwd else n * (2 + 4)) * rows
+    by_launch = (n * 2 + out_row_bytes) * rows
     avg_launch_s = (total_ms / args.steps) * 1e-3
     achieved_tf = fl_launch / avg_launch_s / 1e12
     traffic, traffic_kernel = recorded_traffic(args.workload) if not (args.rows or args.layers) else (None, None)
@@ -511,7 +533,7 @@ def run_ours(args, spec, rank, world, local_rank):
                                      "(carries the launch and event overhead; not the bench value)"},
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, cores, sample = cpu_oracle_rate(w, rows_target_s=10.0, max_rows=rows * 8)
+        rate, cores, sample = cpu_oracle_rate(w, rows_target_s=10.0, max_rows=rows * 8, inverse=inv)
         result["cpu_baseline"] = {"value": rate, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample}
         rate, cores, sample = cpu_dense_rate(w, rows_sample=min(rows, 512))
         result["cpu_baseline_dense"] = {"value": rate, "unit": "rows/s", "cores": cores, "kind": "oracle (dense Q)",
@@ -1033,15 +1055,15 @@ def run_reference(args, spec):
     the workload, the metric and unit of our arm's line for that workload."""
     kind = spec["kind"]
     t0 = time.perf_counter()
-    if kind in ("quant", "fwd"):
+    if kind in ("quant", "fwd", "inv"):
         w = spec["make"](0)
         for _ in range(args.warmup):
-            cpu_oracle_rate(w, rows_target_s=1.0, max_rows=256)
+            cpu_oracle_rate(w, rows_target_s=1.0, max_rows=256, inverse=kind == "inv")
         rates = []
         sample = cores = None
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            rate, cores, sample = cpu_oracle_rate(w, rows_target_s=3.0, max_rows=spec["rows"])
+            rate, cores, sample = cpu_oracle_rate(w, rows_target_s=3.0, max_rows=spec["rows"], inverse=kind == "inv")
             rates.append(rate)
         el = time.perf_counter() - t0
         return _reference_line(args, spec, "butterfly fwd+quant rows/s and GB/s at n=4096 on 1 B200; % of FP32/HBM roofline",
@@ -1130,8 +1152,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="act4096",
-                    choices=["act4096", "fwd4096", "weight4096", "act5120", "bwd", "uniformity", "w2a16",
-                             "wush4096"])
+                    choices=["act4096", "fwd4096", "inv4096", "inv5120", "weight4096", "act5120", "bwd",
+                             "uniformity", "w2a16", "wush4096"])
     ap.add_argument("--rows", type=int, default=0, help="override the workload's rows (tokens per layer for bwd)")
     ap.add_argument("--layers", type=int, default=0, help="override the backward workload's layer count")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1152,6 +1174,7 @@ def main():
             spec = dict(spec, rows=rows, layers=args.layers or spec.get("layers", 1))
         else:
             base = {"act4096": lambda r, k: wl.act_4096(r, seed_offset=k), "fwd4096": lambda r, k: wl.act_4096(r, seed_offset=k),
+                    "inv4096": lambda r, k: wl.act_4096(r, seed_offset=k), "inv5120": lambda r, k: wl.act_5120(r),
                     "weight4096": lambda r, k: wl.weight_4096(r), "act5120": lambda r, k: wl.act_5120(r)}[args.workload]
             spec = dict(spec, rows=rows, make=lambda rank, b=base, r=rows: b(r, rank))
         spec["label"] = spec["label"] + f" [resized: rows={spec['rows']}" + (
