@@ -147,7 +147,8 @@ def quantize_int4_sym(y32):
     """(codes (rows, C) int8 in [-7, 7], scale16 bits (rows, C/32) uint16) of float32 rows."""
     v = _groups(y32, 32)
     amax = np.abs(v).max(axis=-1)
-    s16 = (amax / np.float32(7.0)).astype(np.float32).astype(np.float16)
+    with np.errstate(over="ignore"):  # beyond the fp16 range the scale rounds to infinity
+        s16 = (amax / np.float32(7.0)).astype(np.float32).astype(np.float16)
     s = s16.astype(np.float32)
     bad = (amax == 0) | (s == 0)
     s = np.where(bad, np.float32(1.0), s).astype(np.float32)
