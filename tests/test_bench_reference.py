@@ -1,6 +1,6 @@
 """The reference arm of bench.py (the float64 oracle timed on the host cores) runs
 without a GPU and prints one JSON line with the bench contract's keys, for the
-default workload and for the W2A16 GEMM."""
+default workload, the n=5120 inverse and the W2A16 GEMM."""
 
 import json
 import os
@@ -45,3 +45,10 @@ def test_reference_arm_default_workload():
 def test_reference_arm_w2a16():
     d = _run("--workload", "w2a16")
     _check_contract(d, "W2A16 GEMM TFLOP/s", "TFLOP/s")
+
+
+@pytest.mark.timeout(900)
+def test_reference_arm_inverse():
+    d = _run("--workload", "inv5120")
+    _check_contract(d, "butterfly fwd+quant rows/s", "rows/s")
+    assert d["config"]["n"] == 5120 and "inverse" in d["config"]["workload"]
