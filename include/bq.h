@@ -348,6 +348,18 @@ bq_status bq_block_transform_quantize(const uint16_t* table, int32_t C, int32_t 
  * failed.  Host only; launches nothing. */
 int32_t bq_cuda_last_error(void);
 
+/* The device's wait-fault word.  The m = 4096, r = 1 kernels of bq_butterfly_fwd,
+ * bq_butterfly_inv, bq_transform_quantize and bq_weight_rotate_pack pass rows
+ * between the warps of a row group through shared-memory barriers whose waits give
+ * up after one second, so that a fault elsewhere cannot hold an SM; a wait that
+ * gives up ORs 1 into this word of the library's memory on the current device
+ * (those calls take no status word).  No correct launch sets it.
+ * value: host int32 that receives the word; clear != 0 resets it to 0.
+ * Synchronises `stream` (the word is read after the work queued before it).
+ * Errors: BQ_ERR_INVALID_ARG for a NULL value (checked before any CUDA call),
+ * BQ_ERR_CUDA if a copy or the synchronisation fails. */
+bq_status bq_wait_faults(int32_t* value, int32_t clear, void* stream);
+
 /* Static description of a cudaError_t value from bq_cuda_last_error. */
 const char* bq_cuda_error_string(int32_t code);
 

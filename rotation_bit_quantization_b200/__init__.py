@@ -27,6 +27,7 @@ from ._lib import (  # noqa: F401
     bq_w2a16_gemm_workspace_size,
     bq_w2a16_linear,
     bq_w2a16_linear_workspace_size,
+    bq_wait_faults,
     load,
     quant_outputs,
     status_string,

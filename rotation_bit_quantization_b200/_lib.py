@@ -44,6 +44,7 @@ EXPORTED = (
     "bq_block_transform_quantize",
     "bq_status_string",
     "bq_cuda_last_error",
+    "bq_wait_faults",
     "bq_cuda_error_string",
 )
 
@@ -98,6 +99,7 @@ def load(path: str | None = None):
         "bq_block_transform_quantize": (i32, [vp, i32, i32, vp, i64, i32, ctypes.c_float, vp, i32, vp, vp, vp, vp]),
         "bq_status_string": (ctypes.c_char_p, [i32]),
         "bq_cuda_last_error": (i32, []),
+        "bq_wait_faults": (i32, [ctypes.POINTER(i32), i32, vp]),
         "bq_cuda_error_string": (ctypes.c_char_p, [i32]),
     }
     for name, (res, args) in sig.items():
@@ -303,6 +305,14 @@ def bq_uniformity_loss(y, bits: int, group: int, eps: float, kl_group, dy=None, 
     _check("bq_uniformity_loss", load().bq_uniformity_loss(_ptr(y), rows, n, bits, group, float(eps), _ptr(kl_group),
                                                             _ptr(dy), _ptr(loss), _stream(stream)))
     return kl_group, dy, loss
+
+
+def bq_wait_faults(clear: bool = False, stream=None) -> int:
+    """The device's wait-fault word (0: no bounded wait of the m = 4096 kernels gave up);
+    synchronises the stream, and resets the word when `clear`."""
+    v = ctypes.c_int32(0)
+    _check("bq_wait_faults", load().bq_wait_faults(ctypes.byref(v), 1 if clear else 0, _stream(stream)))
+    return int(v.value)
 
 
 def bq_angle_sgd(theta, dtheta, lr: float, stream=None):

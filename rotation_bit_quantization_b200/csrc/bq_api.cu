@@ -123,6 +123,11 @@ bq_status bq_weight_rotate_pack(const bq_layer* layer, const void* w, bq_dtype w
   return quantize(layer, w, wt, out_features, bits, group, codes, scale_f16, zero_f16, stream);
 }
 
+bq_status bq_wait_faults(int32_t* value, int32_t clear, void* stream) {
+  if (value == nullptr) return BQ_ERR_INVALID_ARG;
+  return bq::read_wait_faults(value, clear != 0, static_cast<cudaStream_t>(stream));
+}
+
 const char* bq_status_string(bq_status status) {
   switch (status) {
     case BQ_OK: return "ok";

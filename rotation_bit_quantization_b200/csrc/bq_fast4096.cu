@@ -21,10 +21,15 @@
 //    and two swizzled shared-memory transposes between them (conflict-free:
 //    one side uses 16-byte vectors, the other 4-byte scalars).  The A -> B
 //    exchange stays inside each warp (bits 10, 11 are the warp index of both
-//    layouts); only B -> C needs the row group's barrier.  Pass C's
+//    layouts); only B -> C crosses the row group's warps.  Pass C's
 //    layout keeps 8 consecutive positions per thread, so the RTN epilogue
 //    (group statistics, packing, coalesced stores) runs in place without a
 //    third transpose.
+//  * The B -> C exchange is a split barrier (an mbarrier per buffer): a
+//    thread arrives after writing its part of row j and waits for row j's
+//    phase only in the next iteration, after row j + 1's pass A, which parks
+//    in the warp's A -> B buffer meanwhile; so the warps of a row group need
+//    not meet at the exchange.  Waits are bounded (bq_wait_faults).
 //  * Rotations use the scaled two-FMA form prepared by bq_precompute_cs
 //    (a_i += alpha a_j, a_j += beta a_i; outputs times sigma), issued as packed
 //    fma.rn.f32x2 where two pairs sit in adjacent registers; when the layer's
@@ -47,7 +52,7 @@ constexpr int kColB = 160, kColC = 320, kColS = 384;
 constexpr int kFillChunks = kImageCols / 16;  // 26 chunks of 16 columns
 
 // forward kernel: kSlots row groups, each with an A -> B buffer, two alternating
-// B -> C buffers and the epilogue's parameter slots
+// B -> C buffers and the epilogue's parameter slots (the inverse's buffers below)
 // Three row groups with double-buffered coefficient loads (168 registers) and four
 // with single-buffered loads (128 registers) measured the same at 16384 rows; three
 // were 6% faster at 2048 rows and for the inverse.
@@ -59,6 +64,11 @@ constexpr int kParamFloats = 4 * 32 * 4;  // 4 warps x 32 slots x float4
 constexpr int kSlotFloats = 3 * kBufFloats + kParamFloats;
 constexpr int kFwdSmemBytes = kSlots * kSlotFloats * static_cast<int>(sizeof(float));
 static_assert(kFwdSmemBytes <= 227 * 1024, "shared memory per CTA");
+// the inverse: per row group one B -> A buffer and kInvBufs rotating C -> B buffers
+constexpr int kInvBufs = 3;
+constexpr int kInvSlotFloats = (1 + kInvBufs) * kBufFloats;
+constexpr int kInvSmemBytes = kSlots * kInvSlotFloats * static_cast<int>(sizeof(float));
+static_assert(kInvSmemBytes <= 227 * 1024, "shared memory per CTA");
 // image chunks a thread loads per round of the start-up fill: all of its chunks at
 // once where registers allow (three row groups: 9 chunks, 144 registers), four at a
 // time with more row groups
@@ -105,11 +115,64 @@ __device__ __forceinline__ void tmem_st16(uint32_t addr, const uint32_t (&r)[16]
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void group_sync(int slot) {
-  asm volatile("bar.sync %0, %1;" ::"r"(1 + slot), "r"(kGroupThreads) : "memory");
-}
 
 __device__ __forceinline__ float u2f(uint32_t v) { return __uint_as_float(v); }
+
+// ------------------------------------------------------------------ row-group barriers
+//
+// The forward's B -> C exchange uses a split barrier: every thread of the row
+// group arrives on the buffer's mbarrier after writing its part of a row, and
+// waits for that phase only when it comes to read the row, with the next row's
+// first pass in between.  A wait gives up after one second and records it in the
+// library's wait-fault word (read and cleared by bq_wait_faults), so that no
+// failure can hold the SM.
+
+constexpr unsigned long long kWaitLimitNs = 1000000000ull;
+
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n .reg .b64 st;\n mbarrier.arrive.shared::cta.b64 st, [%0];\n}" ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+}  // namespace
+
+__device__ int g_wait_faults = 0;
+
+namespace {
+
+__device__ __forceinline__ void mbar_wait(uint32_t bar, uint32_t parity) {
+  if (mbar_try(bar, parity)) return;
+  const unsigned long long t0 = gtimer();
+  while (!mbar_try(bar, parity)) {
+    if (gtimer() - t0 > kWaitLimitNs) {
+      atomicOr(&g_wait_faults, 1);
+      return;
+    }
+  }
+}
 
 // ------------------------------------------------------------------ one stage in registers
 //
@@ -233,7 +296,7 @@ __device__ __forceinline__ void unpack_input(const Prefetch<float>& p, float2 (&
 // halves of each 8-position run swapped by bit 2 of the thread index.  Every
 // access of a warp covers distinct banks in each of its phases.
 
-__device__ __forceinline__ void xpose_ab(float2 (&a)[16], float* buf, int tau) {
+__device__ __forceinline__ void xpose_ab_write(const float2 (&a)[16], float* buf, int tau) {
 #pragma unroll
   for (int c = 0; c < 8; ++c)
     *reinterpret_cast<float4*>(buf + tau * 32 + 4 * (c ^ (tau & 7))) =
@@ -242,6 +305,9 @@ __device__ __forceinline__ void xpose_ab(float2 (&a)[16], float* buf, int tau) {
   // positions of pass-A threads 32 (t >> 5) .. 32 (t >> 5) + 31: position bits 10, 11
   // are the warp index in both layouts, so this exchange stays inside the warp
   __syncwarp();
+}
+
+__device__ __forceinline__ void xpose_ab_read(float2 (&a)[16], const float* buf, int tau) {
   const int base = ((tau >> 5) << 10) + (tau & 3), cq = (tau & 31) >> 2;
 #pragma unroll
   for (int rb = 0; rb < 32; rb += 2) {
@@ -249,6 +315,11 @@ __device__ __forceinline__ void xpose_ab(float2 (&a)[16], float* buf, int tau) {
     const float v1 = buf[base + 32 * (rb + 1) + 4 * (cq ^ ((rb + 1) & 7))];
     a[rb >> 1] = make_float2(v0, v1);
   }
+}
+
+__device__ __forceinline__ void xpose_ab(float2 (&a)[16], float* buf, int tau) {
+  xpose_ab_write(a, buf, tau);
+  xpose_ab_read(a, buf, tau);
 }
 
 __device__ __forceinline__ void xpose_bc_write(const float2 (&a)[16], float* buf, int tau) {
@@ -404,63 +475,93 @@ __device__ __forceinline__ void store_epilogue(const float2 (&a)[16], const Fast
   }
 }
 
-// One row through all twelve stages and the epilogue.  On entry `pre` holds the
-// row's input (and, double-buffered, c0 holds coefficient block 0); on return
-// `pre` holds the next row's input (if ncnt > 0).
-template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
-__device__ __forceinline__ void process(const FastArgs& A, long long row, int ncnt, int slot, int tau, int lane,
-                                        uint32_t tb, float* bufAB, float* bufBC, float4* params,
-                                        Prefetch<TI>& pre, uint32_t (&c0)[32], uint32_t (&c1)[32]) {
-  float2 a[16];
-  unpack_input(pre, a);
-  prefetch(pre, static_cast<const TI*>(A.x), row + 1, ncnt, tau);
+static_assert(kDoubleBuf, "the forward's pass sequence assumes double-buffered coefficient loads");
 
-  // pass A: stages 0..4 on position bits 0..4
-  stage_step<0, SCALED>(a, c0, c1, tb, tb + 32);
-  stage_step<1, SCALED>(a, c1, c0, tb + 32, tb + 64);
-  stage_step<2, SCALED>(a, c0, c1, tb + 64, tb + 96);
-  stage_step<3, SCALED>(a, c1, c0, tb + 96, tb + 128);
-  stage_step<4, SCALED>(a, c0, c1, tb + 128, tb + kColB);
-  xpose_ab(a, bufAB, tau);
-  // pass B: stages 5..9 on position bits 5..9
-  stage_step<0, SCALED>(a, c1, c0, tb + kColB, tb + kColB + 32);
-  stage_step<1, SCALED>(a, c0, c1, tb + kColB + 32, tb + kColB + 64);
-  stage_step<2, SCALED>(a, c1, c0, tb + kColB + 64, tb + kColB + 96);
-  stage_step<3, SCALED>(a, c0, c1, tb + kColB + 96, tb + kColB + 128);
-  stage_step<4, SCALED>(a, c1, c0, tb + kColB + 128, tb + kColC);
-  xpose_bc_write(a, bufBC, tau);
-  group_sync(slot);
-  xpose_bc_read(a, bufBC, tau);
-  // pass C: stages 10, 11 on slot bits 3, 4 (position bits 10, 11)
-  stage_step<3, SCALED>(a, c0, c1, tb + kColC, tb + kColC + 32);
-  stage_step<4, SCALED>(a, c1, c0, tb + kColC + 32, tb + kColS);
-  // output scale (1 for the plain rotation)
-  if constexpr (!kDoubleBuf) {
-    tmem_ld32(tb + kColS, c0);
-    tmem_wait(c0);
-  }
+// The forward's three passes on the row in registers.  Each starts with the
+// coefficient block of its first stage in `x` and returns with the block at `next`
+// in `y` (pass C: in `x` again, loaded while the epilogue runs).
+template <bool SCALED>
+__device__ __forceinline__ void pass_a(float2 (&a)[16], uint32_t (&x)[32], uint32_t (&y)[32], uint32_t tb,
+                                       uint32_t next) {
+  stage_step<0, SCALED>(a, x, y, tb, tb + 32);
+  stage_step<1, SCALED>(a, y, x, tb + 32, tb + 64);
+  stage_step<2, SCALED>(a, x, y, tb + 64, tb + 96);
+  stage_step<3, SCALED>(a, y, x, tb + 96, tb + 128);
+  stage_step<4, SCALED>(a, x, y, tb + 128, next);
+}
+
+template <bool SCALED>
+__device__ __forceinline__ void pass_b(float2 (&a)[16], uint32_t (&x)[32], uint32_t (&y)[32], uint32_t tb,
+                                       uint32_t next) {
+  stage_step<0, SCALED>(a, x, y, tb + kColB, tb + kColB + 32);
+  stage_step<1, SCALED>(a, y, x, tb + kColB + 32, tb + kColB + 64);
+  stage_step<2, SCALED>(a, x, y, tb + kColB + 64, tb + kColB + 96);
+  stage_step<3, SCALED>(a, y, x, tb + kColB + 96, tb + kColB + 128);
+  stage_step<4, SCALED>(a, x, y, tb + kColB + 128, next);
+}
+
+// Pass C (stages 10, 11 on slot bits 3, 4: position bits 10, 11), the output scale
+// (1 for the plain rotation) and the epilogue of row `row`.
+template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
+__device__ __forceinline__ void pass_c(float2 (&a)[16], uint32_t (&x)[32], uint32_t (&y)[32], const FastArgs& A,
+                                       long long row, int tau, int lane, uint32_t tb, float4* params,
+                                       uint32_t next) {
+  stage_step<3, SCALED>(a, x, y, tb + kColC, tb + kColC + 32);
+  stage_step<4, SCALED>(a, y, x, tb + kColC + 32, tb + kColS);
 #pragma unroll
-  for (int q = 0; q < 16; ++q) a[q] = __fmul2_rn(a[q], make_float2(u2f(c0[2 * q]), u2f(c0[2 * q + 1])));
-  if constexpr (kDoubleBuf) tmem_ld32(tb, c0);  // block 0 of the next row
+  for (int q = 0; q < 16; ++q) a[q] = __fmul2_rn(a[q], make_float2(u2f(x[2 * q]), u2f(x[2 * q + 1])));
+  tmem_ld32(next, x);
   if constexpr (MODE == kQuant) {
     quant_epilogue<BITS, GLANES>(a, A, row, tau, lane, params);
   } else {
     store_epilogue<MODE>(a, A, row, tau);
   }
-  if constexpr (kDoubleBuf) tmem_wait(c0);
+  tmem_wait(x);
 }
 
+// Rows rb .. re - 1 of one row group, software-pipelined around the B -> C
+// exchange: row j's pass A runs, and the row parks in the A -> B buffer, before
+// the group waits for row j - 1's B -> C buffer; then row j - 1's pass C and
+// epilogue, row j's pass B and its B -> C writes.  The B -> C buffers and their
+// mbarriers alternate by row.  Buffer reuse: a thread writes row j's B -> C
+// buffer after its wait for row j - 1, which every thread of the group arrives
+// at only after reading row j - 2 from that buffer.  On entry `pre` holds row
+// rb's input and c0 coefficient block 0.
 template <typename TI, int MODE, int BITS, int GLANES, bool SCALED>
-__device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long long re, int slot, int tau, int lane,
-                                         uint32_t tb, float* bufAB, float* bufBC, float4* params, Prefetch<TI>& pre,
-                                         uint32_t (&c0)[32], uint32_t (&c1)[32]) {
-  // the B -> C buffer alternates between rows: with only a warp-level sync before
-  // the next row's B -> C writes, row i's readers and row i+2's writers are kept
-  // apart by row i+1's row-group barrier
+__device__ __forceinline__ void run_rows(const FastArgs& A, long long rb, long long re, int tau, int lane,
+                                         uint32_t tb, float* bufAB, float* bufBC, float4* params, uint32_t bars,
+                                         Prefetch<TI>& pre, uint32_t (&c0)[32], uint32_t (&c1)[32]) {
+  const TI* X = static_cast<const TI*>(A.x);
+  float2 a[16];
 #pragma unroll 1
-  for (long long row = rb; row < re; ++row)
-    process<TI, MODE, BITS, GLANES, SCALED>(A, row, row + 1 < re ? 1 : 0, slot, tau, lane, tb, bufAB,
-                                            bufBC + ((row - rb) & 1) * kBufFloats, params, pre, c0, c1);
+  for (long long row = rb; row < re; ++row) {
+    const int j = static_cast<int>(row - rb);
+    unpack_input(pre, a);
+    prefetch(pre, X, row + 1, row + 1 < re ? 1 : 0, tau);
+    if (j == 0) {
+      pass_a<SCALED>(a, c0, c1, tb, tb + kColB);
+      xpose_ab(a, bufAB, tau);
+    } else {
+      pass_a<SCALED>(a, c0, c1, tb, tb + kColC);
+      xpose_ab_write(a, bufAB, tau);  // row j parks here
+      const int jp = j - 1;
+      mbar_wait(bars + 8 * (jp & 1), (jp >> 1) & 1);
+      xpose_bc_read(a, bufBC + (jp & 1) * kBufFloats, tau);
+      pass_c<TI, MODE, BITS, GLANES, SCALED>(a, c1, c0, A, row - 1, tau, lane, tb, params, tb + kColB);
+      xpose_ab_read(a, bufAB, tau);
+    }
+    pass_b<SCALED>(a, c1, c0, tb, tb);
+    xpose_bc_write(a, bufBC + (j & 1) * kBufFloats, tau);
+    mbar_arrive(bars + 8 * (j & 1));
+  }
+  if (re > rb) {
+    const int jl = static_cast<int>(re - 1 - rb);
+    tmem_ld32(tb + kColC, c1);
+    mbar_wait(bars + 8 * (jl & 1), (jl >> 1) & 1);
+    xpose_bc_read(a, bufBC + (jl & 1) * kBufFloats, tau);
+    tmem_wait(c1);
+    pass_c<TI, MODE, BITS, GLANES, SCALED>(a, c1, c0, A, re - 1, tau, lane, tb, params, tb);
+  }
 }
 
 // Copies this thread's share of a tensor-memory image (NCHUNK chunks of 16
@@ -511,6 +612,7 @@ template <typename TI, int MODE, int BITS, int GLANES>
 __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   extern __shared__ __align__(16) float smem[];
   __shared__ uint32_t s_tmem;
+  __shared__ __align__(8) unsigned long long s_bars[kSlots][2];  // B -> C buffer of rows j, j + 1
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
   float* sbase = smem + slot * kSlotFloats;
@@ -524,6 +626,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   Prefetch<TI> pre;
   prefetch(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
 
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(smem_addr(&s_bars[i][0]), kGroupThreads);
+      mbar_init(smem_addr(&s_bars[i][1]), kGroupThreads);
+    }
+  }
   if (warp == 0) {
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(dst) : "memory");
@@ -539,15 +648,16 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   tc_fence_after();
 
   const bool scaled = A.hdr[0] == 1.f;
+  const uint32_t bars = smem_addr(&s_bars[slot][0]);
   uint32_t c0[32], c1[32];
   if constexpr (kDoubleBuf) {
     tmem_ld32(tb, c0);
     tmem_wait(c0);
   }
   if (scaled)
-    run_rows<TI, MODE, BITS, GLANES, true>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, params, pre, c0, c1);
+    run_rows<TI, MODE, BITS, GLANES, true>(A, rb, re, tau, lane, tb, bufAB, bufBC, params, bars, pre, c0, c1);
   else
-    run_rows<TI, MODE, BITS, GLANES, false>(A, rb, re, slot, tau, lane, tb, bufAB, bufBC, params, pre, c0, c1);
+    run_rows<TI, MODE, BITS, GLANES, false>(A, rb, re, tau, lane, tb, bufAB, bufBC, params, bars, pre, c0, c1);
 
   tc_fence_before();
   __syncthreads();
@@ -599,8 +709,9 @@ bq_status dispatch_quant(const FastArgs& A, int bits, int group, cudaStream_t st
 // bq_precompute_cs (table header[3]); the image holds them in the forward's
 // columns (stage s at column 32 s, the output scale of the pass-A positions at
 // column 384), or (cos, sin) when that form is out of range, in which case the
-// plain transposed rotation [[c, s], [-s, c]] runs.  Same row groups, buffers
-// and coefficient loads as the forward.
+// plain transposed rotation [[c, s], [-s, c]] runs.  Same row groups and
+// coefficient loads as the forward; the C -> B exchange is split the same way, with
+// three buffers rotating by row (see run_inv_rows).
 
 template <int SB>
 __device__ __forceinline__ void stage_inv_plain(float2 (&a)[16], const uint32_t (&c)[32]) {
@@ -662,33 +773,39 @@ __device__ __forceinline__ void prefetch_c(Prefetch<TI>& p, const TI* x, long lo
   }
 }
 
-template <typename TI, typename TO, bool SCALED>
-__device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int ncnt, int slot, int tau, uint32_t tb,
-                                        float* bufAB, float* bufBC, Prefetch<TI>& pre, uint32_t (&c0)[32],
-                                        uint32_t (&c1)[32]) {
-  float2 a[16];
-  unpack_input(pre, a);
-  prefetch_c(pre, static_cast<const TI*>(A.x), row + 1, ncnt, tau);
-  // pass C: stages 11, 10 (slot bits 4, 3); double-buffered, c0 holds block 11 on entry
+// Pass C of the inverse (stages 11, 10 on slot bits 4, 3); c0 holds block 11 on
+// entry and block 9 on return.
+template <bool SCALED>
+__device__ __forceinline__ void inv_pass_c(float2 (&a)[16], uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t tb) {
   inv_step<11, 4, SCALED>(a, c0, c1, tb);
   inv_step<10, 3, SCALED>(a, c1, c0, tb);
-  {
-    const int sw = (tau >> 2) & 1;
+}
+
+// C -> B exchange (across the row group's warps): pass-C threads write 16-byte
+// vectors, pass-B threads read single floats.
+__device__ __forceinline__ void inv_c2b_write(const float2 (&a)[16], float* buf, int tau) {
+  const int sw = (tau >> 2) & 1;
 #pragma unroll
-    for (int h = 0; h < 4; ++h)
+  for (int h = 0; h < 4; ++h)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float4*>(bufBC + h * 1024 + tau * 8 + 4 * (hh ^ sw)) =
-            make_float4(a[4 * h + 2 * hh].x, a[4 * h + 2 * hh].y, a[4 * h + 2 * hh + 1].x, a[4 * h + 2 * hh + 1].y);
-  }
-  group_sync(slot);
-  {
-    const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
+    for (int hh = 0; hh < 2; ++hh)
+      *reinterpret_cast<float4*>(buf + h * 1024 + tau * 8 + 4 * (hh ^ sw)) =
+          make_float4(a[4 * h + 2 * hh].x, a[4 * h + 2 * hh].y, a[4 * h + 2 * hh + 1].x, a[4 * h + 2 * hh + 1].y);
+}
+
+__device__ __forceinline__ void inv_c2b_read(float2 (&a)[16], const float* buf, int tau) {
+  const int base = (tau >> 5) * 1024 + ((tau & 31) >> 3) * 8 + (tau & 3), sw = (tau >> 2) & 1;
 #pragma unroll
-    for (int rb = 0; rb < 32; rb += 2)
-      a[rb >> 1] = make_float2(bufBC[base + 32 * rb + 4 * sw], bufBC[base + 32 * (rb + 1) + 4 * (sw ^ 1)]);
-  }
-  // pass B: stages 9 .. 5
+  for (int rb = 0; rb < 32; rb += 2)
+    a[rb >> 1] = make_float2(buf[base + 32 * rb + 4 * sw], buf[base + 32 * (rb + 1) + 4 * (sw ^ 1)]);
+}
+
+// Passes B and A of the inverse (stages 9 .. 0, the B -> A exchange inside the
+// warp), the output scale and the store of row `row`; c0 holds block 9 on entry and
+// block 11 on return.
+template <typename TO, bool SCALED>
+__device__ __forceinline__ void inv_pass_ba(float2 (&a)[16], uint32_t (&c0)[32], uint32_t (&c1)[32], uint32_t tb,
+                                            float* bufAB, const FastArgs& A, long long row, int tau) {
   inv_step<9, 4, SCALED>(a, c0, c1, tb);
   inv_step<8, 3, SCALED>(a, c1, c0, tb);
   inv_step<7, 2, SCALED>(a, c0, c1, tb);
@@ -709,14 +826,14 @@ __device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int nc
     a[2 * c] = make_float2(v.x, v.y);
     a[2 * c + 1] = make_float2(v.z, v.w);
   }
-  // pass A: stages 4 .. 0 (double-buffered, the last one loads block 11 of the next row)
+  // pass A: stages 4 .. 0 (the last one loads block 11 of the next row)
   inv_step<4, 4, SCALED>(a, c1, c0, tb);
   inv_step<3, 3, SCALED>(a, c0, c1, tb);
   inv_step<2, 2, SCALED>(a, c1, c0, tb);
   inv_step<1, 1, SCALED>(a, c0, c1, tb);
   inv_step<0, 0, SCALED>(a, c1, c0, tb);
   if constexpr (SCALED) {
-    // output scale of the pass-A positions; then block 11 again for the next row
+    // output scale of the pass-A positions
     tmem_ld32(tb + kColS, c1);
     tmem_wait(c1);
 #pragma unroll
@@ -743,20 +860,69 @@ __device__ __forceinline__ void inv_row(const FastArgs& A, long long row, int nc
   }
 }
 
+// Rows rb .. re - 1 of one row group, software-pipelined around the C -> B
+// exchange: row j's pass C runs and the row goes into its C -> B buffer before the
+// group waits for row j - 1's; then row j - 1's passes B and A and its store.
+// Three C -> B buffers (and mbarriers) rotate by row, and a thread arrives for row
+// j only after it has read row j - 1: a thread writes row j into the buffer of row
+// j - 3 after its wait for row j - 2, which every thread arrives at only after
+// reading row j - 3.  On entry `pre` holds row rb's input and c0 block 11.
+template <typename TI, typename TO, bool SCALED>
+__device__ __forceinline__ void run_inv_rows(const FastArgs& A, long long rb, long long re, int tau, uint32_t tb,
+                                             float* bufAB, float* bufCB, uint32_t bars, Prefetch<TI>& pre,
+                                             uint32_t (&c0)[32], uint32_t (&c1)[32]) {
+  const TI* X = static_cast<const TI*>(A.x);
+  float2 a[16];
+#pragma unroll 1
+  for (long long row = rb; row < re; ++row) {
+    const int j = static_cast<int>(row - rb), b = j % kInvBufs;
+    unpack_input(pre, a);
+    prefetch_c(pre, X, row + 1, row + 1 < re ? 1 : 0, tau);
+    inv_pass_c<SCALED>(a, c0, c1, tb);
+    inv_c2b_write(a, bufCB + b * kBufFloats, tau);
+    if (j == 0) {
+      mbar_arrive(bars + 8 * b);
+      tmem_ld32(tb + 32 * 11, c0);  // pass C of the next row comes first
+      tmem_wait(c0);
+    } else {
+      const int jp = j - 1, bp = jp % kInvBufs;
+      mbar_wait(bars + 8 * bp, (jp / kInvBufs) & 1);
+      inv_c2b_read(a, bufCB + bp * kBufFloats, tau);
+      mbar_arrive(bars + 8 * b);
+      inv_pass_ba<TO, SCALED>(a, c0, c1, tb, bufAB, A, row - 1, tau);
+    }
+  }
+  if (re > rb) {
+    const int jl = static_cast<int>(re - 1 - rb), bl = jl % kInvBufs;
+    tmem_ld32(tb + 32 * 9, c0);
+    mbar_wait(bars + 8 * bl, (jl / kInvBufs) & 1);
+    inv_c2b_read(a, bufCB + bl * kBufFloats, tau);
+    tmem_wait(c0);
+    inv_pass_ba<TO, SCALED>(a, c0, c1, tb, bufAB, A, re - 1, tau);
+  }
+}
+
 template <typename TI, typename TO>
 __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   extern __shared__ __align__(16) float smem[];
   __shared__ uint32_t s_tmem;
+  __shared__ __align__(8) unsigned long long s_bars[kSlots][kInvBufs];  // one per C -> B buffer
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int slot = warp >> 2, wq = warp & 3, tau = wq * 32 + lane;
-  float* bufAB = smem + slot * kSlotFloats;
-  float* bufBC = bufAB + kBufFloats;  // two buffers, used alternately
+  float* bufAB = smem + slot * kInvSlotFloats;
+  float* bufCB = bufAB + kBufFloats;  // kInvBufs buffers, rotating by row
   const long long G = static_cast<long long>(gridDim.x) * kSlots;
   const long long g = static_cast<long long>(blockIdx.x) * kSlots + slot;
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
 
   Prefetch<TI> pre;
   prefetch_c(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int i = 0; i < kSlots; ++i)
+#pragma unroll
+      for (int b = 0; b < kInvBufs; ++b) mbar_init(smem_addr(&s_bars[i][b]), kGroupThreads);
+  }
   if (warp == 0) {
     const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(&s_tmem));
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(dst) : "memory");
@@ -772,24 +938,14 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   tc_fence_after();
 
   const bool scaled = A.hdr[3] == 1.f;
+  const uint32_t bars = smem_addr(&s_bars[slot][0]);
   uint32_t c0[32], c1[32];
-  if constexpr (kDoubleBuf) {
-    tmem_ld32(tb + 32 * 11, c0);
-    tmem_wait(c0);
-  }
-  // the C -> B buffer alternates between rows (row i's readers and row i+2's
-  // writers are kept apart by row i+1's barrier)
-  if (scaled) {
-#pragma unroll 1
-    for (long long row = rb; row < re; ++row)
-      inv_row<TI, TO, true>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * kBufFloats,
-                            pre, c0, c1);
-  } else {
-#pragma unroll 1
-    for (long long row = rb; row < re; ++row)
-      inv_row<TI, TO, false>(A, row, row + 1 < re ? 1 : 0, slot, tau, tb, bufAB, bufBC + ((row - rb) & 1) * kBufFloats,
-                             pre, c0, c1);
-  }
+  tmem_ld32(tb + 32 * 11, c0);
+  tmem_wait(c0);
+  if (scaled)
+    run_inv_rows<TI, TO, true>(A, rb, re, tau, tb, bufAB, bufCB, bars, pre, c0, c1);
+  else
+    run_inv_rows<TI, TO, false>(A, rb, re, tau, tb, bufAB, bufCB, bars, pre, c0, c1);
 
   tc_fence_before();
   __syncthreads();
@@ -806,7 +962,7 @@ bq_status launch_inv(const FastArgs& A, cudaStream_t st) {
   if (cudaGetDevice(&dev) != cudaSuccess) return BQ_ERR_CUDA;
   static std::atomic<int> ready[kMaxDevices];
   if (!once_per_device(ready, dev, [&] {
-        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kFwdSmemBytes) ==
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kInvSmemBytes) ==
                cudaSuccess;
       }))
     return BQ_ERR_CUDA;
@@ -815,7 +971,7 @@ bq_status launch_inv(const FastArgs& A, cudaStream_t st) {
   long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, kFwdSmemBytes, st>>>(A);
+  kern<<<static_cast<unsigned>(grid), kThreads, kInvSmemBytes, st>>>(A);
   return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
 }
 
@@ -845,6 +1001,18 @@ bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, 
   if (xt == BQ_F32)
     return yt == BQ_F32 ? launch<float, kOutF32, 4, 16>(A, st) : launch<float, kOutBF16, 4, 16>(A, st);
   return yt == BQ_F32 ? launch<__nv_bfloat16, kOutF32, 4, 16>(A, st) : launch<__nv_bfloat16, kOutBF16, 4, 16>(A, st);
+}
+
+bq_status read_wait_faults(int32_t* value, bool clear, cudaStream_t st) {
+  int v = 0;
+  if (cudaMemcpyFromSymbolAsync(&v, g_wait_faults, sizeof(int), 0, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  static const int kZero = 0;
+  if (clear && cudaMemcpyToSymbolAsync(g_wait_faults, &kZero, sizeof(int), 0, cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return BQ_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return BQ_ERR_CUDA;
+  *value = v;
+  return BQ_OK;
 }
 
 bq_status launch_inv4096(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,

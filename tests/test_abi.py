@@ -113,6 +113,11 @@ def test_quantize_rejects_null_outputs(lib):
     assert lib.bq_transform_quantize(ctypes.byref(good), FAKE, 0, 0, 4, 128, None, None, None, None) == 0
 
 
+def test_wait_faults_rejects_null_before_any_cuda_call(lib):
+    assert lib.bq_wait_faults(None, 0, None) == _lib.BQ_ERR_INVALID_ARG
+    assert lib.bq_wait_faults(None, 1, None) == _lib.BQ_ERR_INVALID_ARG
+
+
 def test_bwd_rejects_bad_arguments(lib):
     L = (_lib.BQLayer * 2)(_layer(64, 64, 1, table=FAKE), _layer(64, 64, 1, table=FAKE))
     ws = lib.bq_butterfly_bwd_workspace_size(64, 2, 10)

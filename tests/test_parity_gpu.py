@@ -284,6 +284,25 @@ def test_full_act_4096_int4(bq):
     check_quant(bq, layer, H.dev_bf16_bits(w.x), H.input_f64(w.x, "bf16"), w.theta, 4, 128)
 
 
+def test_4096_wait_faults_stay_clear(bq):
+    """The m = 4096 forward's and inverse's bounded row-group waits never give up: after
+    launches with one to many rows per row group (every output kind) the device's
+    wait-fault word is 0."""
+    torch = H.torch()
+    bq.bq_wait_faults(clear=True)
+    w = wl.act_4096(64)
+    layer = make_layer(bq, w.theta)
+    for rows in (1, 2, 3, 443, 445, 1000):
+        rng = np.random.default_rng(rows)
+        x = torch.from_numpy(rng.standard_normal((rows, 4096)).astype(np.float32)).cuda().to(torch.bfloat16)
+        bq.bq_transform_quantize(layer, x, 4, 128, *bq.quant_outputs(rows, 4096, 4, 128, "cuda"))
+        bq.bq_butterfly_fwd(layer, x, torch.empty((rows, 4096), dtype=torch.float32, device="cuda"))
+        bq.bq_butterfly_fwd(layer, x.float(), torch.empty((rows, 4096), dtype=torch.bfloat16, device="cuda"))
+        bq.bq_butterfly_inv(layer, x, torch.empty((rows, 4096), dtype=torch.bfloat16, device="cuda"))
+        bq.bq_butterfly_inv(layer, x.float(), torch.empty((rows, 4096), dtype=torch.float32, device="cuda"))
+    assert bq.bq_wait_faults() == 0
+
+
 def test_full_weight_4096_int2(bq):
     w = wl.weight_4096()
     layer = make_layer(bq, w.theta)
