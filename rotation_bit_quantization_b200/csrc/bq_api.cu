@@ -4,6 +4,11 @@
 #include "bq_internal.cuh"
 
 namespace bq {
+
+// The wait-fault word of the m = 4096 kernels on the current device (bq_fast4096.cu,
+// the translation unit that holds the word).
+bq_status read_wait_faults(int32_t* value, bool clear, cudaStream_t st);
+
 namespace {
 
 bq_status check_rows(const void* a, const void* b, int64_t rows) {

@@ -114,8 +114,6 @@ bq_status launch_fast4096(const KLayer& L, const void* x, bq_dtype xt, void* y, 
 bool fast4096_supports(const KLayer& L, const QuantArgs* q);
 bq_status launch_inv4096(const KLayer& L, const void* y, bq_dtype yt, void* x, bq_dtype xt, int64_t rows,
                          cudaStream_t st);
-// The wait-fault word of the m = 4096 forward on the current device (see bq_wait_faults).
-bq_status read_wait_faults(int32_t* value, bool clear, cudaStream_t st);
 bq_status launch_kron1024(const KLayer& L, const void* x, bq_dtype xt, void* y, bq_dtype yt, int64_t rows,
                           const QuantArgs* q, cudaStream_t st);
 bool kron1024_supports(const KLayer& L, const QuantArgs* q);
