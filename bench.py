@@ -183,6 +183,45 @@ def gpu_id_for(device) -> str:
         return str(device.index if hasattr(device, "index") else 0)
 
 
+class GpuLocalCpus:
+    """Context manager: while it is open the process runs on the CPUs NVML reports as
+    local to the GPU, so that pinned host buffers allocated inside it sit on the GPU's
+    NUMA node (host-device copies then do not cross the inter-socket link).  The
+    previous affinity is restored on exit; without NVML it changes nothing.  `cpus` is
+    the number of CPUs used (None when unchanged)."""
+
+    def __init__(self, device):
+        self.device = device
+        self.saved = None
+        self.cpus = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            try:
+                h = pynvml.nvmlDeviceGetHandleByUUID(gpu_id_for(self.device))
+                words = pynvml.nvmlDeviceGetCpuAffinity(h, 64)
+            finally:
+                pynvml.nvmlShutdown()
+            local = {64 * i + b for i, wd in enumerate(words) for b in range(64) if (int(wd) >> b) & 1}
+            self.saved = os.sched_getaffinity(0)
+            use = local & self.saved
+            if use and use != self.saved:
+                os.sched_setaffinity(0, use)
+                self.cpus = len(use)
+            else:
+                self.saved = None
+        except Exception:
+            self.saved = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+
 def cpu_oracle_rate(w, rows_target_s: float, max_rows: int, inverse: bool = False):
     """Rows/s of the float64 oracle (transform + float32-step quantizer, or the inverse
     transform alone) on the host cores."""
@@ -448,38 +487,39 @@ def run_ours(args, spec, rank, world, local_rank):
     # end to end through the public API with host buffers: H2D input, kernel, D2H codes/scale/zero
     e2e = None
     if not args.no_e2e:
-        x_pin = x_host.pin_memory()
-        if fwd or inv:
-            outs_pin = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()]
+        with GpuLocalCpus(dev) as host_cpus:  # pinned buffers on the GPU's NUMA node
+            x_pin = x_host.pin_memory()
+            if fwd or inv:
+                outs_pin = [torch.empty(outs[0].shape, dtype=outs[0].dtype).pin_memory()]
 
-            def make_dev():
-                return torch.empty_like(x), [torch.empty_like(outs[0])]
+                def make_dev():
+                    return torch.empty_like(x), [torch.empty_like(outs[0])]
 
-            def call(xc, oc):
-                (bq.bq_butterfly_fwd if fwd else bq.bq_butterfly_inv)(layer, xc, oc[0])
-        else:
-            outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[0]]
+                def call(xc, oc):
+                    (bq.bq_butterfly_fwd if fwd else bq.bq_butterfly_inv)(layer, xc, oc[0])
+            else:
+                outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs[0]]
 
-            def make_dev():
-                return torch.empty_like(x), list(bq.quant_outputs(rows, n, bits, group, dev))
+                def make_dev():
+                    return torch.empty_like(x), list(bq.quant_outputs(rows, n, bits, group, dev))
 
-            def call(xc, oc):
-                bq.bq_transform_quantize(layer, xc, bits, group, *oc)
+                def call(xc, oc):
+                    bq.bq_transform_quantize(layer, xc, bits, group, *oc)
 
-        if world > 1:
-            dist.barrier()
-        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
-                                           args.warmup)
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e_ms = float(te.item())
-        e2e = {"value": rows * world / (e2e_ms * 1e-3), "unit": "rows/s",
-               "h2d_bytes_per_step": int(x_pin.numel() * x_pin.element_size()),
-               "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
-               "ms_per_step": e2e_ms,
-               "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
-                           f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
+            if world > 1:
+                dist.barrier()
+            e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
+                                               args.warmup)
+            te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e_ms = float(te.item())
+            e2e = {"value": rows * world / (e2e_ms * 1e-3), "unit": "rows/s", "host_cpus": host_cpus.cpus,
+                   "h2d_bytes_per_step": int(x_pin.numel() * x_pin.element_size()),
+                   "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
+                   "ms_per_step": e2e_ms,
+                   "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
+                               f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
 
     peaks, peak_src = load_peaks()
     fl_launch = flops_per_row(w.m, w.r) * rows
@@ -605,42 +645,43 @@ def run_bwd_bench(args, spec, rank, world, local_rank):
     # the launch, D2H of Y, dX and dtheta
     e2e = None
     if not args.no_e2e:
-        x1 = x[0].cpu().pin_memory()
-        dy1 = dy[0].cpu().pin_memory()
-        y1h = torch.empty(y[0].shape, dtype=y.dtype).pin_memory()
-        dx1h = torch.empty(dx[0].shape, dtype=dx.dtype).pin_memory()
-        dth1h = torch.empty(dth[0:1].shape, dtype=dth.dtype).pin_memory()
-        x1d, dy1d = torch.empty_like(x[0:1]), torch.empty_like(dy[0:1])
-        y1d, dx1d, dth1d = torch.empty_like(y[0:1]), torch.empty_like(dx[0:1]), torch.empty_like(dth[0:1])
-        ws1 = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, 1, T), dtype=torch.uint8, device=dev)
+        with GpuLocalCpus(dev) as host_cpus:  # pinned buffers on the GPU's NUMA node
+            x1 = x[0].cpu().pin_memory()
+            dy1 = dy[0].cpu().pin_memory()
+            y1h = torch.empty(y[0].shape, dtype=y.dtype).pin_memory()
+            dx1h = torch.empty(dx[0].shape, dtype=dx.dtype).pin_memory()
+            dth1h = torch.empty(dth[0:1].shape, dtype=dth.dtype).pin_memory()
+            x1d, dy1d = torch.empty_like(x[0:1]), torch.empty_like(dy[0:1])
+            y1d, dx1d, dth1d = torch.empty_like(y[0:1]), torch.empty_like(dx[0:1]), torch.empty_like(dth[0:1])
+            ws1 = torch.empty(bq.bq_butterfly_bwd_workspace_size(m, 1, T), dtype=torch.uint8, device=dev)
 
-        def e2e_step():
-            x1d[0].copy_(x1, non_blocking=True)
-            dy1d[0].copy_(dy1, non_blocking=True)
-            bq.bq_butterfly_bwd(layers[:1], x1d, y1d, dy1d, dx1d, dth1d, ws1)
-            y1h.copy_(y1d[0], non_blocking=True)
-            dx1h.copy_(dx1d[0], non_blocking=True)
-            dth1h.copy_(dth1d, non_blocking=True)
+            def e2e_step():
+                x1d[0].copy_(x1, non_blocking=True)
+                dy1d[0].copy_(dy1, non_blocking=True)
+                bq.bq_butterfly_bwd(layers[:1], x1d, y1d, dy1d, dx1d, dth1d, ws1)
+                y1h.copy_(y1d[0], non_blocking=True)
+                dx1h.copy_(dx1d[0], non_blocking=True)
+                dth1h.copy_(dth1d, non_blocking=True)
 
-        e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        n_e2e = min(args.steps, 3)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
             e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": T * world / (float(te.item()) * 1e-3), "unit": "tokens/s",
-               "h2d_bytes_per_step": x1.numel() * 2 + dy1.numel() * 4,
-               "d2h_bytes_per_step": y1h.numel() * 2 + dx1h.numel() * 4 + dth1h.numel() * 4,
-               "scope": f"one layer of the workload ({T} tokens), host buffers pinned"}
-        del x1, dy1, y1h, dx1h, x1d, dy1d, y1d, dx1d
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            n_e2e = min(args.steps, 3)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e = {"value": T * world / (float(te.item()) * 1e-3), "unit": "tokens/s", "host_cpus": host_cpus.cpus,
+                   "h2d_bytes_per_step": x1.numel() * 2 + dy1.numel() * 4,
+                   "d2h_bytes_per_step": y1h.numel() * 2 + dx1h.numel() * 4 + dth1h.numel() * 4,
+                   "scope": f"one layer of the workload ({T} tokens), host buffers pinned"}
+            del x1, dy1, y1h, dx1h, x1d, dy1d, y1d, dx1d
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, sample = cpu_bwd_rate(0, 256, m)
@@ -719,36 +760,37 @@ def run_uniformity_bench(args, spec, rank, world, local_rank):
     # dL/dY, the per-group KL and the loss
     e2e = None
     if not args.no_e2e:
-        y_pin = y.cpu().pin_memory()
-        dy_pin = torch.empty(dy.shape, dtype=dy.dtype).pin_memory()
-        kl_pin = torch.empty(kl.shape, dtype=kl.dtype).pin_memory()
-        loss_pin = torch.empty(1, dtype=torch.float32).pin_memory()
-        y_dev = torch.empty_like(y)
+        with GpuLocalCpus(dev) as host_cpus:  # pinned buffers on the GPU's NUMA node
+            y_pin = y.cpu().pin_memory()
+            dy_pin = torch.empty(dy.shape, dtype=dy.dtype).pin_memory()
+            kl_pin = torch.empty(kl.shape, dtype=kl.dtype).pin_memory()
+            loss_pin = torch.empty(1, dtype=torch.float32).pin_memory()
+            y_dev = torch.empty_like(y)
 
-        def e2e_step():
-            y_dev.copy_(y_pin, non_blocking=True)
-            bq.bq_uniformity_loss(y_dev, bits, group, 1e-4, kl, dy, loss)
-            dy_pin.copy_(dy, non_blocking=True)
-            kl_pin.copy_(kl, non_blocking=True)
-            loss_pin.copy_(loss, non_blocking=True)
+            def e2e_step():
+                y_dev.copy_(y_pin, non_blocking=True)
+                bq.bq_uniformity_loss(y_dev, bits, group, 1e-4, kl, dy, loss)
+                dy_pin.copy_(dy, non_blocking=True)
+                kl_pin.copy_(kl, non_blocking=True)
+                loss_pin.copy_(loss, non_blocking=True)
 
-        e2e_step()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        n_e2e = min(args.steps, 5)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(n_e2e):
             e2e_step()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s",
-               "h2d_bytes_per_step": y.numel() * 4, "d2h_bytes_per_step": dy.numel() * 4 + kl.numel() * 4 + 4}
-        del y_pin, dy_pin, y_dev
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            n_e2e = min(args.steps, 5)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(n_e2e):
+                e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            te = torch.tensor([e0.elapsed_time(e1) / n_e2e], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s", "host_cpus": host_cpus.cpus,
+                   "h2d_bytes_per_step": y.numel() * 4, "d2h_bytes_per_step": dy.numel() * 4 + kl.numel() * 4 + 4}
+            del y_pin, dy_pin, y_dev
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import calib as oc
@@ -859,29 +901,30 @@ def run_block_bench(args, spec, rank, world, local_rank):
 
     e2e = None
     if not args.no_e2e:
-        codes, scales = outs[0]
-        x_pin = x_host.pin_memory()
-        outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (codes, scales)]
+        with GpuLocalCpus(dev) as host_cpus:  # pinned buffers on the GPU's NUMA node
+            codes, scales = outs[0]
+            x_pin = x_host.pin_memory()
+            outs_pin = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (codes, scales)]
 
-        def make_dev():
-            return torch.empty_like(x), list(bq.block_outputs(rows, C, fmt, dev))
+            def make_dev():
+                return torch.empty_like(x), list(bq.block_outputs(rows, C, fmt, dev))
 
-        def call(xc, oc):
-            bq.bq_block_transform_quantize(bt, xc, fmt, *oc, status=status)
+            def call(xc, oc):
+                bq.bq_block_transform_quantize(bt, xc, fmt, *oc, status=status)
 
-        if world > 1:
-            dist.barrier()
-        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
-                                           args.warmup)
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s",
-               "h2d_bytes_per_step": int(x_pin.numel() * 2),
-               "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
-               "ms_per_step": float(te.item()),
-               "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
-                           f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
+            if world > 1:
+                dist.barrier()
+            e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, outs_pin, make_dev, call, args.steps,
+                                               args.warmup)
+            te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e = {"value": rows * world / (float(te.item()) * 1e-3), "unit": "rows/s", "host_cpus": host_cpus.cpus,
+                   "h2d_bytes_per_step": int(x_pin.numel() * 2),
+                   "d2h_bytes_per_step": int(sum(t.numel() * t.element_size() for t in outs_pin)),
+                   "ms_per_step": float(te.item()),
+                   "pipeline": f"{E2E_CHUNKS} row chunks per step on three streams (copy-in, the library call, "
+                               f"copy-out), two device buffer sets alternating by step; timed as {e2e_method}"}
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import blockq as obq
@@ -977,32 +1020,33 @@ def run_gemm_bench(args, spec, rank, world, local_rank):
 
     e2e = None
     if not args.no_e2e:
-        x_pin = x_host.pin_memory()
-        o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        # token chunks of the same GEMM (the weights stay on the device, as for a served layer)
-        chunk_tokens = -(-tokens // E2E_CHUNKS)
-        ws_c = torch.empty(max(256, bq.bq_w2a16_gemm_workspace_size(chunk_tokens, n, out_f)), dtype=torch.uint8,
-                           device=dev)
+        with GpuLocalCpus(dev) as host_cpus:  # pinned buffers on the GPU's NUMA node
+            x_pin = x_host.pin_memory()
+            o_pin = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+            # token chunks of the same GEMM (the weights stay on the device, as for a served layer)
+            chunk_tokens = -(-tokens // E2E_CHUNKS)
+            ws_c = torch.empty(max(256, bq.bq_w2a16_gemm_workspace_size(chunk_tokens, n, out_f)), dtype=torch.uint8,
+                               device=dev)
 
-        def make_dev():
-            return torch.empty_like(x), [torch.empty_like(out)]
+            def make_dev():
+                return torch.empty_like(x), [torch.empty_like(out)]
 
-        def call(xc, oc):
-            bq.bq_w2a16_gemm(xc, codes, scale, zero, bits, group, oc[0],
-                             workspace=ws_c if xc.shape[0] == chunk_tokens else None, status=status)
+            def call(xc, oc):
+                bq.bq_w2a16_gemm(xc, codes, scale, zero, bits, group, oc[0],
+                                 workspace=ws_c if xc.shape[0] == chunk_tokens else None, status=status)
 
-        if world > 1:
-            dist.barrier()
-        e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, [o_pin], make_dev, call, args.steps,
-                                           args.warmup)
-        te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": flops * world / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s",
-               "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
-               "ms_per_step": float(te.item()),
-               "pipeline": f"{E2E_CHUNKS} token chunks per step on three streams (copy-in, the GEMM, copy-out), "
-                           f"two device buffer sets alternating by step; timed as {e2e_method}"}
+            if world > 1:
+                dist.barrier()
+            e2e_ms, e2e_method = pipelined_e2e(torch, dev, stream, x_pin, [o_pin], make_dev, call, args.steps,
+                                               args.warmup)
+            te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+            if world > 1:
+                dist.all_reduce(te, op=dist.ReduceOp.MAX)
+            e2e = {"value": flops * world / (float(te.item()) * 1e-3) / 1e12, "unit": "TFLOP/s", "host_cpus": host_cpus.cpus,
+                   "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+                   "ms_per_step": float(te.item()),
+                   "pipeline": f"{E2E_CHUNKS} token chunks per step on three streams (copy-in, the GEMM, copy-out), "
+                               f"two device buffer sets alternating by step; timed as {e2e_method}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -52,3 +52,40 @@ def test_reference_arm_inverse():
     d = _run("--workload", "inv5120")
     _check_contract(d, "butterfly fwd+quant rows/s", "rows/s")
     assert d["config"]["n"] == 5120 and "inverse" in d["config"]["workload"]
+
+
+def _bench_module():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("bench_under_test", os.path.join(ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def test_gpu_local_cpus_sets_and_restores_affinity(monkeypatch):
+    """The e2e legs allocate pinned buffers on the CPUs NVML reports as local to the GPU
+    (a fake NVML here: the first allowed CPU) and restore the affinity afterwards."""
+    import types
+    bench = _bench_module()
+    before = os.sched_getaffinity(0)
+    if len(before) < 2:
+        pytest.skip("needs two allowed CPUs")
+    first = min(before)
+    fake = types.SimpleNamespace(
+        nvmlInit=lambda: None, nvmlShutdown=lambda: None,
+        nvmlDeviceGetHandleByUUID=lambda uuid: "handle",
+        nvmlDeviceGetCpuAffinity=lambda h, n: [(1 << (first % 64)) if i == first // 64 else 0 for i in range(n)])
+    monkeypatch.setitem(sys.modules, "pynvml", fake)
+    monkeypatch.setattr(bench, "gpu_id_for", lambda dev: "GPU-fake")
+    with bench.GpuLocalCpus(0) as loc:
+        assert os.sched_getaffinity(0) == {first} and loc.cpus == 1
+    assert os.sched_getaffinity(0) == before
+
+
+def test_gpu_local_cpus_without_nvml_changes_nothing(monkeypatch):
+    bench = _bench_module()
+    before = os.sched_getaffinity(0)
+    monkeypatch.setitem(sys.modules, "pynvml", None)  # import fails
+    with bench.GpuLocalCpus(0) as loc:
+        assert os.sched_getaffinity(0) == before and loc.cpus is None
+    assert os.sched_getaffinity(0) == before
