@@ -39,6 +39,13 @@
 //    tensor-memory image (warps w, w + 4, ... use the same lanes); each thread
 //    reads the next stage's coefficients while it computes the current one
 //    (kDoubleBuf) and the next row's input is prefetched into registers.
+//  * Programmatic dependent launch: both kernels are launched with programmatic
+//    stream serialization and let their dependents launch as soon as they start,
+//    so a launch's CTAs take SMs as the previous launch's CTAs leave them and do
+//    their set-up (mbarriers, TMEM allocation) meanwhile.  griddepcontrol.wait
+//    comes before the first global-memory access of any thread (input prefetch,
+//    coefficient image, table header, outputs), so every read sees the previous
+//    kernel's writes and no write lands before that kernel has finished reading.
 #include <cfloat>
 
 #include "bq_rtn.cuh"
@@ -160,6 +167,15 @@ __device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t parity) {
 }  // namespace
 
 __device__ int g_wait_faults = 0;
+
+// Lets the next kernel of the stream launch (if it was launched with programmatic
+// stream serialization); it still waits for this grid in its own griddep_wait.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Returns once the grids this one depends on have completed and their memory
+// operations are visible; a no-op when the launch had no programmatic dependency.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 namespace {
 
@@ -624,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
 
   Prefetch<TI> pre;
-  prefetch(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
+  griddep_launch_dependents();
 
   if (threadIdx.x == 0) {
 #pragma unroll
@@ -642,6 +658,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  griddep_wait();  // everything above touches only shared and tensor memory
+  prefetch(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
   fill_tmem<kFillChunks, kSlots, kFillRound>(A.image, tb, slot, tau);
   tc_fence_before();
   __syncthreads();
@@ -667,6 +685,24 @@ __global__ void __launch_bounds__(kThreads, 1) k_fast4096(const FastArgs A) {
   }
 }
 
+// Launches one of this file's kernels with programmatic stream serialization: it may
+// start while the previous kernel of the stream is still running, and waits for it
+// (griddep_wait) before its first global-memory access.
+template <typename K>
+bq_status launch_dependent(K kern, long long grid, int smem_bytes, const FastArgs& A, cudaStream_t st) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, A) == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+}
+
 template <typename TI, int MODE, int BITS, int GLANES>
 bq_status launch(const FastArgs& A, cudaStream_t st) {
   auto kern = k_fast4096<TI, MODE, BITS, GLANES>;
@@ -683,8 +719,7 @@ bq_status launch(const FastArgs& A, cudaStream_t st) {
   long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, kFwdSmemBytes, st>>>(A);
-  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+  return launch_dependent(kern, grid, kFwdSmemBytes, A, st);
 }
 
 template <typename TI>
@@ -916,7 +951,7 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   const long long rb = g * A.rows / G, re = (g + 1) * A.rows / G;
 
   Prefetch<TI> pre;
-  prefetch_c(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
 #pragma unroll
     for (int i = 0; i < kSlots; ++i)
@@ -932,6 +967,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_inv4096(const FastArgs A) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tb = s_tmem + (static_cast<uint32_t>(wq * 32) << 16);
+  griddep_wait();  // everything above touches only shared and tensor memory
+  prefetch_c(pre, static_cast<const TI*>(A.x), rb, re > rb ? 1 : 0, tau);
   fill_tmem<kImageInvCols / 16, kSlots, kFillRound>(A.image, tb, slot, tau);
   tc_fence_before();
   __syncthreads();
@@ -971,8 +1008,7 @@ bq_status launch_inv(const FastArgs& A, cudaStream_t st) {
   long long grid = (A.rows + kSlots - 1) / kSlots;
   if (grid > sms) grid = sms;
   if (grid < 1) grid = 1;
-  kern<<<static_cast<unsigned>(grid), kThreads, kInvSmemBytes, st>>>(A);
-  return cudaPeekAtLastError() == cudaSuccess ? BQ_OK : BQ_ERR_CUDA;
+  return launch_dependent(kern, grid, kInvSmemBytes, A, st);
 }
 
 }  // namespace

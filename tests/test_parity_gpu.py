@@ -730,6 +730,58 @@ def test_inv4096_round_trip_full_rows(bq):
     H.assert_f32_close(H.host(back), xf, xf)
 
 
+def test_4096_dependent_launch_chains(bq):
+    """The n = 4096 kernels may start while the previous kernel of the stream still runs
+    (programmatic dependent launch) and wait for it before their first global-memory
+    access. In a chain where every launch reads what the previous one wrote and
+    overwrites what the one before it read (forward a -> b, inverse b -> a, twelve
+    times, then the forward and the fused INT4 quantizer of its float32 output), the
+    results are bitwise the same with a host synchronisation after every call, back to
+    back on one stream, and replayed as one CUDA graph; the twelve round trips return x
+    within their accumulated error bound."""
+    torch = H.torch()
+    w = wl.act_4096(2048)
+    layer = make_layer(bq, w.theta)
+    xf = H.input_f64(w.x, "bf16")
+    x0 = H.dev_f32(xf)
+    trips = 12
+
+    def chain(a, b, outs, sync):
+        calls = []
+        for _ in range(trips):
+            calls += [lambda: bq.bq_butterfly_fwd(layer, a, b), lambda: bq.bq_butterfly_inv(layer, b, a)]
+        calls += [lambda: bq.bq_butterfly_fwd(layer, a, b), lambda: bq.bq_transform_quantize(layer, b, 4, 128, *outs)]
+        for call in calls:
+            call()
+            if sync:
+                torch.cuda.synchronize()
+
+    results = {}
+    bq.bq_wait_faults(clear=True)
+    for mode in ("synced", "back_to_back", "graph"):
+        a, b = x0.clone(), torch.empty_like(x0)
+        outs = bq.quant_outputs(2048, 4096, 4, 128, "cuda")
+        if mode == "graph":
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    chain(a, b, outs, False)
+            torch.cuda.current_stream().wait_stream(side)
+            a.copy_(x0)
+            g.replay()
+        else:
+            chain(a, b, outs, mode == "synced")
+        torch.cuda.synchronize()
+        results[mode] = [H.host(t) for t in (a, b, *outs)]
+    for mode in ("back_to_back", "graph"):
+        for name, ref, got in zip(("a", "b", "codes", "scale", "zero"), results["synced"], results[mode]):
+            assert np.array_equal(ref.view(np.uint8), got.view(np.uint8)), f"{mode}: {name} differs"
+    H.assert_f32_close(results["synced"][0], xf, xf, tol=2 * trips * H.F32_TOL)
+    assert bq.bq_wait_faults() == 0
+
+
 @pytest.mark.parametrize("io", ["f32", "bf16"])
 def test_kron5120_inverse_many_rows(bq, io):
     """x = (B^T (x) O^T) y on more rows than one wave of row CTAs, bf16 and float32."""
