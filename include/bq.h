@@ -16,11 +16,20 @@
  * ---------------------------------------
  *  - All data pointers are DEVICE pointers unless stated; the caller owns
  *    every buffer.  The library never allocates device memory and keeps no
- *    global state (the one exception is the fixed scratch array of
- *    bq_butterfly_bwd_noalloc); calls on different streams are independent.
+ *    global state (the exceptions are the fixed scratch array of
+ *    bq_butterfly_bwd_noalloc and the wait-fault word of bq_wait_faults);
+ *    calls on different streams are independent.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call is asynchronous on that stream; an error status is
  *    returned before anything is launched when host-side validation fails.
+ *  - The m = 4096, r = 1 kernels of bq_butterfly_fwd, bq_butterfly_inv,
+ *    bq_transform_quantize and bq_weight_rotate_pack are launched with
+ *    programmatic stream serialization: one may start its set-up while the
+ *    previous kernel on the stream is still running, and it waits for that
+ *    kernel to finish before it reads or writes any buffer, so the caller sees
+ *    plain stream order.  A kernel the caller queues next on the stream starts
+ *    early only if the caller launched it with that attribute, and must then
+ *    call cudaGridDependencySynchronize before it reads these outputs.
  *  - Rows are contiguous and row-major: element (row, i) is at row*n + i.
  *  - Element index i = i1*r + i2 with i1 < m, i2 < r; B_m acts on i1, O_r on i2.
  *  - Angle layout: theta[s*(m/2) + p] for stage s < log2(m) and pair number
