@@ -1,7 +1,7 @@
-"""Out-of-bounds write checks (the sanitizer is not available on this machine): every
-output of every entry point is allocated between two 4 KiB guard bands filled with
-a sentinel byte, the call runs on ragged shapes, and the bands must be untouched
-afterwards.  Inputs must be unchanged too."""
+"""Out-of-bounds write checks that need no memory checker: every output of every
+entry point is allocated between two 4 KiB guard bands filled with a sentinel byte,
+the call runs on ragged shapes, and the bands must be untouched afterwards.  Inputs
+must be unchanged too."""
 
 import numpy as np
 import pytest
